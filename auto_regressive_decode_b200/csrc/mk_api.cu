@@ -1,0 +1,285 @@
+// C ABI of the decode megakernel (declared in include/mk.h).
+//
+// mk_create validates the model, lowers it (mk_plan.cpp), and allocates one
+// device region holding everything the library owns.  mk_decode_step is a
+// single cooperative launch with no host synchronisation.  Errors found on the
+// device are recorded in a status word that mk_get_status reads and clears.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "mk_device.h"
+#include "mk_internal.h"
+
+namespace mk {
+int validate_desc(const mk_model_desc* d);
+int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p);
+}  // namespace mk
+
+struct mk_plan;  // defined in mk_plan.cpp
+extern "C" int mk_plan_create(const mk_model_desc*, int, mk_plan**);
+extern "C" int mk_plan_n_instrs(const mk_plan*);
+extern "C" int mk_plan_copy(const mk_plan*, mk_instr*, int32_t*);
+extern "C" int mk_plan_n_counters(const mk_plan*);
+extern "C" int mk_plan_attn_chunk(const mk_plan*, int32_t*, int32_t*);
+extern "C" int mk_plan_destroy(mk_plan*);
+
+struct mk_handle {
+  mk_model_desc d;
+  mk::Params p;
+  int n_sm;
+  int device;
+  int n_counters;
+  size_t n_tickets;
+  void* region;
+  size_t region_bytes;
+  uint32_t epoch;
+};
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+
+bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    size_t o = off;
+    off += (bytes + 255) / 256 * 256;
+    return o;
+  }
+};
+
+}  // namespace
+
+extern "C" const char* mk_status_string(int s) {
+  switch (s) {
+    case MK_OK: return "ok";
+    case MK_ERR_INVALID_ARG: return "invalid argument";
+    case MK_ERR_UNSUPPORTED: return "unsupported shape, alignment or device";
+    case MK_ERR_CUDA: return "CUDA runtime error";
+    case MK_ERR_DEVICE_TIMEOUT: return "in-kernel wait timed out";
+    case MK_ERR_RANGE: return "token, position or sequence length out of range";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const mk_kv* kv, mk_handle** out) {
+  if (!out) return MK_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!desc || !w || !kv || !w->layers) return MK_ERR_INVALID_ARG;
+  int rc = mk::validate_desc(desc);
+  if (rc) return rc;
+  const mk_model_desc& d = *desc;
+  // pointers: present and 16-byte aligned
+  if (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(kv->k) || !aligned16(kv->v))
+    return w->embed && w->final_norm && kv->k && kv->v ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
+  if (!d.tied_embeddings && !aligned16(w->lm_head)) return w->lm_head ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
+  for (int l = 0; l < d.n_layers; ++l) {
+    const mk_layer_weights& lw = w->layers[l];
+    const void* need[] = {lw.attn_norm, lw.wq, lw.wk, lw.wv, lw.wo, lw.mlp_norm, lw.w_gate, lw.w_up, lw.w_down};
+    for (const void* q : need)
+      if (!aligned16(q)) return q ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
+    if (d.qk_norm && (!aligned16(lw.q_norm) || !aligned16(lw.k_norm))) return MK_ERR_INVALID_ARG;
+  }
+
+  int dev = 0, n_sm = 0, coop = 0, smem_optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MK_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MK_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) return MK_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return MK_ERR_CUDA;
+  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes()) return MK_ERR_UNSUPPORTED;
+  if (mk::kernel_prepare() != cudaSuccess) return MK_ERR_CUDA;
+  int per_sm = 0;
+  if (mk::kernel_occupancy(&per_sm) != cudaSuccess) return MK_ERR_CUDA;
+  if (per_sm < 1) return MK_ERR_UNSUPPORTED;
+
+  mk_plan* plan = nullptr;
+  rc = mk_plan_create(desc, n_sm, &plan);
+  if (rc) return rc;
+  const int n_instr = mk_plan_n_instrs(plan);
+  std::vector<mk_instr> instrs(n_instr > 0 ? n_instr : 1);
+  std::vector<int32_t> offsets(n_sm + 1);
+  mk_plan_copy(plan, instrs.data(), offsets.data());
+  const int n_cnt = mk_plan_n_counters(plan);
+  int32_t chunk = 0, n_chunks = 0;
+  mk_plan_attn_chunk(plan, &chunk, &n_chunks);
+  mk_plan_destroy(plan);
+
+  mk_handle* h = new (std::nothrow) mk_handle();
+  if (!h) return MK_ERR_INVALID_ARG;
+  h->d = d;
+  h->n_sm = n_sm;
+  h->device = dev;
+  h->n_counters = n_cnt;
+  h->epoch = 0;
+  const int L = d.n_layers, B = d.batch, H = d.hidden, hd = d.head_dim, nq = d.n_q_heads, nkv = d.n_kv_heads;
+  const size_t qd = (size_t)nq * hd, kvd = (size_t)nkv * hd;
+  h->n_tickets = (size_t)L * B * nkv;
+
+  Carve cv;
+  const size_t o_xres = cv.take(sizeof(float) * (size_t)(2 * L + 1) * B * H);
+  const size_t o_qkv = cv.take(sizeof(float) * (size_t)B * (qd + 2 * kvd));
+  const size_t o_attn = cv.take(sizeof(float) * (size_t)B * qd);
+  const size_t o_act = cv.take(sizeof(float) * (size_t)B * d.ffn_dim);
+  const size_t o_po = cv.take(sizeof(float) * (size_t)B * nq * n_chunks * hd);
+  const size_t o_pml = cv.take(sizeof(float) * (size_t)B * nq * n_chunks * 2);
+  const size_t o_cnt = cv.take(sizeof(uint32_t) * (size_t)n_cnt);
+  const size_t o_tk = cv.take(sizeof(uint32_t) * h->n_tickets);
+  const size_t o_st = cv.take(sizeof(int) * 4);
+  const size_t o_ins = cv.take(sizeof(mk_instr) * instrs.size());
+  const size_t o_off = cv.take(sizeof(int32_t) * offsets.size());
+  const size_t o_lay = cv.take(sizeof(mk::LayerPtrs) * (size_t)L);
+  const size_t o_rope = cv.take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
+  h->region_bytes = cv.off;
+  if (cudaMalloc(&h->region, h->region_bytes) != cudaSuccess) {
+    delete h;
+    return MK_ERR_CUDA;
+  }
+  uint8_t* base = static_cast<uint8_t*>(h->region);
+
+  std::vector<mk::LayerPtrs> lp(L);
+  for (int l = 0; l < L; ++l) {
+    const mk_layer_weights& s = w->layers[l];
+    mk::LayerPtrs& t = lp[l];
+    t.attn_norm = (const uint16_t*)s.attn_norm;
+    t.wq = (const uint16_t*)s.wq;
+    t.wk = (const uint16_t*)s.wk;
+    t.wv = (const uint16_t*)s.wv;
+    t.q_norm = (const uint16_t*)s.q_norm;
+    t.k_norm = (const uint16_t*)s.k_norm;
+    t.wo = (const uint16_t*)s.wo;
+    t.mlp_norm = (const uint16_t*)s.mlp_norm;
+    t.w_gate = (const uint16_t*)s.w_gate;
+    t.w_up = (const uint16_t*)s.w_up;
+    t.w_down = (const uint16_t*)s.w_down;
+    t.router = (const uint16_t*)s.router;
+  }
+  // RoPE table: angle pos * theta^(-2i/hd) in double, stored as fp32 (cos, sin)
+  std::vector<float2> rope((size_t)d.max_ctx * (hd / 2));
+  for (int pos = 0; pos < d.max_ctx; ++pos)
+    for (int i = 0; i < hd / 2; ++i) {
+      const double ang = (double)pos * pow((double)d.rope_theta, -2.0 * i / hd);
+      rope[(size_t)pos * (hd / 2) + i] = make_float2((float)cos(ang), (float)sin(ang));
+    }
+
+  bool ok = cudaMemset(base, 0, h->region_bytes) == cudaSuccess &&
+            cudaMemcpy(base + o_ins, instrs.data(), sizeof(mk_instr) * instrs.size(), cudaMemcpyHostToDevice) ==
+                cudaSuccess &&
+            cudaMemcpy(base + o_off, offsets.data(), sizeof(int32_t) * offsets.size(), cudaMemcpyHostToDevice) ==
+                cudaSuccess &&
+            cudaMemcpy(base + o_lay, lp.data(), sizeof(mk::LayerPtrs) * L, cudaMemcpyHostToDevice) == cudaSuccess &&
+            cudaMemcpy(base + o_rope, rope.data(), sizeof(float2) * rope.size(), cudaMemcpyHostToDevice) ==
+                cudaSuccess;
+  if (!ok) {
+    cudaFree(h->region);
+    delete h;
+    return MK_ERR_CUDA;
+  }
+
+  mk::Params& p = h->p;
+  memset(&p, 0, sizeof(p));
+  p.L = L;
+  p.H = H;
+  p.nq = nq;
+  p.nkv = nkv;
+  p.hd = hd;
+  p.I = d.ffn_dim;
+  p.V = d.vocab;
+  p.B = B;
+  p.T = d.max_ctx;
+  p.qk_norm = d.qk_norm;
+  p.eps = d.rms_eps;
+  p.chunk = chunk;
+  p.n_chunks = n_chunks;
+  p.embed = (const uint16_t*)w->embed;
+  p.final_norm = (const uint16_t*)w->final_norm;
+  p.lm_head = (const uint16_t*)(d.tied_embeddings ? w->embed : w->lm_head);
+  p.layers = (const mk::LayerPtrs*)(base + o_lay);
+  p.kc = (uint16_t*)kv->k;
+  p.vc = (uint16_t*)kv->v;
+  p.rope = (const float2*)(base + o_rope);
+  p.xres = (float*)(base + o_xres);
+  p.qkv = (float*)(base + o_qkv);
+  p.attn = (float*)(base + o_attn);
+  p.act = (float*)(base + o_act);
+  p.part_o = (float*)(base + o_po);
+  p.part_ml = (float*)(base + o_pml);
+  p.counters = (uint32_t*)(base + o_cnt);
+  p.tickets = (uint32_t*)(base + o_tk);
+  p.status = (int*)(base + o_st);
+  p.instrs = (const mk_instr*)(base + o_ins);
+  p.offsets = (const int32_t*)(base + o_off);
+  p.timeout_ns = d.wait_timeout_ns ? d.wait_timeout_ns : kDefaultTimeoutNs;
+  *out = h;
+  return MK_OK;
+}
+
+extern "C" int mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions, const int32_t* seq_lens,
+                              void* stream, float* out_logits) {
+  if (!h || !tokens || !positions || !seq_lens || !out_logits) return MK_ERR_INVALID_ARG;
+  mk::Params p = h->p;
+  p.tokens = tokens;
+  p.positions = positions;
+  p.seq_lens = seq_lens;
+  p.logits = out_logits;
+  p.epoch = h->epoch + 1;
+  cudaError_t e = mk::launch_step(p, h->n_sm, (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  h->epoch = p.epoch;
+  return MK_OK;
+}
+
+extern "C" int mk_get_status(mk_handle* h, void* stream) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  int st[4] = {0, 0, 0, 0};
+  if (cudaMemcpyAsync(st, h->p.status, sizeof(st), cudaMemcpyDeviceToHost, (cudaStream_t)stream) != cudaSuccess ||
+      cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+    return MK_ERR_CUDA;
+  if (st[0] != 0) {
+    // the abandoned step left counters part-way: start again from epoch 0
+    if (cudaMemsetAsync(h->p.counters, 0, sizeof(uint32_t) * h->n_counters, (cudaStream_t)stream) != cudaSuccess ||
+        cudaMemsetAsync(h->p.tickets, 0, sizeof(uint32_t) * h->n_tickets, (cudaStream_t)stream) != cudaSuccess ||
+        cudaMemsetAsync(h->p.status, 0, sizeof(int) * 4, (cudaStream_t)stream) != cudaSuccess ||
+        cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+      return MK_ERR_CUDA;
+    h->epoch = 0;
+  }
+  return st[0];
+}
+
+extern "C" int mk_destroy(mk_handle* h) {
+  if (!h) return MK_OK;
+  cudaError_t e = cudaFree(h->region);
+  delete h;
+  return e == cudaSuccess ? MK_OK : MK_ERR_CUDA;
+}
+
+extern "C" size_t mk_state_bytes(const mk_handle* h, int which) {
+  if (!h) return 0;
+  const mk_model_desc& d = h->d;
+  switch (which) {
+    case MK_STATE_HIDDEN: return sizeof(float) * (size_t)(2 * d.n_layers + 1) * d.batch * d.hidden;
+    default: return 0;
+  }
+}
+
+extern "C" int mk_read_state(mk_handle* h, int which, void* dst, size_t bytes, void* stream) {
+  if (!h || !dst) return MK_ERR_INVALID_ARG;
+  const size_t need = mk_state_bytes(h, which);
+  if (need == 0) return MK_ERR_INVALID_ARG;
+  if (bytes < need) return MK_ERR_INVALID_ARG;
+  const void* src = nullptr;
+  if (which == MK_STATE_HIDDEN) src = h->p.xres;
+  if (cudaMemcpyAsync(dst, src, need, cudaMemcpyDefault, (cudaStream_t)stream) != cudaSuccess) return MK_ERR_CUDA;
+  return MK_OK;
+}

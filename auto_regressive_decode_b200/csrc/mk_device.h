@@ -1,0 +1,56 @@
+// Kernel parameters shared by the C ABI (host) and the persistent kernel.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mk_internal.h"
+
+namespace mk {
+
+struct LayerPtrs {
+  const uint16_t *attn_norm, *wq, *wk, *wv, *q_norm, *k_norm, *wo, *mlp_norm;
+  const uint16_t *w_gate, *w_up, *w_down, *router;
+};
+
+struct Params {
+  // shape
+  int L, H, nq, nkv, hd, I, V, B, T, qk_norm;
+  float eps;
+  int chunk, n_chunks;
+  // weights (device)
+  const uint16_t* embed;
+  const uint16_t* final_norm;
+  const uint16_t* lm_head;
+  const LayerPtrs* layers;  // [L]
+  uint16_t* kc;             // [L][B][nkv][T][hd]
+  uint16_t* vc;
+  const float2* rope;       // [T][hd/2] (cos, sin)
+  // library scratch (device)
+  float* xres;              // [2L+1][B][H]
+  float* qkv;               // [B][nq*hd + 2*nkv*hd]
+  float* attn;              // [B][nq*hd]
+  float* act;               // [B][I]
+  float* part_o;            // [B][nq][n_chunks][hd]
+  float* part_ml;           // [B][nq][n_chunks][2]
+  uint32_t* counters;       // [n_counters]
+  uint32_t* tickets;        // [L][B][nkv]
+  const mk_instr* instrs;
+  const int32_t* offsets;   // [n_sm + 1]
+  int* status;              // [0] code, [1] detail, [2] block
+  // per step
+  const int32_t* tokens;
+  const int32_t* positions;
+  const int32_t* seq_lens;
+  float* logits;            // [B][V]
+  uint32_t epoch;
+  uint64_t timeout_ns;
+};
+
+// Dynamic shared memory of one CTA.
+size_t kernel_smem_bytes();
+cudaError_t kernel_prepare();  // set the function's shared-memory limit
+cudaError_t kernel_occupancy(int* blocks_per_sm);
+cudaError_t launch_step(const Params& p, int n_blocks, cudaStream_t stream);
+
+}  // namespace mk

@@ -1,0 +1,96 @@
+// Internal definitions shared by the host scheduler (mk_plan.cpp), the C ABI
+// (mk_api.cu) and the persistent kernel (mk_kernel.cu).
+#pragma once
+
+#include <stdint.h>
+
+#include "../../include/mk.h"
+
+#if defined(__CUDACC__)
+#define MK_HD __host__ __device__ __forceinline__
+#else
+#define MK_HD inline
+#endif
+
+namespace mk {
+
+// ---- instruction ops (low 8 bits of mk_instr::op_layer) --------------------
+enum Op : int32_t {
+  OP_NOP = 0,
+  OP_EMBED = 1,    // a,b: hidden slice [a,b) of x0 = embed[token]
+  OP_QKV = 2,      // a,b: rows of matrix c (0 wq, 1 wk, 2 wv); RMSNorm(x_{2l}) prologue
+  OP_ATTN = 3,     // a: sequence, b: kv head, c: chunk; last chunk of (a,b) merges
+  OP_OPROJ = 4,    // a,b: rows of wo; x_{2l+1} = x_{2l} + wo . attn
+  OP_GATEUP = 5,   // a,b: rows of w_gate/w_up; act = silu(g) * u; RMSNorm(x_{2l+1}) prologue
+  OP_DOWN = 6,     // a,b: rows of w_down; x_{2l+2} = x_{2l+1} + w_down . act
+  OP_LMHEAD = 7,   // a,b: vocabulary rows; RMSNorm(x_{2L}) prologue
+  OP_ROUTER = 8,   // a: sequence; router logits, top-k, expert list (MoE)
+  OP_EXP_GATEUP = 9,  // a,b: rows of every used expert's gate/up (MoE)
+  OP_EXP_DOWN = 10,   // a,b: rows of every used expert's down + weighted combine (MoE)
+};
+
+MK_HD int op_of(int32_t op_layer) { return op_layer & 0xFF; }
+MK_HD int layer_of(int32_t op_layer) { return op_layer >> 8; }
+
+// ---- pipeline geometry -----------------------------------------------------
+constexpr int kConsumerWarps = 8;                      // compute warps
+constexpr int kConsumerThreads = kConsumerWarps * 32;  // 256
+constexpr int kThreads = kConsumerThreads + 32;        // + one producer warp
+constexpr int kStageBytes = 32 * 1024;                 // one ring slot
+constexpr int kStages = 6;                             // ring depth (192 KB)
+constexpr int kMaxRows = 256;                          // rows per GEMV instruction
+constexpr int kRedFloats = 4096;                       // cross-warp reduction buffer
+constexpr int kMaxBatch = 8;
+constexpr int kMaxGroup = 8;                           // query heads per KV head
+constexpr int kMaxHeadDim = 128;
+
+// ---- dependency counters -----------------------------------------------------
+// Each counter is bumped once per producing instruction per step; a waiter
+// needs epoch * producers.  Per layer: QKV, ATTN (one per merged (seq, kv head)),
+// OPROJ, GATEUP / ROUTER, DOWN / EXP_GATEUP, EXP_DOWN.
+enum CounterSlot : int32_t {
+  C_QKV = 0,
+  C_ATTN = 1,
+  C_OPROJ = 2,
+  C_GATEUP = 3,
+  C_DOWN = 4,
+  C_ROUTER = 5,
+  C_EXP_GATEUP = 6,
+  C_EXP_DOWN = 7,
+  C_PER_LAYER = 8
+};
+inline int counter_index(int layer, int slot) { return layer * C_PER_LAYER + slot; }
+// global counters after the per-layer block
+inline int counter_embed(int n_layers) { return n_layers * C_PER_LAYER; }
+inline int counter_lmhead(int n_layers) { return n_layers * C_PER_LAYER + 1; }
+inline int n_counters(int n_layers) { return n_layers * C_PER_LAYER + 2; }
+
+// ---- GEMV tiling (host and device agree on it) -------------------------------
+// A GEMV instruction streams full rows of K bf16.  The 256 consumer threads
+// split each row over `tpr` threads (16-byte vectors, round-robin), so rpp =
+// 256 / tpr rows are in flight at once and each thread keeps nv = ceil(K/8/tpr)
+// input vectors of 8 floats in registers for the whole instruction.
+struct GemvTile {
+  int tpr, rpp, nv, rows_per_stage;
+};
+
+MK_HD GemvTile gemv_tile(int K, int n_mats) {
+  GemvTile t;
+  int vt = K / 8;
+  int tpr = 32;
+  while (tpr < vt && tpr < kConsumerThreads) tpr *= 2;
+  t.tpr = tpr;
+  t.rpp = kConsumerThreads / tpr;
+  t.nv = (vt + tpr - 1) / tpr;
+  int r = kStageBytes / (K * 2 * n_mats);
+  int cap = 8 * t.rpp;  // at most 8 rows per thread per stage
+  if (r > cap) r = cap;
+  t.rows_per_stage = r;
+  return t;
+}
+
+// ---- attention split -------------------------------------------------------------
+// Positions of K (or V) that fit one ring slot.
+MK_HD int attn_stage_positions(int head_dim) { return kStageBytes / (head_dim * 2); }
+
+}  // namespace mk

@@ -1,0 +1,949 @@
+// The persistent decode-step kernel for sm_100a.
+//
+// One CTA per SM, launched cooperatively so that every CTA is resident.  Each
+// CTA walks its own instruction list (built by mk_plan.cpp) with two roles:
+//
+//  * warp 8, the producer: streams the bytes every instruction reads from
+//    HBM and never changes during a step -- weight rows and the KV-cache
+//    positions cached by earlier steps -- into a 6-slot x 32 KB shared-memory
+//    ring with 1-D bulk copies (cp.async.bulk, completion on an mbarrier,
+//    L2 evict-first).  It runs ahead of the compute across instruction and
+//    layer boundaries, so weight streaming continues while the consumers wait
+//    on a dependency.
+//  * warps 0-7, the consumers: wait on the dependency counter of each
+//    instruction (bounded spin on an acquire load), compute from the ring
+//    (GEMV with a fused RMSNorm prologue and residual / SwiGLU epilogue,
+//    split-K attention with an online softmax), write fp32 activations with
+//    generic stores, then bump the instruction's counter with a release add.
+//
+// ForgeMegakernel (arXiv 2609.12379, abstract) gives the properties followed:
+// a per-SM instruction stream and dependency counters replacing global
+// synchronisation; the page names no data layout, tile shape or instruction
+// format, so those below are this library's own.
+//
+// Failure handling: every wait is bounded by Params::timeout_ns.  A CTA that
+// gives up records MK_ERR_DEVICE_TIMEOUT in the status word and every other
+// CTA leaves at its next counter wait; the producer waits for its own copies
+// in flight before leaving.  Nothing traps.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mk_device.h"
+
+namespace mk {
+
+// ---------------------------------------------------------------------------
+// shared memory layout
+// ---------------------------------------------------------------------------
+struct Ctl {
+  unsigned long long full[kStages];
+  unsigned long long empty[kStages];
+  int dead;       // this CTA gives up: every wait returns at once
+  int last;       // attention: this CTA merges (broadcast)
+  int flag;       // generic broadcast
+  float sred[kConsumerWarps * 2];
+  float qs[kMaxGroup * kMaxHeadDim];
+  float knew[kMaxHeadDim];
+  float vnew[kMaxHeadDim];
+};
+
+constexpr size_t kRingBytes = (size_t)kStages * kStageBytes;
+constexpr size_t kRedBytes = (size_t)kRedFloats * sizeof(float);
+constexpr size_t kSmemBytes = kRingBytes + kRedBytes + sizeof(Ctl);
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar,
+                                         uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ int ld_relaxed_i32(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Named barrier 1 over the 256 consumer threads, OR-reducing a predicate.
+__device__ __forceinline__ bool consumer_bar_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+__device__ __forceinline__ void unpack8(const uint4 w, float f[8]) {
+  f[0] = bf16_lo(w.x); f[1] = bf16_hi(w.x);
+  f[2] = bf16_lo(w.y); f[3] = bf16_hi(w.y);
+  f[4] = bf16_lo(w.z); f[5] = bf16_hi(w.z);
+  f[6] = bf16_lo(w.w); f[7] = bf16_hi(w.w);
+}
+
+__device__ __forceinline__ float dot8(const uint4 w, const float x[8], float acc) {
+  acc = fmaf(bf16_lo(w.x), x[0], acc);
+  acc = fmaf(bf16_hi(w.x), x[1], acc);
+  acc = fmaf(bf16_lo(w.y), x[2], acc);
+  acc = fmaf(bf16_hi(w.y), x[3], acc);
+  acc = fmaf(bf16_lo(w.z), x[4], acc);
+  acc = fmaf(bf16_hi(w.z), x[5], acc);
+  acc = fmaf(bf16_lo(w.w), x[6], acc);
+  acc = fmaf(bf16_hi(w.w), x[7], acc);
+  return acc;
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+
+__device__ void set_status(const Params& p, int code, int detail) {
+  if (atomicCAS(p.status, 0, code) == 0) {
+    p.status[1] = detail;
+    p.status[2] = blockIdx.x;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Instruction geometry (identical on the producer and consumer side)
+// ---------------------------------------------------------------------------
+struct Gemv {
+  const uint16_t* w0;  // first matrix, row 0
+  const uint16_t* w1;  // second matrix (gate/up pair) or nullptr
+  int K, r0, r1;
+  GemvTile tile;
+};
+
+__device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, int op, int layer) {
+  Gemv g;
+  g.w1 = nullptr;
+  g.r0 = in.a;
+  g.r1 = in.b;
+  if (op == OP_LMHEAD) {
+    g.w0 = p.lm_head;
+    g.K = p.H;
+  } else {
+    const LayerPtrs& lp = p.layers[layer];
+    switch (op) {
+      case OP_QKV:
+        g.w0 = in.c == 0 ? lp.wq : (in.c == 1 ? lp.wk : lp.wv);
+        g.K = p.H;
+        break;
+      case OP_OPROJ:
+        g.w0 = lp.wo;
+        g.K = p.nq * p.hd;
+        break;
+      case OP_GATEUP:
+        g.w0 = lp.w_gate;
+        g.w1 = lp.w_up;
+        g.K = p.H;
+        break;
+      default:  // OP_DOWN
+        g.w0 = lp.w_down;
+        g.K = p.I;
+        break;
+    }
+  }
+  g.tile = gemv_tile(g.K, g.w1 ? 2 : 1);
+  return g;
+}
+
+struct Attn {
+  int b, kvh, c, S, p0, n_cached, nsub, P;
+  bool active, owns_new;
+  size_t cache_base;  // element offset of (layer, b, kvh, position p0)
+};
+
+__device__ __forceinline__ Attn attn_geo(const Params& p, const mk_instr& in, int layer, int head_dim) {
+  Attn a;
+  a.b = in.a;
+  a.kvh = in.b;
+  a.c = in.c;
+  a.S = p.seq_lens[a.b];
+  a.p0 = a.c * p.chunk;
+  const int p1 = min(a.p0 + p.chunk, p.T);
+  a.active = a.p0 <= a.S;
+  a.owns_new = a.active && a.S < p1;
+  a.n_cached = max(0, min(p1, a.S) - a.p0);
+  a.P = attn_stage_positions(head_dim);
+  a.nsub = (a.n_cached + a.P - 1) / a.P;
+  a.cache_base = ((((size_t)layer * p.B + a.b) * p.nkv + a.kvh) * p.T + a.p0) * head_dim;
+  return a;
+}
+
+// ---------------------------------------------------------------------------
+// Producer warp (lane 0 issues everything)
+// ---------------------------------------------------------------------------
+struct Producer {
+  const Params& p;
+  Ctl* ctl;
+  uint8_t* ring;
+  uint64_t pol;
+  uint32_t k = 0;  // stages issued
+
+  __device__ Producer(const Params& pp, Ctl* c, uint8_t* r) : p(pp), ctl(c), ring(r) { pol = evict_first_policy(); }
+
+  // Claim the next slot (waiting until the consumers released it).
+  __device__ bool claim(uint8_t** dst, unsigned long long** bar) {
+    const int slot = k % kStages;
+    if (k >= (uint32_t)kStages) {
+      const uint32_t parity = ((k / kStages) - 1) & 1;
+      if (!mbar_try_wait(&ctl->empty[slot], parity)) {
+        const uint64_t t0 = globaltimer();
+        uint32_t spins = 0;
+        while (!mbar_try_wait(&ctl->empty[slot], parity)) {
+          if (*(volatile int*)&ctl->dead) return false;
+          if ((++spins & 63) == 0) {
+            if (ld_relaxed_i32(p.status) != 0) return false;
+            if (globaltimer() - t0 > p.timeout_ns) {
+              set_status(p, MK_ERR_DEVICE_TIMEOUT, -1);
+              return false;
+            }
+          }
+        }
+      }
+    }
+    *dst = ring + (size_t)slot * kStageBytes;
+    *bar = &ctl->full[slot];
+    return true;
+  }
+
+  __device__ bool gemv(const Gemv& g) {
+    const int R = g.tile.rows_per_stage;
+    const uint32_t row_bytes = (uint32_t)g.K * 2u;
+    for (int r = g.r0; r < g.r1; r += R) {
+      const int n = min(R, g.r1 - r);
+      uint8_t* dst;
+      unsigned long long* bar;
+      if (!claim(&dst, &bar)) return false;
+      const uint32_t bytes = (uint32_t)n * row_bytes;
+      mbar_arrive_expect_tx(bar, g.w1 ? 2 * bytes : bytes);
+      bulk_g2s(dst, g.w0 + (size_t)r * g.K, bytes, bar, pol);
+      if (g.w1) bulk_g2s(dst + (size_t)R * row_bytes, g.w1 + (size_t)r * g.K, bytes, bar, pol);
+      ++k;
+    }
+    return true;
+  }
+
+  __device__ bool attn(const Attn& a, int hd) {
+    for (int s = 0; s < a.nsub; ++s) {
+      const int np = min(a.P, a.n_cached - s * a.P);
+      const uint32_t bytes = (uint32_t)np * hd * 2u;
+      const size_t off = a.cache_base + (size_t)s * a.P * hd;
+      for (int kv = 0; kv < 2; ++kv) {
+        uint8_t* dst;
+        unsigned long long* bar;
+        if (!claim(&dst, &bar)) return false;
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(dst, (kv == 0 ? p.kc : p.vc) + off, bytes, bar, pol);
+        ++k;
+      }
+    }
+    return true;
+  }
+
+  // After giving up: wait (bounded) for the copies still in flight.
+  __device__ void drain() {
+    const uint32_t first = k > (uint32_t)kStages ? k - kStages : 0;
+    for (uint32_t j = first; j < k; ++j) {
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&ctl->full[j % kStages], (j / kStages) & 1)) {
+        if (globaltimer() - t0 > p.timeout_ns) break;
+      }
+    }
+  }
+};
+
+__device__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
+  Producer pr(p, ctl, ring);
+  bool ok = true;
+  for (int i = 0; i < n && ok; ++i) {
+    const mk_instr in = list[i];
+    const int op = op_of(in.op_layer), layer = layer_of(in.op_layer);
+    switch (op) {
+      case OP_QKV:
+      case OP_OPROJ:
+      case OP_GATEUP:
+      case OP_DOWN:
+      case OP_LMHEAD:
+        ok = pr.gemv(gemv_geo(p, in, op, layer));
+        break;
+      case OP_ATTN:
+        ok = pr.attn(attn_geo(p, in, layer, p.hd), p.hd);
+        break;
+      default:
+        break;
+    }
+  }
+  if (!ok) {
+    ctl->dead = 1;
+    pr.drain();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Consumer warps
+// ---------------------------------------------------------------------------
+struct Consumer {
+  const Params& p;
+  Ctl* ctl;
+  uint8_t* ring;
+  float* red;
+  uint32_t k = 0;  // stages consumed
+  const int t = threadIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  __device__ Consumer(const Params& pp, Ctl* c, uint8_t* r, float* rd) : p(pp), ctl(c), ring(r), red(rd) {}
+
+  // Wait until slot k holds its data.  Never changes control flow: on a
+  // timeout it marks the CTA dead and returns, and the caller carries on
+  // until the next uniform decision point.
+  __device__ const uint8_t* wait_full() { return wait_stage(k); }
+
+  __device__ const uint8_t* wait_stage(uint32_t kk) {
+    const int slot = kk % kStages;
+    const uint32_t parity = (kk / kStages) & 1;
+    if (!mbar_try_wait(&ctl->full[slot], parity)) {
+      const uint64_t t0 = globaltimer();
+      uint32_t spins = 0;
+      while (!mbar_try_wait(&ctl->full[slot], parity)) {
+        if (*(volatile int*)&ctl->dead) break;
+        if ((++spins & 63) == 0 && globaltimer() - t0 > p.timeout_ns) {
+          set_status(p, MK_ERR_DEVICE_TIMEOUT, -2);
+          ctl->dead = 1;
+          break;
+        }
+      }
+    }
+    return ring + (size_t)slot * kStageBytes;
+  }
+
+  __device__ void release() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->empty[k % kStages]);
+    ++k;
+  }
+
+  // Dependency wait on `idx` reaching epoch * count.  Uniform result.
+  __device__ bool wait_counter(int idx, int count) {
+    bool fail = false;
+    if (idx >= 0 && t == 0) {
+      const uint32_t target = p.epoch * (uint32_t)count;
+      const uint32_t* c = p.counters + idx;
+      if ((int32_t)(ld_acquire(c) - target) < 0) {
+        const uint64_t t0 = globaltimer();
+        while (true) {
+          if ((int32_t)(ld_acquire(c) - target) >= 0) break;
+          if (ld_relaxed_i32(p.status) != 0 || *(volatile int*)&ctl->dead) {
+            fail = true;
+            break;
+          }
+          if (globaltimer() - t0 > p.timeout_ns) {
+            set_status(p, MK_ERR_DEVICE_TIMEOUT, idx);
+            fail = true;
+            break;
+          }
+          __nanosleep(40);
+        }
+      }
+    }
+    if (t == 0 && *(volatile int*)&ctl->dead) fail = true;
+    return !consumer_bar_or(fail);
+  }
+
+  __device__ void signal(int idx) {
+    consumer_bar();
+    if (t == 0 && idx >= 0) {
+      __threadfence();
+      red_release_add(p.counters + idx, 1u);
+    }
+  }
+
+  // Block-wide sum over the 256 consumer threads (result in every thread).
+  __device__ float block_sum(float v) {
+    v = warp_sum(v);
+    consumer_bar();
+    if (lane == 0) ctl->sred[warp] = v;
+    consumer_bar();
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) s += ctl->sred[w];
+    return s;
+  }
+
+  // ---- embedding ------------------------------------------------------------
+  __device__ void embed(const mk_instr& in) {
+    for (int b = 0; b < p.B; ++b) {
+      const uint16_t* row = p.embed + (size_t)p.tokens[b] * p.H;
+      float* x = p.xres + (size_t)b * p.H;
+      for (int i = in.a + t; i < in.b; i += kConsumerThreads) x[i] = bf16_bits_to_f32(row[i]);
+    }
+  }
+
+  // ---- GEMV ------------------------------------------------------------------
+  // Input vector x (fp32, written by other CTAs) optionally RMS-normalised
+  // with a bf16 gain; each thread keeps its NVT vectors in registers.
+  template <int NVT>
+  __device__ __forceinline__ void load_x(const float* src, const uint16_t* gain, int K, const GemvTile& tl, float xr[NVT][8]) {
+    float scale = 1.f;
+    if (gain) {
+      float ss = 0.f;
+      for (int i = t; i < K / 4; i += kConsumerThreads) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src) + i);
+        ss = fmaf(v.x, v.x, ss);
+        ss = fmaf(v.y, v.y, ss);
+        ss = fmaf(v.z, v.z, ss);
+        ss = fmaf(v.w, v.w, ss);
+      }
+      ss = block_sum(ss);
+      scale = 1.f / sqrtf(ss / (float)K + p.eps);
+    }
+    const int ct = t % tl.tpr, vt = K / 8;
+#pragma unroll
+    for (int j = 0; j < NVT; ++j) {
+      const int v = ct + j * tl.tpr;
+      if (v < vt) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(src + v * 8));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(src + v * 8) + 1);
+        xr[j][0] = a.x; xr[j][1] = a.y; xr[j][2] = a.z; xr[j][3] = a.w;
+        xr[j][4] = b.x; xr[j][5] = b.y; xr[j][6] = b.z; xr[j][7] = b.w;
+        if (gain) {
+          float g[8];
+          unpack8(__ldg(reinterpret_cast<const uint4*>(gain + v * 8)), g);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xr[j][e] = xr[j][e] * scale * g[e];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
+      }
+    }
+  }
+
+  // Stream the instruction's stages, leaving per-(row, warp) partial dots in red.
+  template <int NVT, bool GATED>
+  __device__ __forceinline__ void gemv_stream(const Gemv& g, const float xr[NVT][8]) {
+    const GemvTile& tl = g.tile;
+    const int R = tl.rows_per_stage, K = g.K, vt = K / 8;
+    const int rs = t / tl.tpr, ct = t % tl.tpr, wpr = tl.tpr / 32, wir = ct / 32;
+    const int nm = GATED ? 2 : 1;
+    for (int r = g.r0; r < g.r1; r += R) {
+      const int n = min(R, g.r1 - r);
+      const uint16_t* w0 = reinterpret_cast<const uint16_t*>(wait_full());
+      const uint16_t* w1 = w0 + (size_t)R * K;
+      for (int i = rs; i < n; i += tl.rpp) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < NVT; ++j) {
+          const int v = ct + j * tl.tpr;
+          if (v < vt) {
+            a0 = dot8(*reinterpret_cast<const uint4*>(w0 + (size_t)i * K + v * 8), xr[j], a0);
+            if (GATED) a1 = dot8(*reinterpret_cast<const uint4*>(w1 + (size_t)i * K + v * 8), xr[j], a1);
+          }
+        }
+        a0 = warp_sum(a0);
+        if (GATED) a1 = warp_sum(a1);
+        if (lane == 0) {
+          const int rl = r - g.r0 + i;
+          red[(rl * nm) * wpr + wir] = a0;
+          if (GATED) red[(rl * nm + 1) * wpr + wir] = a1;
+        }
+      }
+      release();
+    }
+    consumer_bar();
+  }
+
+  template <int NVT>
+  __device__ __forceinline__ void gemv_run(const mk_instr& in, int op, int layer) {
+    const Gemv g = gemv_geo(p, in, op, layer);
+    const int BH = p.B * p.H;
+    // input vector and prologue
+    const float* src;
+    const uint16_t* gain = nullptr;
+    if (op == OP_QKV) {
+      src = p.xres + (size_t)(2 * layer) * BH;
+      gain = p.layers[layer].attn_norm;
+    } else if (op == OP_OPROJ) {
+      src = p.attn;
+    } else if (op == OP_GATEUP) {
+      src = p.xres + (size_t)(2 * layer + 1) * BH;
+      gain = p.layers[layer].mlp_norm;
+    } else if (op == OP_DOWN) {
+      src = p.act;
+    } else {  // LM head
+      src = p.xres + (size_t)(2 * p.L) * BH;
+      gain = p.final_norm;
+    }
+    float xr[NVT][8];
+    load_x<NVT>(src, gain, g.K, g.tile, xr);
+    if (op == OP_GATEUP)
+      gemv_stream<NVT, true>(g, xr);
+    else
+      gemv_stream<NVT, false>(g, xr);
+    // epilogue: fixed-order sum of the per-warp partials, then the op's output
+    const int wpr = g.tile.tpr / 32, n = g.r1 - g.r0;
+    for (int i = t; i < n; i += kConsumerThreads) {
+      const int row = g.r0 + i;
+      if (op == OP_GATEUP) {
+        float gs = 0.f, us = 0.f;
+        for (int w = 0; w < wpr; ++w) {
+          gs += red[(i * 2) * wpr + w];
+          us += red[(i * 2 + 1) * wpr + w];
+        }
+        p.act[row] = gs / (1.f + expf(-gs)) * us;
+        continue;
+      }
+      float y = 0.f;
+      for (int w = 0; w < wpr; ++w) y += red[i * wpr + w];
+      if (op == OP_QKV) {
+        const int qd = p.nq * p.hd, kvd = p.nkv * p.hd;
+        const int off = in.c == 0 ? 0 : (in.c == 1 ? qd : qd + kvd);
+        p.qkv[off + row] = y;
+      } else if (op == OP_OPROJ) {
+        p.xres[(size_t)(2 * layer + 1) * BH + row] = __ldcg(p.xres + (size_t)(2 * layer) * BH + row) + y;
+      } else if (op == OP_DOWN) {
+        p.xres[(size_t)(2 * layer + 2) * BH + row] = __ldcg(p.xres + (size_t)(2 * layer + 1) * BH + row) + y;
+      } else {
+        p.logits[row] = y;
+      }
+    }
+  }
+
+  __device__ void gemv(const mk_instr& in, int op, int layer) {
+    const int K = op == OP_OPROJ ? p.nq * p.hd : (op == OP_DOWN ? p.I : p.H);
+    const int nv = gemv_tile(K, op == OP_GATEUP ? 2 : 1).nv;
+    if (nv <= 1)
+      gemv_run<1>(in, op, layer);
+    else if (nv <= 2)
+      gemv_run<2>(in, op, layer);
+    else if (nv <= 4)
+      gemv_run<4>(in, op, layer);
+    else
+      gemv_run<8>(in, op, layer);
+  }
+
+  // ---- attention ---------------------------------------------------------------
+  // One (sequence, KV head, chunk of positions): q of the G query heads of
+  // the group against the chunk's cached K/V rows (streamed through the ring)
+  // and, in the chunk that holds it, the new token's own K/V row.  The
+  // result is an unnormalised partial (o, m, l) in log2 units; the last
+  // chunk of the (sequence, KV head) to finish merges all partials.
+  template <int HD, int G>
+  __device__ __forceinline__ void attn_run(const mk_instr& in, int layer, int sig_idx) {
+    constexpr int LPP = HD / 8;    // lanes per position (16-byte vectors)
+    constexpr int PPW = 32 / LPP;  // positions per warp pass
+    const Attn a = attn_geo(p, in, layer, HD);
+    const int qd = p.nq * HD, kvd = p.nkv * HD;
+    const float* qkv = p.qkv + (size_t)a.b * (qd + 2 * kvd);
+    const float qscale = 1.4426950408889634f * rsqrtf((float)HD);  // log2(e) / sqrt(hd)
+    const int pl = lane / LPP, vi = lane % LPP;
+    if (a.active) {
+      // -- prologue: q heads (qk-norm, RoPE, scale) and the new K/V row
+      const int pos = p.positions[a.b];
+      const float2* cs = p.rope + (size_t)pos * (HD / 2);
+      const int tasks = G + (a.owns_new ? 2 : 0);
+      for (int task = warp; task < tasks; task += kConsumerWarps) {
+        const bool is_v = task == G + 1;
+        const float* src = task < G ? qkv + (a.kvh * G + task) * HD
+                                    : qkv + qd + (is_v ? kvd : 0) + a.kvh * HD;
+        constexpr int NP = HD / 64;  // rotation pairs per lane
+        float lo[NP], hi[NP];
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+          lo[j] = __ldcg(src + lane + 32 * j);
+          hi[j] = __ldcg(src + lane + 32 * j + HD / 2);
+          ss += lo[j] * lo[j] + hi[j] * hi[j];
+        }
+        if (!is_v) {
+          if (p.qk_norm) {
+            ss = warp_sum(ss);
+            const float sc = 1.f / sqrtf(ss / (float)HD + p.eps);
+            const uint16_t* gn = task < G ? p.layers[layer].q_norm : p.layers[layer].k_norm;
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+              lo[j] = lo[j] * sc * bf16_bits_to_f32(gn[lane + 32 * j]);
+              hi[j] = hi[j] * sc * bf16_bits_to_f32(gn[lane + 32 * j + HD / 2]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            const float2 r = cs[lane + 32 * j];
+            const float x0 = lo[j], x1 = hi[j];
+            lo[j] = x0 * r.x - x1 * r.y;
+            hi[j] = x1 * r.x + x0 * r.y;
+          }
+        }
+        if (task < G) {
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            ctl->qs[task * HD + lane + 32 * j] = lo[j] * qscale;
+            ctl->qs[task * HD + lane + 32 * j + HD / 2] = hi[j] * qscale;
+          }
+        } else {
+          // append the new row (bf16) at index S and keep its rounded value
+          uint16_t* cache = (is_v ? p.vc : p.kc) + a.cache_base + (size_t)(a.S - a.p0) * HD;
+          float* keep = is_v ? ctl->vnew : ctl->knew;
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            const uint16_t b0 = f32_to_bf16_bits(lo[j]), b1 = f32_to_bf16_bits(hi[j]);
+            cache[lane + 32 * j] = b0;
+            cache[lane + 32 * j + HD / 2] = b1;
+            keep[lane + 32 * j] = bf16_bits_to_f32(b0);
+            keep[lane + 32 * j + HD / 2] = bf16_bits_to_f32(b1);
+          }
+        }
+      }
+      consumer_bar();
+      // q stays in registers up to 4 heads per KV head; with 8 it is read
+      // from shared memory (a broadcast across position groups) so that the
+      // 8 x 8 running outputs fit the 168-register budget of a 9-warp CTA.
+      constexpr bool kQRegs = G <= 4;
+      float q[kQRegs ? G : 1][8], o[G][8], m[G], l[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        m[h] = -1e30f;
+        l[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (kQRegs) q[kQRegs ? h : 0][e] = ctl->qs[h * HD + vi * 8 + e];
+          o[h][e] = 0.f;
+        }
+      }
+      auto qv = [&](int h, int e) -> float { return kQRegs ? q[kQRegs ? h : 0][e] : ctl->qs[h * HD + vi * 8 + e]; };
+      // -- cached positions, streamed K stage then V stage
+      for (int s = 0; s < a.nsub; ++s) {
+        const int np = min(a.P, a.n_cached - s * a.P);
+        const uint16_t* Ks = reinterpret_cast<const uint16_t*>(wait_stage(k));
+        const uint16_t* Vs = reinterpret_cast<const uint16_t*>(wait_stage(k + 1));
+        for (int tb = warp * PPW; tb < np; tb += kConsumerWarps * PPW) {
+          const int tp = tb + pl;
+          const bool valid = tp < np;
+          float kf[8], vf[8];
+          if (valid) {
+            unpack8(*reinterpret_cast<const uint4*>(Ks + (size_t)tp * HD + vi * 8), kf);
+            unpack8(*reinterpret_cast<const uint4*>(Vs + (size_t)tp * HD + vi * 8), vf);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) kf[e] = vf[e] = 0.f;
+          }
+          float sc[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) d = fmaf(qv(h, e), kf[e], d);
+#pragma unroll
+            for (int off = LPP / 2; off; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+            sc[h] = d;
+          }
+          if (valid) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float mn = fmaxf(m[h], sc[h]);
+              const float corr = exp2f(m[h] - mn), pr = exp2f(sc[h] - mn);
+              l[h] = l[h] * corr + pr;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) o[h][e] = fmaf(o[h][e], corr, pr * vf[e]);
+              m[h] = mn;
+            }
+          }
+        }
+        release();  // K slot
+        release();  // V slot
+      }
+      // -- the new token (warp 0, first position group)
+      if (a.owns_new && warp == 0) {
+        float kf[8], vf[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          kf[e] = ctl->knew[vi * 8 + e];
+          vf[e] = ctl->vnew[vi * 8 + e];
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) d = fmaf(qv(h, e), kf[e], d);
+#pragma unroll
+          for (int off = LPP / 2; off; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+          if (pl == 0) {
+            const float mn = fmaxf(m[h], d);
+            const float corr = exp2f(m[h] - mn), pr = exp2f(d - mn);
+            l[h] = l[h] * corr + pr;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[h][e] = fmaf(o[h][e], corr, pr * vf[e]);
+            m[h] = mn;
+          }
+        }
+      }
+      // -- merge the position groups of each warp
+#pragma unroll
+      for (int off = LPP; off < 32; off <<= 1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float m2 = __shfl_xor_sync(0xffffffffu, m[h], off);
+          const float l2 = __shfl_xor_sync(0xffffffffu, l[h], off);
+          const float mn = fmaxf(m[h], m2);
+          const float c1 = exp2f(m[h] - mn), c2 = exp2f(m2 - mn);
+          l[h] = l[h] * c1 + l2 * c2;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float o2 = __shfl_xor_sync(0xffffffffu, o[h][e], off);
+            o[h][e] = o[h][e] * c1 + o2 * c2;
+          }
+          m[h] = mn;
+        }
+      }
+      // -- merge the warps through shared memory, one head at a time
+      const size_t pbase = ((size_t)a.b * p.nq + (size_t)a.kvh * G) * p.n_chunks + a.c;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (pl == 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) red[warp * (HD + 2) + vi * 8 + e] = o[h][e];
+          if (vi == 0) {
+            red[warp * (HD + 2) + HD] = m[h];
+            red[warp * (HD + 2) + HD + 1] = l[h];
+          }
+        }
+        consumer_bar();
+        if (t < HD) {
+          float M = -1e30f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * (HD + 2) + HD]);
+          float den = 0.f, num = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float c = exp2f(red[w * (HD + 2) + HD] - M);
+            den = fmaf(c, red[w * (HD + 2) + HD + 1], den);
+            num = fmaf(c, red[w * (HD + 2) + t], num);
+          }
+          const size_t pi = pbase + (size_t)h * p.n_chunks;
+          p.part_o[pi * HD + t] = num;
+          if (t == 0) {
+            p.part_ml[pi * 2] = M;
+            p.part_ml[pi * 2 + 1] = den;
+          }
+        }
+        consumer_bar();
+      }
+    }
+    // -- ticket: the last chunk of (sequence, KV head) to arrive merges
+    consumer_bar();
+    if (t == 0) {
+      __threadfence();
+      const uint32_t old = atom_acq_rel_add(p.tickets + ((size_t)layer * p.B + a.b) * p.nkv + a.kvh, 1u);
+      ctl->last = (old + 1u == p.epoch * (uint32_t)p.n_chunks);
+    }
+    consumer_bar();
+    if (ctl->last) {
+      const int nvalid = a.S / p.chunk + 1;  // chunks holding a position <= S
+      for (int idx = t; idx < G * HD; idx += kConsumerThreads) {
+        const int h = idx / HD, d = idx % HD;
+        const size_t pi0 = ((size_t)a.b * p.nq + (size_t)a.kvh * G + h) * p.n_chunks;
+        float M = -1e30f;
+        for (int c = 0; c < nvalid; ++c) M = fmaxf(M, __ldcg(p.part_ml + (pi0 + c) * 2));
+        float den = 0.f, num = 0.f;
+        for (int c = 0; c < nvalid; ++c) {
+          const float w = exp2f(__ldcg(p.part_ml + (pi0 + c) * 2) - M);
+          den = fmaf(w, __ldcg(p.part_ml + (pi0 + c) * 2 + 1), den);
+          num = fmaf(w, __ldcg(p.part_o + (pi0 + c) * HD + d), num);
+        }
+        p.attn[(size_t)a.b * qd + (size_t)(a.kvh * G + h) * HD + d] = num / den;
+      }
+      signal(sig_idx);
+    }
+  }
+
+  __device__ void attn(const mk_instr& in, int layer, int sig_idx) {
+    const int G = p.nq / p.nkv;
+    if (p.hd == 128) {
+      switch (G) {
+        case 1: attn_run<128, 1>(in, layer, sig_idx); break;
+        case 2: attn_run<128, 2>(in, layer, sig_idx); break;
+        case 4: attn_run<128, 4>(in, layer, sig_idx); break;
+        default: attn_run<128, 8>(in, layer, sig_idx); break;
+      }
+    } else {
+      switch (G) {
+        case 1: attn_run<64, 1>(in, layer, sig_idx); break;
+        case 2: attn_run<64, 2>(in, layer, sig_idx); break;
+        case 4: attn_run<64, 4>(in, layer, sig_idx); break;
+        default: attn_run<64, 8>(in, layer, sig_idx); break;
+      }
+    }
+  }
+};
+
+__device__ void run_consumers(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring, float* red) {
+  Consumer cs(p, ctl, ring, red);
+  for (int i = 0; i < n; ++i) {
+    const mk_instr in = list[i];
+    const int op = op_of(in.op_layer), layer = layer_of(in.op_layer);
+    if (!cs.wait_counter(in.wait_idx, in.wait_count)) {
+      ctl->dead = 1;
+      return;
+    }
+    switch (op) {
+      case OP_EMBED:
+        cs.embed(in);
+        cs.signal(in.sig_idx);
+        break;
+      case OP_QKV:
+      case OP_OPROJ:
+      case OP_GATEUP:
+      case OP_DOWN:
+      case OP_LMHEAD:
+        cs.gemv(in, op, layer);
+        cs.signal(in.sig_idx);
+        break;
+      case OP_ATTN:
+        cs.attn(in, layer, in.sig_idx);
+        break;
+      default:
+        break;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* ring = smem;
+  float* red = reinterpret_cast<float*>(smem + kRingBytes);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + kRingBytes + kRedBytes);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], kConsumerWarps);
+    }
+    ctl->dead = 0;
+    ctl->last = 0;
+    // a sticky error from an earlier step, or out-of-range inputs: do nothing
+    int bad = ld_relaxed_i32(p.status) != 0;
+    for (int b = 0; b < p.B && !bad; ++b) {
+      const int S = p.seq_lens[b], pos = p.positions[b], tok = p.tokens[b];
+      if (S < 0 || S >= p.T || pos < 0 || pos >= p.T || tok < 0 || tok >= p.V) {
+        set_status(p, MK_ERR_RANGE, b);
+        bad = 1;
+      }
+    }
+    ctl->flag = bad;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (ctl->flag) return;
+
+  const int n = p.offsets[blockIdx.x + 1] - p.offsets[blockIdx.x];
+  const mk_instr* list = p.instrs + p.offsets[blockIdx.x];
+  if (threadIdx.x >= kConsumerThreads) {
+    if (threadIdx.x == kConsumerThreads) run_producer(p, list, n, ctl, ring);
+  } else {
+    run_consumers(p, list, n, ctl, ring, red);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+size_t kernel_smem_bytes() { return kSmemBytes; }
+
+cudaError_t kernel_prepare() {
+  return cudaFuncSetAttribute(mk_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+}
+
+cudaError_t kernel_occupancy(int* blocks_per_sm) {
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_persistent, kThreads, kSmemBytes);
+}
+
+cudaError_t launch_step(const Params& p, int n_blocks, cudaStream_t stream) {
+  void* args[] = {const_cast<Params*>(&p)};
+  return cudaLaunchCooperativeKernel((const void*)mk_persistent, dim3(n_blocks), dim3(kThreads), args, kSmemBytes,
+                                     stream);
+}
+
+}  // namespace mk

@@ -1,0 +1,221 @@
+// Host scheduler: lowers one decode step of a model into per-SM instruction
+// lists with producer/consumer dependency counters.
+//
+// ForgeMegakernel (arXiv 2609.12379, abstract) names the two structural
+// properties followed here: "a fine-grained instruction stream for each SM"
+// and "dependency counters replacing the global synchronization".  The
+// lowering below is this library's own: every GEMV is cut into one contiguous
+// row range per SM (so each SM streams the same number of weight bytes per
+// op), attention is cut into (sequence, KV head, chunk) pieces dealt
+// round-robin over the SMs, and every instruction waits on exactly one
+// counter: the one bumped by the op it reads.
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "mk_internal.h"
+
+struct mk_plan {
+  mk_model_desc d;
+  int n_sm;
+  int chunk, n_chunks;
+  std::vector<std::vector<mk_instr>> lists;
+  std::vector<int32_t> targets;
+};
+
+namespace mk {
+
+static bool aligned_ok(int K, int n_mats) {
+  // a full row (or a gate+up row pair) must fit one ring slot, and each
+  // thread holds at most 8 input vectors
+  if (K <= 0 || K % 8) return false;
+  if ((int64_t)K * 2 * n_mats > kStageBytes) return false;
+  GemvTile t = gemv_tile(K, n_mats);
+  return t.nv <= 8 && t.rows_per_stage >= 1;
+}
+
+int validate_desc(const mk_model_desc* d) {
+  if (!d) return MK_ERR_INVALID_ARG;
+  if (d->n_layers <= 0 || d->hidden <= 0 || d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0 ||
+      d->vocab <= 0 || d->batch <= 0 || d->max_ctx <= 0 || d->n_layers > (1 << 20))
+    return MK_ERR_INVALID_ARG;
+  if (!(d->rms_eps >= 0.0f) || !(d->rope_theta > 0.0f)) return MK_ERR_INVALID_ARG;
+  if (d->n_experts < 0 || d->ffn_dim < 0) return MK_ERR_INVALID_ARG;
+  if (d->n_q_heads % d->n_kv_heads) return MK_ERR_UNSUPPORTED;
+  const int g = d->n_q_heads / d->n_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return MK_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128) return MK_ERR_UNSUPPORTED;
+  if (d->batch > 1) return MK_ERR_UNSUPPORTED;  // batch > 1 needs the tensor-core projections
+  if (d->n_experts) return MK_ERR_UNSUPPORTED;   // MoE lowering not built yet
+  if (d->ffn_dim <= 0) return MK_ERR_INVALID_ARG;
+  const int qd = d->n_q_heads * d->head_dim;
+  if (!aligned_ok(d->hidden, 1) || !aligned_ok(d->hidden, 2) || !aligned_ok(qd, 1) || !aligned_ok(d->ffn_dim, 1))
+    return MK_ERR_UNSUPPORTED;
+  if ((int64_t)d->max_ctx * d->head_dim > (1ll << 31)) return MK_ERR_UNSUPPORTED;
+  return MK_OK;
+}
+
+namespace {
+
+struct Builder {
+  mk_plan* p;
+  int emit(int sm, int op, int layer, int wait_idx, int wait_count, int sig_idx, int a, int b, int c = 0, int d = 0) {
+    mk_instr in;
+    in.op_layer = op | (layer << 8);
+    in.wait_idx = wait_idx;
+    in.wait_count = wait_count;
+    in.sig_idx = sig_idx;
+    in.a = a;
+    in.b = b;
+    in.c = c;
+    in.d = d;
+    p->lists[sm].push_back(in);
+    return 1;
+  }
+  // Rows [0, N) of one op split evenly over the SMs, each SM's share cut
+  // into instructions of at most kMaxRows rows (and at the boundaries in
+  // `cuts`, e.g. between wq/wk/wv).  Returns the number of instructions.
+  int rows_op(int op, int layer, int N, const std::vector<int>& cuts, int wait_idx, int wait_count, int sig_idx) {
+    int n = 0;
+    const int n_sm = p->n_sm;
+    for (int s = 0; s < n_sm; ++s) {
+      int r0 = (int)((int64_t)N * s / n_sm), r1 = (int)((int64_t)N * (s + 1) / n_sm);
+      while (r0 < r1) {
+        int e = std::min(r1, r0 + kMaxRows);
+        int seg = 0, base = 0;
+        for (size_t k = 0; k < cuts.size(); ++k) {
+          if (r0 >= cuts[k]) { seg = (int)k + 1; base = cuts[k]; }
+        }
+        if (seg < (int)cuts.size()) e = std::min(e, cuts[seg]);
+        n += emit(s, op, layer, wait_idx, wait_count, sig_idx, r0 - base, e - base, seg);
+        r0 = e;
+      }
+    }
+    return n;
+  }
+};
+
+int default_chunk(const mk_model_desc* d, int n_sm) {
+  const char* env = getenv("MK_ATTN_CHUNK");
+  if (env && atoi(env) > 0) return atoi(env);
+  const int P = attn_stage_positions(d->head_dim);
+  int64_t total = (int64_t)d->batch * d->n_kv_heads * d->max_ctx;
+  int64_t c = (total + n_sm - 1) / n_sm;
+  c = (c + P - 1) / P * P;
+  c = std::max<int64_t>(P, std::min<int64_t>(c, 1024));
+  return (int)c;
+}
+
+}  // namespace
+
+int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
+  p->d = *d;
+  p->n_sm = n_sm;
+  p->lists.assign(n_sm, {});
+  const int L = d->n_layers, H = d->hidden, hd = d->head_dim;
+  const int qd = d->n_q_heads * hd, kvd = d->n_kv_heads * hd;
+  p->targets.assign(n_counters(L), 0);
+  p->chunk = default_chunk(d, n_sm);
+  p->n_chunks = (d->max_ctx + p->chunk - 1) / p->chunk;
+  Builder b{p};
+
+  // x0 = embedding rows, hidden dimension split over the SMs
+  int n_embed = 0;
+  const int c_embed = counter_embed(L);
+  for (int s = 0; s < n_sm; ++s) {
+    int r0 = (int)((int64_t)H * s / n_sm), r1 = (int)((int64_t)H * (s + 1) / n_sm);
+    if (r0 < r1) n_embed += b.emit(s, OP_EMBED, 0, -1, 0, c_embed, r0, r1);
+  }
+  p->targets[c_embed] = n_embed;
+
+  int prev_idx = c_embed, prev_count = n_embed;
+  int64_t attn_rr = 0;
+  for (int l = 0; l < L; ++l) {
+    const int cq = counter_index(l, C_QKV), ca = counter_index(l, C_ATTN), co = counter_index(l, C_OPROJ);
+    const int cg = counter_index(l, C_GATEUP), cd = counter_index(l, C_DOWN);
+    int n_qkv = b.rows_op(OP_QKV, l, qd + 2 * kvd, {qd, qd + kvd}, prev_idx, prev_count, cq);
+    p->targets[cq] = n_qkv;
+    for (int s = 0; s < d->batch; ++s)
+      for (int h = 0; h < d->n_kv_heads; ++h)
+        for (int c = 0; c < p->n_chunks; ++c) {
+          b.emit((int)(attn_rr % n_sm), OP_ATTN, l, cq, n_qkv, ca, s, h, c);
+          ++attn_rr;
+        }
+    p->targets[ca] = d->batch * d->n_kv_heads;  // one bump per merged (sequence, KV head)
+    int n_o = b.rows_op(OP_OPROJ, l, H, {}, ca, p->targets[ca], co);
+    p->targets[co] = n_o;
+    int n_gu = b.rows_op(OP_GATEUP, l, d->ffn_dim, {}, co, n_o, cg);
+    p->targets[cg] = n_gu;
+    int n_dn = b.rows_op(OP_DOWN, l, H, {}, cg, n_gu, cd);
+    p->targets[cd] = n_dn;
+    prev_idx = cd;
+    prev_count = n_dn;
+  }
+  const int c_lm = counter_lmhead(L);
+  p->targets[c_lm] = b.rows_op(OP_LMHEAD, L, d->vocab, {}, prev_idx, prev_count, c_lm);
+  return MK_OK;
+}
+
+}  // namespace mk
+
+// ---- C ABI: host-only lowering ---------------------------------------------------
+
+extern "C" int mk_plan_create(const mk_model_desc* desc, int n_sm, mk_plan** out) {
+  if (!out || n_sm <= 0) return MK_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = mk::validate_desc(desc);
+  if (rc) return rc;
+  mk_plan* p = new (std::nothrow) mk_plan();
+  if (!p) return MK_ERR_INVALID_ARG;
+  rc = mk::build_plan(desc, n_sm, p);
+  if (rc) {
+    delete p;
+    return rc;
+  }
+  *out = p;
+  return MK_OK;
+}
+
+extern "C" int mk_plan_n_sm(const mk_plan* p) { return p ? p->n_sm : MK_ERR_INVALID_ARG; }
+
+extern "C" int mk_plan_n_counters(const mk_plan* p) { return p ? (int)p->targets.size() : MK_ERR_INVALID_ARG; }
+
+extern "C" int mk_plan_n_instrs(const mk_plan* p) {
+  if (!p) return MK_ERR_INVALID_ARG;
+  size_t n = 0;
+  for (auto& l : p->lists) n += l.size();
+  return (int)n;
+}
+
+extern "C" int mk_plan_copy(const mk_plan* p, mk_instr* instrs, int32_t* offsets) {
+  if (!p || !instrs || !offsets) return MK_ERR_INVALID_ARG;
+  int32_t o = 0;
+  for (int s = 0; s < p->n_sm; ++s) {
+    offsets[s] = o;
+    memcpy(instrs + o, p->lists[s].data(), p->lists[s].size() * sizeof(mk_instr));
+    o += (int32_t)p->lists[s].size();
+  }
+  offsets[p->n_sm] = o;
+  return MK_OK;
+}
+
+extern "C" int mk_plan_counter_targets(const mk_plan* p, int32_t* targets) {
+  if (!p || !targets) return MK_ERR_INVALID_ARG;
+  memcpy(targets, p->targets.data(), p->targets.size() * sizeof(int32_t));
+  return MK_OK;
+}
+
+extern "C" int mk_plan_attn_chunk(const mk_plan* p, int32_t* chunk, int32_t* n_chunks) {
+  if (!p || !chunk || !n_chunks) return MK_ERR_INVALID_ARG;
+  *chunk = p->chunk;
+  *n_chunks = p->n_chunks;
+  return MK_OK;
+}
+
+extern "C" int mk_plan_destroy(mk_plan* p) {
+  delete p;
+  return MK_OK;
+}

@@ -1,0 +1,352 @@
+"""Decode-step benchmark of the persistent megakernel on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config dense-8b] [--impl mk|reference]
+
+A step is one decode step of the whole model (every layer, LM head) for the
+batch, through the C ABI (mk_decode_step).  Inputs are seeded and synthetic
+(random-init weights of the named shape, prefilled KV cache, uniform token ids,
+teacher forcing).  One JSON line on stdout (rank 0):
+
+  value   decode tokens/s with inputs resident in HBM (CUDA events on the launching stream,
+          K consecutive steps, max over ranks)
+  e2e     the same metric with tokens/positions/lengths copied from pinned host memory and
+          the logits copied back inside the timed region
+  roofline / mbu
+          algorithmic bytes per step (bf16 weights read + KV-cache positions read/written)
+          / kernel time, against the measured HBM copy bandwidth (MEASURED_PEAKS.json) and
+          against the 8 TB/s B200 specification
+  cpu_baseline
+          the CPU oracle (single-threaded fp64) on a bounded sample of the same step
+
+Multi-GPU (torchrun): independent replicas, one model per GPU, no collective on the data
+path; value = tokens/s summed over ranks, timed as the slowest rank.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import fixtures as fx  # noqa: E402
+
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def weight_bytes_read(cfg) -> int:
+    """bf16 weight bytes a dense step reads: every layer matrix and norm, the LM head, B embedding rows."""
+    H, L = cfg.hidden, cfg.n_layers
+    per = 2 * H + cfg.q_dim * H * 2 + cfg.kv_dim * H * 2 + 3 * cfg.ffn_dim * H
+    if cfg.qk_norm:
+        per += 2 * cfg.head_dim
+    return 2 * (L * per + H + cfg.vocab * H + cfg.batch * H)
+
+
+def kv_bytes(cfg, seq_lens) -> int:
+    """KV-cache bytes a step touches: S_b cached positions read + 1 new row written, K and V, all layers."""
+    return 2 * cfg.n_layers * cfg.n_kv_heads * cfg.head_dim * 2 * int(np.sum(np.asarray(seq_lens) + 1))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "auto_regressive_decode_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_source") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples of this process's GPU during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if len(s) > 3 + i and s[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------------------------
+# CPU baseline: the oracle, as it stands, on a bounded sample of the step
+# ---------------------------------------------------------------------------------------------------------
+
+def cpu_baseline(cfg, seed=fx.DEFAULT_SEED, max_layers=2):
+    import oracle as ora
+    from tests.helpers import host_model
+    n = min(max_layers, cfg.n_layers)
+    g, ls = host_model(cfg, seed, layers=range(n))
+    S = fx.context_lengths(cfg, seed)
+    kc = [fx.kv_prefill(cfg, l, 0, S, seed) for l in range(n)]
+    vc = [fx.kv_prefill(cfg, l, 1, S, seed) for l in range(n)]
+    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls)
+    tok = fx.tokens(cfg, seed)[0]
+    x = fx.bf16_to_f32(g["embed"][tok]).astype(np.float64)
+    t0 = time.perf_counter()
+    for l in range(n):
+        model.layer_forward(l, x, kc[l], vc[l], S, S)
+    t_layers = (time.perf_counter() - t0) / n
+    t1 = time.perf_counter()
+    for b in range(cfg.batch):
+        model.lm_head(x[b])
+    t_head = time.perf_counter() - t1
+    step_s = t_layers * cfg.n_layers + t_head
+    return {"value": cfg.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {cfg.n_layers} layers + LM head of step 0 (fp64, single thread), "
+                      f"extrapolated to the full step: {step_s:.3f} s/step",
+            "step_s": step_s}
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    base = cpu_baseline(cfg)
+    out = {"impl": "reference", "metric": "decode tokens/s (batch tokens per decode step / step time)",
+           "value": base["value"], "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": base["step_s"] * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": workload_config(cfg),
+           "cpu_baseline": {k: base[k] for k in ("kind", "cores", "sample", "value", "unit")},
+           "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def workload_config(cfg):
+    ctx = f"ctx U[{cfg.ctx_lo},{cfg.ctx_hi}]" if cfg.ragged else f"ctx {cfg.ctx}"
+    return {"workload": f"{cfg.name}: {cfg.n_layers} layers, hidden {cfg.hidden}, {cfg.n_q_heads}q/{cfg.n_kv_heads}kv "
+                        f"heads x {cfg.head_dim}, ffn {cfg.ffn_dim or cfg.expert_ffn_dim}, vocab {cfg.vocab}; "
+                        f"batch {cfg.batch}, {ctx}, teacher-forced decode",
+            "batch": cfg.batch, "max_ctx": cfg.max_ctx, "weights": "bf16 ~N(0,0.02), seeded",
+            "kv_cache": "bf16 ~N(0,1), seeded", "accumulate": "fp32",
+            "l2": "inputs larger than L2 (weights stream from HBM every step)"}
+
+
+# ---------------------------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------------------------
+
+def run_mk(args, cfg, rank, world):
+    import torch
+    import auto_regressive_decode_b200.mk as mk
+    from fixtures.device import device_caches, device_model
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    seed = fx.DEFAULT_SEED + rank
+    S0 = fx.context_lengths(cfg, seed)
+    toks = fx.tokens(cfg, seed)
+    w = device_model(cfg, seed)
+    kc, vc = device_caches(cfg, S0, seed)
+    dec = mk.Decoder(cfg, w, kc, vc)
+    B, V = cfg.batch, cfg.vocab
+    n_total = args.warmup + args.steps
+    # per-step inputs, resident on the device (teacher forcing; positions wrap after cfg.steps)
+    steps_idx = np.arange(n_total) % cfg.steps
+    all_tok = torch.from_numpy(toks[steps_idx].astype(np.int32)).to(dev)
+    all_len = torch.from_numpy((S0[None, :] + steps_idx[:, None]).astype(np.int32)).to(dev)
+    logits = torch.empty((B, V), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for i in range(args.warmup):
+        dec.step(all_tok[i], all_len[i], all_len[i], logits)
+    torch.cuda.synchronize()
+    st = dec.status()
+    if st != 0:
+        raise RuntimeError(f"device status {mk.mk_status_string(st)}")
+
+    # ---- device-resident timing: one event pair per step, on the launching stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    props = torch.cuda.get_device_properties(dev)
+    uuid = "GPU-" + str(props.uuid) if not str(props.uuid).startswith("GPU-") else str(props.uuid)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(uuid) as clk:
+        ev[0].record(stream)
+        for j in range(args.steps):
+            i = args.warmup + j
+            dec.step(all_tok[i], all_len[i], all_len[i], logits)
+            ev[j + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    st = dec.status()
+    if st != 0:
+        raise RuntimeError(f"device status {mk.mk_status_string(st)}")
+    per_step_ms = [ev[j].elapsed_time(ev[j + 1]) for j in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+
+    # ---- end to end through the C ABI with host buffers
+    h_tok = torch.from_numpy(toks[steps_idx].astype(np.int32)).pin_memory()
+    h_len = torch.from_numpy((S0[None, :] + steps_idx[:, None]).astype(np.int32)).pin_memory()
+    h_logits = torch.empty((B, V), dtype=torch.float32).pin_memory()
+    d_tok = torch.empty(B, dtype=torch.int32, device=dev)
+    d_len = torch.empty(B, dtype=torch.int32, device=dev)
+    d_pos = torch.empty(B, dtype=torch.int32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for j in range(args.steps):
+        i = args.warmup + j
+        d_tok.copy_(h_tok[i], non_blocking=True)
+        d_len.copy_(h_len[i], non_blocking=True)
+        d_pos.copy_(h_len[i], non_blocking=True)
+        dec.step(d_tok, d_pos, d_len, logits)
+        h_logits.copy_(logits, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    st = dec.status()
+    if st != 0:
+        raise RuntimeError(f"device status {mk.mk_status_string(st)}")
+
+    # ---- max over ranks
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+    dec.close()
+    if rank != 0:
+        return
+
+    ms = total_ms / args.steps
+    tok_s = world * B * args.steps / (total_ms / 1e3)
+    e2e_tok_s = world * B * args.steps / (e2e_ms / 1e3)
+    lens = [S0 + (k % cfg.steps) for k in range(args.warmup, n_total)]
+    bytes_step = weight_bytes_read(cfg) + float(np.mean([kv_bytes(cfg, s) for s in lens]))
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_step / (ms / 1e3) / 1e9
+    traffic = ncu_traffic(cfg.name)
+    out = {
+        "metric": "decode tokens/s (batch tokens per decode step / step time)",
+        "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights and KV cache, uniform token ids)",
+        "config": dict(workload_config(cfg), parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
+        "step_latency_ms": {"median": statistics.median(per_step_ms), "p10": float(np.percentile(per_step_ms, 10)),
+                            "p90": float(np.percentile(per_step_ms, 90))},
+        "bytes_per_step": bytes_step,
+        "mbu": {"vs_spec_8tbs": achieved / SPEC_HBM_GBS, f"vs_{peak_kind}_{peak:.0f}gbs": achieved / peak},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback", "traffic": traffic, "kernel": "mk_persistent"},
+        "e2e": {"value": e2e_tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 3 * 4 * B,
+                "d2h_bytes_per_step": 4 * B * V},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline:
+        base = cpu_baseline(cfg)
+        out["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="dense-8b", choices=sorted(fx.CONFIGS))
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = fx.CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_mk(args, cfg, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

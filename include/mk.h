@@ -1,0 +1,171 @@
+/*
+ * mk — one auto-regressive decode step of a decoder-only transformer as ONE
+ * persistent CUDA kernel for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the decode step of ForgeMegakernel (arXiv 2609.12379,
+ * abstract): per token, embed -> for every layer [RMSNorm, Q/K/V projection,
+ * optional per-head q/k RMSNorm, RoPE, KV-cache append, attention over the
+ * cache, output projection + residual, RMSNorm, SwiGLU MLP or top-k MoE +
+ * residual] -> final RMSNorm -> LM head.  The abstract names the structural
+ * properties the kernel follows: a fine-grained instruction stream per SM and
+ * dependency counters in place of grid-wide synchronisation.
+ *
+ * Conventions of every entry point:
+ *   - Plain C types only.  Pointers documented "device" must be device
+ *     memory of the current CUDA device; "host" pointers are host memory.
+ *   - Return value: MK_OK (0) or a negative mk_status code.  No call aborts
+ *     or throws.  mk_status_string() names a code.
+ *   - A handle is not thread-safe: calls on one handle must be serialised.
+ *
+ * Data types: weights and the KV cache are bfloat16 (bit patterns, 2 bytes);
+ * activations and logits are float32; token ids, positions and lengths are
+ * int32.  All weight matrices are row-major [out][in] (y = W x), every
+ * weight/cache pointer 16-byte aligned.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mk_status {
+  MK_OK = 0,
+  MK_ERR_INVALID_ARG = -1,    /* NULL pointer, non-positive size, bad enum */
+  MK_ERR_UNSUPPORTED = -2,    /* shape, alignment or device not supported */
+  MK_ERR_CUDA = -3,           /* a CUDA runtime call failed (allocation, launch) */
+  MK_ERR_DEVICE_TIMEOUT = -4, /* a bounded in-kernel wait ran out; the step was abandoned */
+  MK_ERR_RANGE = -5           /* seq_lens/positions/tokens out of range (detected on the device) */
+} mk_status;
+
+/* Model shape, fixed at creation (all sizes in elements). */
+typedef struct mk_model_desc {
+  int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn_dim, vocab;
+  int32_t n_experts, top_k, expert_ffn_dim; /* n_experts == 0: dense SwiGLU MLP */
+  int32_t qk_norm;                          /* 1: per-head RMSNorm of q and k (gain [head_dim]) before RoPE */
+  int32_t tied_embeddings;                  /* 1: LM head is the embedding matrix */
+  float rms_eps, rope_theta;
+  int32_t batch;                            /* sequences decoded together */
+  int32_t max_ctx;                          /* KV-cache capacity (positions) per sequence */
+  uint64_t wait_timeout_ns;                 /* bound of every in-kernel wait; 0 -> 2 s */
+} mk_model_desc;
+
+/* Per-layer weights (device, bf16).  Shapes with H = hidden, D = head_dim:
+ *   attn_norm, mlp_norm [H]; q_norm, k_norm [D] (qk_norm only, else NULL)
+ *   wq [n_q_heads*D][H]; wk, wv [n_kv_heads*D][H]; wo [H][n_q_heads*D]
+ *   dense:  w_gate, w_up [ffn_dim][H]; w_down [H][ffn_dim]; router NULL
+ *   MoE:    w_gate, w_up [n_experts][expert_ffn_dim][H] (stacked);
+ *           w_down [n_experts][H][expert_ffn_dim]; router [n_experts][H] */
+typedef struct mk_layer_weights {
+  const void *attn_norm, *wq, *wk, *wv, *q_norm, *k_norm, *wo, *mlp_norm;
+  const void *w_gate, *w_up, *w_down, *router;
+} mk_layer_weights;
+
+/* Model-global weights (device, bf16): embed [vocab][H], final_norm [H],
+ * lm_head [vocab][H] (ignored when tied_embeddings).  layers: HOST array of
+ * n_layers entries, read during mk_create only. */
+typedef struct mk_weights {
+  const void *embed, *final_norm, *lm_head;
+  const mk_layer_weights* layers;
+} mk_weights;
+
+/* KV cache (device, bf16, caller-owned): k and v are each
+ * [n_layers][batch][n_kv_heads][max_ctx][head_dim]. */
+typedef struct mk_kv {
+  void *k, *v;
+} mk_kv;
+
+typedef struct mk_handle mk_handle;
+
+/*
+ * Validate the shape, lower the model into per-SM instruction lists, and
+ * allocate the library-owned device state (instruction lists, dependency
+ * counters, activation scratch, RoPE cos/sin table) on the current device.
+ * Weight and cache pointers are borrowed: they must stay valid until
+ * mk_destroy and are never freed by the library.
+ * Returns MK_ERR_UNSUPPORTED for shapes the kernel cannot run (e.g. a matrix
+ * row wider than one pipeline stage, head_dim not 64/128, misaligned pointers).
+ */
+int mk_create(const mk_model_desc* desc, const mk_weights* weights, const mk_kv* kv, mk_handle** out);
+
+/*
+ * One decode step for every sequence, asynchronous on `stream` (a
+ * cudaStream_t; NULL = legacy default stream): one kernel launch, no host
+ * synchronisation and no allocation.
+ *   tokens    device int32[batch]  token id entering the model
+ *   positions device int32[batch]  RoPE position of that token (normally seq_lens[b])
+ *   seq_lens  device int32[batch]  tokens already cached; the step writes the new K/V
+ *                                  row at index seq_lens[b] and attends over
+ *                                  seq_lens[b]+1 positions.  The caller advances it.
+ *   out_logits device float[batch][vocab]
+ * A device-side failure (range error, wait timeout) is reported by
+ * mk_get_status; until then later steps return at once without computing.
+ */
+int mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions, const int32_t* seq_lens,
+                   void* stream, float* out_logits);
+
+/* Synchronise `stream` and return the device-side status of the last steps
+ * (MK_OK, MK_ERR_DEVICE_TIMEOUT or MK_ERR_RANGE).  A failure is cleared and
+ * the dependency counters are reset, so the handle is usable again. */
+int mk_get_status(mk_handle* h, void* stream);
+
+/* Free the library-owned device state.  NULL is accepted. */
+int mk_destroy(mk_handle* h);
+
+const char* mk_status_string(int status);
+
+/* Mid-states of the last step, copied (async on `stream`, device-to-device or
+ * device-to-host per `dst`) into dst[bytes]:
+ *   MK_STATE_HIDDEN      float[2*n_layers+1][batch][hidden]: index 0 is the
+ *                        embedding, 2l+1 the residual after layer l's
+ *                        attention block, 2l+2 after its MLP block
+ *   MK_STATE_ROUTER      float[n_layers][batch][n_experts] router logits (MoE)
+ *   MK_STATE_SELECTION   int32[n_layers][batch][top_k] chosen experts (MoE)
+ *   MK_STATE_SEL_WEIGHT  float[n_layers][batch][top_k] their weights (MoE)
+ *   MK_STATE_EXPERT_COUNT int32[n_layers] distinct experts used (MoE) */
+enum {
+  MK_STATE_HIDDEN = 0,
+  MK_STATE_ROUTER = 1,
+  MK_STATE_SELECTION = 2,
+  MK_STATE_SEL_WEIGHT = 3,
+  MK_STATE_EXPERT_COUNT = 4
+};
+int mk_read_state(mk_handle* h, int which, void* dst, size_t bytes, void* stream);
+
+/* Bytes of the mid-state `which` (0 if the model has none). */
+size_t mk_state_bytes(const mk_handle* h, int which);
+
+/* ---- host-only lowering (no GPU needed) ---------------------------------- */
+
+/* One instruction of a per-SM list (8 x int32); see mk_plan_* below. */
+typedef struct mk_instr {
+  int32_t op_layer;   /* op | layer << 8 */
+  int32_t wait_idx;   /* counter waited on, -1 none */
+  int32_t wait_count; /* producers per step the wait needs */
+  int32_t sig_idx;    /* counter bumped on completion, -1 none */
+  int32_t a, b, c, d; /* op arguments */
+} mk_instr;
+
+typedef struct mk_plan mk_plan;
+
+/* Lower `desc` for `n_sm` SMs on the host (no CUDA call).  Same validation
+ * and the same lists that mk_create builds for a device with n_sm SMs. */
+int mk_plan_create(const mk_model_desc* desc, int n_sm, mk_plan** out);
+int mk_plan_n_sm(const mk_plan* p);
+int mk_plan_n_counters(const mk_plan* p);
+/* offsets: int32[n_sm+1] (SM s owns instructions [offsets[s], offsets[s+1])). */
+int mk_plan_n_instrs(const mk_plan* p);
+int mk_plan_copy(const mk_plan* p, mk_instr* instrs, int32_t* offsets);
+/* Per-step producers of each counter: int32[n_counters]. */
+int mk_plan_counter_targets(const mk_plan* p, int32_t* targets);
+/* Attention split: positions per chunk and chunks per sequence. */
+int mk_plan_attn_chunk(const mk_plan* p, int32_t* chunk, int32_t* n_chunks);
+int mk_plan_destroy(mk_plan* p);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,87 @@
+"""Teacher-forced GPU-vs-oracle runs shared by the GPU parity tests and the smoke check.
+
+Tolerances (stated by the decode-step parity contract this library is held to):
+per-layer hidden-state relative L2 <= 1e-2, logits max abs <= 5e-2,
+appended K/V relative L2 <= 1e-2, top-1 token identical on >= 99% of steps.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import fixtures as fx
+import oracle as ora
+from fixtures.device import device_caches, device_model
+from tests.helpers import bf16_f64, expert_loader, host_caches, host_model, rel_l2
+
+TOL_HIDDEN = 1e-2
+TOL_LOGITS_ABS = 5e-2
+TOL_KV = 1e-2
+MIN_TOP1 = 0.99
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def run_teacher_forced(cfg, steps=None, gains="ones", seed=fx.DEFAULT_SEED, seq_lens=None, wait_timeout_ns=0):
+    """Run `steps` decode steps on the GPU and in the oracle; return per-step error metrics."""
+    import auto_regressive_decode_b200.mk as mk
+    steps = cfg.steps if steps is None else steps
+    S0 = fx.context_lengths(cfg, seed) if seq_lens is None else np.asarray(seq_lens, dtype=np.int32)
+    toks = fx.tokens(cfg, seed)
+    # GPU side: poisoned cache tail, so that a read past a sequence's length shows up as NaN
+    w = device_model(cfg, seed, gains)
+    kc, vc = device_caches(cfg, S0, seed, poison=True)
+    k_init, v_init = kc.clone(), vc.clone()
+    dec = mk.Decoder(cfg, w, kc, vc, wait_timeout_ns=wait_timeout_ns)
+    # oracle side: its own caches from the same generator
+    g, ls = host_model(cfg, seed, gains)
+    okc, ovc = host_caches(cfg, S0, seed)
+    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls,
+                      expert_loader(cfg, seed) if cfg.n_experts else None)
+    B, L = cfg.batch, cfg.n_layers
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    res = {"hidden": [], "logits_abs": [], "kv": [], "top1": [], "status": []}
+    for t in range(steps):
+        S = (S0 + t).astype(np.int32)
+        tok = toks[t % toks.shape[0]]
+        dt = torch.from_numpy(tok.copy()).cuda()
+        ds = torch.from_numpy(S.copy()).cuda()
+        dec.step(dt, ds, ds, logits)
+        st = dec.status()
+        res["status"].append(st)
+        hid = dec.hidden_states().cpu().numpy().astype(np.float64)
+        lg = logits.cpu().numpy().astype(np.float64)
+        ref = model.decode_step(okc, ovc, tok, S, S)
+        errs = []
+        for l in range(L):
+            errs.append(rel_l2(hid[2 * l + 1], ref["h_attn"][l]))
+            errs.append(rel_l2(hid[2 * l + 2], ref["h_mlp"][l]))
+        res["hidden"].append(max(errs))
+        res["logits_abs"].append(float(np.max(np.abs(lg - ref["logits"]))))
+        kv_err = 0.0
+        for b in range(B):
+            gk = bf16_f64(bits(kc[:, b, :, S[b]].contiguous()))
+            gv = bf16_f64(bits(vc[:, b, :, S[b]].contiguous()))
+            kv_err = max(kv_err, rel_l2(gk, bf16_f64(okc[:, b, :, S[b]])), rel_l2(gv, bf16_f64(ovc[:, b, :, S[b]])))
+        res["kv"].append(kv_err)
+        res["top1"].extend(list(np.argmax(lg, axis=1) == np.argmax(ref["logits"], axis=1)))
+    # cache bytes other than the appended rows are untouched
+    kc_h, vc_h, ki, vi = bits(kc), bits(vc), bits(k_init), bits(v_init)
+    touched = np.zeros(kc_h.shape[:4], dtype=bool)   # [L][B][nkv][T]
+    for b in range(B):
+        touched[:, b, :, S0[b]:S0[b] + steps] = True
+    res["untouched_ok"] = bool(np.array_equal(kc_h[~touched], ki[~touched]) and
+                               np.array_equal(vc_h[~touched], vi[~touched]))
+    dec.close()
+    return res
+
+
+def assert_parity(res):
+    assert all(s == 0 for s in res["status"]), res["status"]
+    assert max(res["hidden"]) <= TOL_HIDDEN, res["hidden"]
+    assert max(res["logits_abs"]) <= TOL_LOGITS_ABS, res["logits_abs"]
+    assert max(res["kv"]) <= TOL_KV, res["kv"]
+    assert np.mean(res["top1"]) >= MIN_TOP1, np.mean(res["top1"])
+    assert res["untouched_ok"]
