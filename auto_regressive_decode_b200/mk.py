@@ -69,6 +69,8 @@ def _load():
         "mk_status_string": (ctypes.c_char_p, [_i32]),
         "mk_read_state": (_i32, [H, _i32, _P, ctypes.c_size_t, _P]),
         "mk_state_bytes": (ctypes.c_size_t, [H, _i32]),
+        "mk_decode_step_noalloc": (_i32, [ctypes.POINTER(mk_model_desc), ctypes.POINTER(mk_weights),
+                                          ctypes.POINTER(mk_kv), _P, _P, _P, _P, _P]),
         "mk_plan_create": (_i32, [ctypes.POINTER(mk_model_desc), _i32, ctypes.POINTER(H)]),
         "mk_plan_n_sm": (_i32, [H]),
         "mk_plan_n_counters": (_i32, [H]),
@@ -94,6 +96,7 @@ mk_get_status = lib.mk_get_status
 mk_destroy = lib.mk_destroy
 mk_read_state = lib.mk_read_state
 mk_state_bytes = lib.mk_state_bytes
+mk_decode_step_noalloc = lib.mk_decode_step_noalloc
 mk_plan_create = lib.mk_plan_create
 mk_plan_n_sm = lib.mk_plan_n_sm
 mk_plan_n_counters = lib.mk_plan_n_counters
@@ -226,3 +229,19 @@ class Decoder:
             self.close()
         except Exception:
             pass
+
+
+def weight_structs(cfg, weights, k_cache, v_cache):
+    """(mk_model_desc, mk_weights, mk_kv, keep-alive) for a stateless call such as mk_decode_step_noalloc."""
+    L = cfg.n_layers
+    layers = (mk_layer_weights * L)()
+    for l in range(L):
+        lw = weights["layers"][l]
+        for name, _ in mk_layer_weights._fields_:
+            t = lw.get(name)
+            setattr(layers[l], name, None if t is None else t.data_ptr())
+    lm = weights.get("lm_head")
+    w = mk_weights(weights["embed"].data_ptr(), weights["final_norm"].data_ptr(),
+                   None if lm is None else lm.data_ptr(), layers)
+    kv = mk_kv(k_cache.data_ptr(), v_cache.data_ptr())
+    return model_desc(cfg), w, kv, (layers, weights, k_cache, v_cache)

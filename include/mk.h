@@ -138,6 +138,31 @@ int mk_read_state(mk_handle* h, int which, void* dst, size_t bytes, void* stream
 /* Bytes of the mid-state `which` (0 if the model has none). */
 size_t mk_state_bytes(const mk_handle* h, int which);
 
+/*
+ * mk_decode_step_noalloc: one decode step that allocates no device memory.
+ * (No counterpart in the paper: an addition for callers that cannot call
+ * cudaMalloc where they decode, e.g. a plugin inside another engine that owns
+ * every device byte, or a real-time path that must not enter the allocator.)
+ *
+ * Same model, weights, cache and per-step arguments as mk_create followed by
+ * mk_decode_step, and the same kernel, but every byte of library state lives
+ * in one static device array of 8 MiB that each GPU loading the library holds
+ * until the process exits.  A model whose state (instruction lists, counters,
+ * activations, RoPE table) needs more returns MK_ERR_UNSUPPORTED.
+ *   - The first call on a device resolves the array's address there
+ *     (cudaGetSymbolAddress with that device current); make that first call
+ *     before any stream capture.
+ *   - Each call clears the counters and status words it uses, uploads the
+ *     instruction lists from temporary host memory, launches on `stream` and
+ *     then synchronises `stream` so that it can return the device-side status
+ *     (MK_OK, MK_ERR_RANGE, MK_ERR_DEVICE_TIMEOUT).
+ *   - All calls share the array, which keeps the last call's contents: calls
+ *     that overlap on the GPU (other streams, other host threads) race.
+ */
+int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weights* weights, const mk_kv* kv,
+                           const int32_t* tokens, const int32_t* positions, const int32_t* seq_lens, void* stream,
+                           float* out_logits);
+
 /* ---- host-only lowering (no GPU needed) ---------------------------------- */
 
 /* One instruction of a per-SM list (8 x int32); see mk_plan_* below. */
