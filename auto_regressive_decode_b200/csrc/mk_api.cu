@@ -37,6 +37,7 @@ struct mk_handle {
   size_t n_tickets;
   void* region;
   size_t region_bytes;
+  size_t n_instr;
   uint32_t epoch;
 };
 
@@ -137,6 +138,10 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const size_t o_off = cv.take(sizeof(int32_t) * offsets.size());
   const size_t o_lay = cv.take(sizeof(mk::LayerPtrs) * (size_t)L);
   const size_t o_rope = cv.take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
+  const char* trace_env = getenv("MK_TRACE");
+  const bool tracing = trace_env && atoi(trace_env) > 0;
+  const size_t o_trace = tracing ? cv.take(sizeof(uint64_t) * mk::kTraceStamps * instrs.size()) : 0;
+  h->n_instr = tracing ? (size_t)n_instr : 0;
   h->region_bytes = cv.off;
   if (cudaMalloc(&h->region, h->region_bytes) != cudaSuccess) {
     delete h;
@@ -217,6 +222,9 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   p.instrs = (const mk_instr*)(base + o_ins);
   p.offsets = (const int32_t*)(base + o_off);
   p.timeout_ns = d.wait_timeout_ns ? d.wait_timeout_ns : kDefaultTimeoutNs;
+  p.trace = tracing ? (uint64_t*)(base + o_trace) : nullptr;
+  const char* l2_env = getenv("MK_L2_AHEAD_KB");  // diagnostic knob: L2 prefetch window per SM
+  p.l2_ahead = l2_env ? (uint32_t)atoi(l2_env) * 1024u : mk::kDefaultL2AheadBytes;
   *out = h;
   return MK_OK;
 }
@@ -269,6 +277,7 @@ extern "C" size_t mk_state_bytes(const mk_handle* h, int which) {
   const mk_model_desc& d = h->d;
   switch (which) {
     case MK_STATE_HIDDEN: return sizeof(float) * (size_t)(2 * d.n_layers + 1) * d.batch * d.hidden;
+    case MK_STATE_TRACE: return sizeof(uint64_t) * mk::kTraceStamps * h->n_instr;
     default: return 0;
   }
 }
@@ -280,6 +289,7 @@ extern "C" int mk_read_state(mk_handle* h, int which, void* dst, size_t bytes, v
   if (bytes < need) return MK_ERR_INVALID_ARG;
   const void* src = nullptr;
   if (which == MK_STATE_HIDDEN) src = h->p.xres;
+  if (which == MK_STATE_TRACE) src = h->p.trace;
   if (cudaMemcpyAsync(dst, src, need, cudaMemcpyDefault, (cudaStream_t)stream) != cudaSuccess) return MK_ERR_CUDA;
   return MK_OK;
 }

@@ -45,6 +45,8 @@ struct Params {
   float* logits;            // [B][V]
   uint32_t epoch;
   uint64_t timeout_ns;
+  uint64_t* trace;          // [n_instr][kTraceStamps] timestamps, or nullptr
+  uint32_t l2_ahead;        // bytes the producer prefetches into L2 beyond its ring (0 = off)
 };
 
 // Dynamic shared memory of one CTA.

@@ -18,7 +18,7 @@ namespace mk {
 enum Op : int32_t {
   OP_NOP = 0,
   OP_EMBED = 1,    // a,b: hidden slice [a,b) of x0 = embed[token]
-  OP_QKV = 2,      // a,b: rows of matrix c (0 wq, 1 wk, 2 wv); RMSNorm(x_{2l}) prologue
+  OP_QKV = 2,      // a,b: rows of wq|wk|wv concatenated; RMSNorm(x_{2l}) prologue
   OP_ATTN = 3,     // a: sequence, b: kv head, c: chunk; last chunk of (a,b) merges
   OP_OPROJ = 4,    // a,b: rows of wo; x_{2l+1} = x_{2l} + wo . attn
   OP_GATEUP = 5,   // a,b: rows of w_gate/w_up; act = silu(g) * u; RMSNorm(x_{2l+1}) prologue
@@ -43,6 +43,8 @@ constexpr int kRedFloats = 4096;                       // cross-warp reduction b
 constexpr int kMaxBatch = 8;
 constexpr int kMaxGroup = 8;                           // query heads per KV head
 constexpr int kMaxHeadDim = 128;
+constexpr int kTraceStamps = 8;                        // per-instruction trace words
+constexpr uint32_t kDefaultL2AheadBytes = 0;  // L2 prefetch window beyond the ring (measured: no gain)
 
 // ---- dependency counters -----------------------------------------------------
 // Each counter is bumped once per producing instruction per step; a waiter
@@ -83,10 +85,26 @@ MK_HD GemvTile gemv_tile(int K, int n_mats) {
   t.rpp = kConsumerThreads / tpr;
   t.nv = (vt + tpr - 1) / tpr;
   int r = kStageBytes / (K * 2 * n_mats);
-  int cap = 8 * t.rpp;  // at most 8 rows per thread per stage
+  // rows per thread per stage: at most 16 / (vectors x matrices), so that the
+  // loads in flight and the accumulators stay within the register budget
+  const int nvp = t.nv > 2 ? 4 : t.nv > 1 ? 2 : 1;
+  int rpt = 16 / (nvp * n_mats);
+  if (rpt > 8) rpt = 8;
+  int cap = rpt * t.rpp;
   if (r > cap) r = cap;
   t.rows_per_stage = r;
   return t;
+}
+
+// Rows longer than 8 vectors per thread are streamed in ks column slices of
+// K/ks (each slice a separate pass over the same rows); 0 = unsupported.
+MK_HD int gemv_ksplit(int K, int n_mats) {
+  for (int ks = 1; ks <= 4; ks *= 2) {
+    if (K % (8 * ks)) break;
+    const GemvTile t = gemv_tile(K / ks, n_mats);
+    if (t.nv <= 8 && t.rows_per_stage >= 1) return ks;
+  }
+  return 0;
 }
 
 // ---- attention split -------------------------------------------------------------

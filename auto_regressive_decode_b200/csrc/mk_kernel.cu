@@ -150,6 +150,44 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Reduce R independent per-lane values over the 32 lanes of a warp with
+// R - 1 + 5 - log2(R) shuffles: each butterfly level halves the number of
+// values a lane carries (the lane keeps one half and receives its partner's
+// copy of that half), then plain xor levels finish the sum.  Afterwards lane l
+// holds the total of value index row_of_lane<R>(l) (lanes sharing the top
+// log2(R) bits hold the same total).
+template <int R>
+__device__ __forceinline__ float warp_reduce_multi(float (&v)[R], int lane) {
+  constexpr int LOG = R >= 16 ? 4 : R >= 8 ? 3 : R >= 4 ? 2 : R >= 2 ? 1 : 0;
+#pragma unroll
+  for (int lvl = 0; lvl < LOG; ++lvl) {
+    const int off = 16 >> lvl;
+    const int half = R >> (lvl + 1);
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < (R >> 1); ++k) {
+      if (k < half) {
+        const float send = up ? v[k] : v[k + half];
+        const float keep = up ? v[k + half] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      }
+    }
+  }
+  float s = v[0];
+#pragma unroll
+  for (int off = 16 >> LOG; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  return s;
+}
+
+template <int R>
+__device__ __forceinline__ int row_of_lane(int lane) {
+  constexpr int LOG = R >= 16 ? 4 : R >= 8 ? 3 : R >= 4 ? 2 : R >= 2 ? 1 : 0;
+  int r = 0;
+#pragma unroll
+  for (int lvl = 0; lvl < LOG; ++lvl) r |= ((lane >> (4 - lvl)) & 1) << (LOG - 1 - lvl);
+  return r;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
@@ -178,7 +216,7 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
-__device__ void set_status(const Params& p, int code, int detail) {
+__device__ __forceinline__ void set_status(const Params& p, int code, int detail) {
   if (atomicCAS(p.status, 0, code) == 0) {
     p.status[1] = detail;
     p.status[2] = blockIdx.x;
@@ -188,44 +226,74 @@ __device__ void set_status(const Params& p, int code, int detail) {
 // ---------------------------------------------------------------------------
 // Instruction geometry (identical on the producer and consumer side)
 // ---------------------------------------------------------------------------
+// A GEMV instruction covers rows [r0, r1) of its op's row space.  For QKV that
+// space is wq | wk | wv concatenated, so an instruction may span up to three
+// matrices ("segments"); a stage never crosses a segment.  Fields are named
+// (not arrays) so that the geometry stays in registers.
 struct Gemv {
-  const uint16_t* w0;  // first matrix, row 0
-  const uint16_t* w1;  // second matrix (gate/up pair) or nullptr
+  const uint16_t *sw0, *sw1, *sw2;  // first row of each segment
+  const uint16_t* wup;              // gate/up: first row of the up matrix (one segment)
+  int sn0, sn1, sn2, nseg;          // rows per segment
   int K, r0, r1;
-  GemvTile tile;
+  int ks, Kc;                       // column slices per row, slice width (K = ks * Kc)
+  GemvTile tile;                    // tiling of one slice
+  __device__ __forceinline__ const uint16_t* seg_ptr(int s) const { return s == 0 ? sw0 : (s == 1 ? sw1 : sw2); }
+  __device__ __forceinline__ int seg_rows(int s) const { return s == 0 ? sn0 : (s == 1 ? sn1 : sn2); }
 };
 
 __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, int op, int layer) {
   Gemv g;
-  g.w1 = nullptr;
+  g.wup = nullptr;
   g.r0 = in.a;
   g.r1 = in.b;
+  g.nseg = 1;
+  g.sn0 = g.r1 - g.r0;
+  g.sn1 = g.sn2 = 0;
+  g.sw1 = g.sw2 = nullptr;
   if (op == OP_LMHEAD) {
-    g.w0 = p.lm_head;
     g.K = p.H;
+    g.sw0 = p.lm_head + (size_t)g.r0 * g.K;
   } else {
     const LayerPtrs& lp = p.layers[layer];
     switch (op) {
-      case OP_QKV:
-        g.w0 = in.c == 0 ? lp.wq : (in.c == 1 ? lp.wk : lp.wv);
+      case OP_QKV: {
         g.K = p.H;
+        const int qd = p.nq * p.hd, kvd = p.nkv * p.hd;
+        g.nseg = 0;
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          const int base = m == 0 ? 0 : (m == 1 ? qd : qd + kvd);
+          const int end = m == 0 ? qd : (m == 1 ? qd + kvd : qd + 2 * kvd);
+          const uint16_t* mat = m == 0 ? lp.wq : (m == 1 ? lp.wk : lp.wv);
+          const int a = max(g.r0, base), b = min(g.r1, end);
+          if (a < b) {
+            const uint16_t* w = mat + (size_t)(a - base) * g.K;
+            if (g.nseg == 0) { g.sw0 = w; g.sn0 = b - a; }
+            else if (g.nseg == 1) { g.sw1 = w; g.sn1 = b - a; }
+            else { g.sw2 = w; g.sn2 = b - a; }
+            ++g.nseg;
+          }
+        }
         break;
+      }
       case OP_OPROJ:
-        g.w0 = lp.wo;
         g.K = p.nq * p.hd;
+        g.sw0 = lp.wo + (size_t)g.r0 * g.K;
         break;
       case OP_GATEUP:
-        g.w0 = lp.w_gate;
-        g.w1 = lp.w_up;
         g.K = p.H;
+        g.sw0 = lp.w_gate + (size_t)g.r0 * g.K;
+        g.wup = lp.w_up + (size_t)g.r0 * g.K;
         break;
       default:  // OP_DOWN
-        g.w0 = lp.w_down;
         g.K = p.I;
+        g.sw0 = lp.w_down + (size_t)g.r0 * g.K;
         break;
     }
   }
-  g.tile = gemv_tile(g.K, g.w1 ? 2 : 1);
+  g.ks = gemv_ksplit(g.K, g.wup ? 2 : 1);
+  g.Kc = g.K / g.ks;
+  g.tile = gemv_tile(g.Kc, g.wup ? 2 : 1);
   return g;
 }
 
@@ -255,21 +323,122 @@ __device__ __forceinline__ Attn attn_geo(const Params& p, const mk_instr& in, in
 // ---------------------------------------------------------------------------
 // Producer warp (lane 0 issues everything)
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Walks the stages of an SM's instruction list in order.  A GEMV stage is R
+// rows (one column slice) of one segment, plus the same rows of the up matrix
+// for gate/up; an attention stage is up to P cached positions of K or of V.
+struct Cursor {
+  const Params* pp;  // pointer (not reference) so that cursors can be assigned
+  const mk_instr* list;
+  int n;
+  int i;  // instruction index; >= n when every stage has been walked
+  int op;
+  Gemv g;
+  int kc, sg, rr;  // GEMV: slice, segment, first row within the segment
+  Attn a;
+  int sub, kv;     // attention: sub-chunk, K (0) or V (1)
+
+  __device__ Cursor(const Params& prm, const mk_instr* l, int nn) : pp(&prm), list(l), n(nn), i(0) {}
+
+  // Position on the first stage of instruction j or of the next one that has stages.
+  __device__ __forceinline__ void seek(int j) {
+    for (i = j; i < n; ++i) {
+      const mk_instr in = list[i];
+      op = op_of(in.op_layer);
+      const int layer = layer_of(in.op_layer);
+      if (op == OP_ATTN) {
+        a = attn_geo(*pp, in, layer, pp->hd);
+        sub = kv = 0;
+        if (a.nsub > 0) return;
+      } else if (op >= OP_QKV && op <= OP_LMHEAD) {
+        g = gemv_geo(*pp, in, op, layer);
+        kc = sg = rr = 0;
+        return;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void advance() {
+    if (op == OP_ATTN) {
+      kv ^= 1;
+      if (!kv && ++sub >= a.nsub) seek(i + 1);
+      return;
+    }
+    rr += g.tile.rows_per_stage;
+    if (rr >= g.seg_rows(sg)) {
+      rr = 0;
+      if (++sg >= g.nseg) {
+        sg = 0;
+        if (++kc >= g.ks) seek(i + 1);
+      }
+    }
+  }
+
+  // f(src, bytes, smem offset) for every copy of the current stage; returns the stage's bytes.
+  template <typename F>
+  __device__ __forceinline__ uint32_t copies(F&& f) const {
+    if (op == OP_ATTN) {
+      const int np = min(a.P, a.n_cached - sub * a.P);
+      const uint32_t bytes = (uint32_t)np * pp->hd * 2u;
+      f((kv ? pp->vc : pp->kc) + a.cache_base + (size_t)sub * a.P * pp->hd, bytes, 0u);
+      return bytes;
+    }
+    const int R = g.tile.rows_per_stage;
+    const int nr = min(R, g.seg_rows(sg) - rr);
+    const uint32_t seg = (uint32_t)g.Kc * 2u;
+    const size_t off = (size_t)rr * g.K + (size_t)kc * g.Kc;
+    const uint32_t bytes = (uint32_t)nr * seg;
+    for (int m = 0; m < (g.wup ? 2 : 1); ++m) {
+      const uint16_t* src = (m ? g.wup : g.seg_ptr(sg)) + off;
+      const uint32_t base = (uint32_t)m * R * seg;
+      if (g.ks == 1) {
+        f(src, bytes, base);
+      } else {
+        for (int r = 0; r < nr; ++r) f(src + (size_t)r * g.K, seg, base + r * seg);
+      }
+    }
+    return g.wup ? 2 * bytes : bytes;
+  }
+
+  __device__ __forceinline__ uint32_t stage_bytes() const {
+    if (op == OP_ATTN) return (uint32_t)min(a.P, a.n_cached - sub * a.P) * pp->hd * 2u;
+    const uint32_t b = (uint32_t)min(g.tile.rows_per_stage, g.seg_rows(sg) - rr) * (uint32_t)g.Kc * 2u;
+    return g.wup ? 2 * b : b;
+  }
+};
+
 struct Producer {
   const Params& p;
   Ctl* ctl;
   uint8_t* ring;
   uint64_t pol;
   uint32_t k = 0;  // stages issued
+  Cursor pf;       // L2 prefetch cursor, pf_ahead bytes past the issue cursor
+  uint32_t pf_ahead = 0;
 
-  __device__ Producer(const Params& pp, Ctl* c, uint8_t* r) : p(pp), ctl(c), ring(r) { pol = evict_first_policy(); }
+  __device__ Producer(const Params& pp, Ctl* c, uint8_t* r, const mk_instr* l, int nn)
+      : p(pp), ctl(c), ring(r), pf(pp, l, nn) {
+    pol = evict_first_policy();
+  }
+
+  // While blocked on the ring: prefetch the next stages into L2, up to Params::l2_ahead bytes.
+  __device__ __forceinline__ void prefetch_ahead() {
+    while (pf_ahead < p.l2_ahead && pf.i < pf.n) {
+      pf_ahead += pf.copies([&](const uint16_t* src, uint32_t bytes, uint32_t) { prefetch_l2(src, bytes); });
+      pf.advance();
+    }
+  }
 
   // Claim the next slot (waiting until the consumers released it).
-  __device__ bool claim(uint8_t** dst, unsigned long long** bar) {
+  __device__ __forceinline__ bool claim(uint8_t** dst, unsigned long long** bar) {
     const int slot = k % kStages;
     if (k >= (uint32_t)kStages) {
       const uint32_t parity = ((k / kStages) - 1) & 1;
       if (!mbar_try_wait(&ctl->empty[slot], parity)) {
+        prefetch_ahead();
         const uint64_t t0 = globaltimer();
         uint32_t spins = 0;
         while (!mbar_try_wait(&ctl->empty[slot], parity)) {
@@ -289,42 +458,8 @@ struct Producer {
     return true;
   }
 
-  __device__ bool gemv(const Gemv& g) {
-    const int R = g.tile.rows_per_stage;
-    const uint32_t row_bytes = (uint32_t)g.K * 2u;
-    for (int r = g.r0; r < g.r1; r += R) {
-      const int n = min(R, g.r1 - r);
-      uint8_t* dst;
-      unsigned long long* bar;
-      if (!claim(&dst, &bar)) return false;
-      const uint32_t bytes = (uint32_t)n * row_bytes;
-      mbar_arrive_expect_tx(bar, g.w1 ? 2 * bytes : bytes);
-      bulk_g2s(dst, g.w0 + (size_t)r * g.K, bytes, bar, pol);
-      if (g.w1) bulk_g2s(dst + (size_t)R * row_bytes, g.w1 + (size_t)r * g.K, bytes, bar, pol);
-      ++k;
-    }
-    return true;
-  }
-
-  __device__ bool attn(const Attn& a, int hd) {
-    for (int s = 0; s < a.nsub; ++s) {
-      const int np = min(a.P, a.n_cached - s * a.P);
-      const uint32_t bytes = (uint32_t)np * hd * 2u;
-      const size_t off = a.cache_base + (size_t)s * a.P * hd;
-      for (int kv = 0; kv < 2; ++kv) {
-        uint8_t* dst;
-        unsigned long long* bar;
-        if (!claim(&dst, &bar)) return false;
-        mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(dst, (kv == 0 ? p.kc : p.vc) + off, bytes, bar, pol);
-        ++k;
-      }
-    }
-    return true;
-  }
-
   // After giving up: wait (bounded) for the copies still in flight.
-  __device__ void drain() {
+  __device__ __forceinline__ void drain() {
     const uint32_t first = k > (uint32_t)kStages ? k - kStages : 0;
     for (uint32_t j = first; j < k; ++j) {
       const uint64_t t0 = globaltimer();
@@ -335,27 +470,37 @@ struct Producer {
   }
 };
 
-__device__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
-  Producer pr(p, ctl, ring);
+__device__ __forceinline__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
+  Producer pr(p, ctl, ring, list, n);
+  uint64_t* trace = p.trace ? p.trace + (size_t)p.offsets[blockIdx.x] * kTraceStamps : nullptr;
+  Cursor cur(p, list, n);
+  cur.seek(0);
+  pr.pf = cur;
   bool ok = true;
-  for (int i = 0; i < n && ok; ++i) {
-    const mk_instr in = list[i];
-    const int op = op_of(in.op_layer), layer = layer_of(in.op_layer);
-    switch (op) {
-      case OP_QKV:
-      case OP_OPROJ:
-      case OP_GATEUP:
-      case OP_DOWN:
-      case OP_LMHEAD:
-        ok = pr.gemv(gemv_geo(p, in, op, layer));
-        break;
-      case OP_ATTN:
-        ok = pr.attn(attn_geo(p, in, layer, p.hd), p.hd);
-        break;
-      default:
-        break;
+  int last = -1;
+  while (cur.i < n) {
+    if (trace && cur.i != last) {
+      const uint64_t now = globaltimer();
+      if (last >= 0) trace[last * kTraceStamps + 7] = now;
+      for (int j = last + 1; j <= cur.i; ++j) trace[j * kTraceStamps + 3] = now;
+      last = cur.i;
+    }
+    uint8_t* dst;
+    unsigned long long* bar;
+    if (!(ok = pr.claim(&dst, &bar))) break;
+    const uint32_t bytes = cur.stage_bytes();
+    mbar_arrive_expect_tx(bar, bytes);
+    cur.copies([&](const uint16_t* src, uint32_t b, uint32_t off) { bulk_g2s(dst + off, src, b, bar, pr.pol); });
+    ++pr.k;
+    cur.advance();
+    if (pr.pf_ahead > bytes) {
+      pr.pf_ahead -= bytes;
+    } else {
+      pr.pf = cur;
+      pr.pf_ahead = 0;
     }
   }
+  if (trace && last >= 0) trace[last * kTraceStamps + 7] = globaltimer();
   if (!ok) {
     ctl->dead = 1;
     pr.drain();
@@ -371,6 +516,7 @@ struct Consumer {
   uint8_t* ring;
   float* red;
   uint32_t k = 0;  // stages consumed
+  uint64_t* tr = nullptr;  // this instruction's trace stamps (thread 0, tracing only)
   const int t = threadIdx.x;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -380,9 +526,9 @@ struct Consumer {
   // Wait until slot k holds its data.  Never changes control flow: on a
   // timeout it marks the CTA dead and returns, and the caller carries on
   // until the next uniform decision point.
-  __device__ const uint8_t* wait_full() { return wait_stage(k); }
+  __device__ __forceinline__ const uint8_t* wait_full() { return wait_stage(k); }
 
-  __device__ const uint8_t* wait_stage(uint32_t kk) {
+  __device__ __forceinline__ const uint8_t* wait_stage(uint32_t kk) {
     const int slot = kk % kStages;
     const uint32_t parity = (kk / kStages) & 1;
     if (!mbar_try_wait(&ctl->full[slot], parity)) {
@@ -400,14 +546,14 @@ struct Consumer {
     return ring + (size_t)slot * kStageBytes;
   }
 
-  __device__ void release() {
+  __device__ __forceinline__ void release() {
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl->empty[k % kStages]);
     ++k;
   }
 
   // Dependency wait on `idx` reaching epoch * count.  Uniform result.
-  __device__ bool wait_counter(int idx, int count) {
+  __device__ __forceinline__ bool wait_counter(int idx, int count) {
     bool fail = false;
     if (idx >= 0 && t == 0) {
       const uint32_t target = p.epoch * (uint32_t)count;
@@ -433,7 +579,7 @@ struct Consumer {
     return !consumer_bar_or(fail);
   }
 
-  __device__ void signal(int idx) {
+  __device__ __forceinline__ void signal(int idx) {
     consumer_bar();
     if (t == 0 && idx >= 0) {
       __threadfence();
@@ -442,7 +588,7 @@ struct Consumer {
   }
 
   // Block-wide sum over the 256 consumer threads (result in every thread).
-  __device__ float block_sum(float v) {
+  __device__ __forceinline__ float block_sum(float v) {
     v = warp_sum(v);
     consumer_bar();
     if (lane == 0) ctl->sred[warp] = v;
@@ -454,7 +600,7 @@ struct Consumer {
   }
 
   // ---- embedding ------------------------------------------------------------
-  __device__ void embed(const mk_instr& in) {
+  __device__ __forceinline__ void embed(const mk_instr& in) {
     for (int b = 0; b < p.B; ++b) {
       const uint16_t* row = p.embed + (size_t)p.tokens[b] * p.H;
       float* x = p.xres + (size_t)b * p.H;
@@ -465,22 +611,25 @@ struct Consumer {
   // ---- GEMV ------------------------------------------------------------------
   // Input vector x (fp32, written by other CTAs) optionally RMS-normalised
   // with a bf16 gain; each thread keeps its NVT vectors in registers.
-  template <int NVT>
-  __device__ __forceinline__ void load_x(const float* src, const uint16_t* gain, int K, const GemvTile& tl, float xr[NVT][8]) {
-    float scale = 1.f;
-    if (gain) {
-      float ss = 0.f;
-      for (int i = t; i < K / 4; i += kConsumerThreads) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src) + i);
-        ss = fmaf(v.x, v.x, ss);
-        ss = fmaf(v.y, v.y, ss);
-        ss = fmaf(v.z, v.z, ss);
-        ss = fmaf(v.w, v.w, ss);
-      }
-      ss = block_sum(ss);
-      scale = 1.f / sqrtf(ss / (float)K + p.eps);
-    }
+  // Gains of the RMSNorm prologue are weights: fetch them before the dependency wait.
+  template <int NVT, bool NORM>
+  __device__ __forceinline__ void load_gain(const uint16_t* gain, int K, const GemvTile& tl, uint4 graw[NVT]) {
     const int ct = t % tl.tpr, vt = K / 8;
+#pragma unroll
+    for (int j = 0; j < NVT; ++j) {
+      const int v = ct + j * tl.tpr;
+      graw[j] = NORM && v < vt ? __ldg(reinterpret_cast<const uint4*>(gain + v * 8)) : make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  template <int NVT, bool NORM>
+  __device__ __forceinline__ void load_x(const float* src, const uint4 graw[NVT], int K, const GemvTile& tl,
+                                         float xr[NVT][8]) {
+    // One pass: every group of tpr threads holds all of x, so the block sum
+    // of the per-thread squares counts each element rpp times (a power of 2).
+    const int ct = t % tl.tpr, vt = K / 8;
+
+    float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < NVT; ++j) {
       const int v = ct + j * tl.tpr;
@@ -489,55 +638,87 @@ struct Consumer {
         const float4 b = __ldcg(reinterpret_cast<const float4*>(src + v * 8) + 1);
         xr[j][0] = a.x; xr[j][1] = a.y; xr[j][2] = a.z; xr[j][3] = a.w;
         xr[j][4] = b.x; xr[j][5] = b.y; xr[j][6] = b.z; xr[j][7] = b.w;
-        if (gain) {
-          float g[8];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(gain + v * 8)), g);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xr[j][e] = xr[j][e] * scale * g[e];
-        }
       } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
       }
+      if (NORM) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
+      }
+    }
+    if (NORM) {
+      ss = block_sum(ss) / (float)tl.rpp;
+      const float scale = 1.f / sqrtf(ss / (float)K + p.eps);
+#pragma unroll
+      for (int j = 0; j < NVT; ++j)
+        if (ct + j * tl.tpr < vt) {
+          float gf[8];
+          unpack8(graw[j], gf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xr[j][e] = xr[j][e] * scale * gf[e];
+        }
     }
   }
 
   // Stream the instruction's stages, leaving per-(row, warp) partial dots in red.
-  template <int NVT, bool GATED>
-  __device__ __forceinline__ void gemv_stream(const Gemv& g, const float xr[NVT][8]) {
+  // Each thread accumulates RPT rows of the stage (rows rs, rs+rpp, ...) and
+  // the warp reduces all of them at once with warp_reduce_multi.
+  template <int NVT, int RPT, bool GATED>
+  __device__ __forceinline__ void gemv_stream(const Gemv& g, const float xr[NVT][8], int kc) {
+    constexpr int NM = GATED ? 2 : 1;
     const GemvTile& tl = g.tile;
-    const int R = tl.rows_per_stage, K = g.K, vt = K / 8;
+    const int R = tl.rows_per_stage, K = g.Kc, vt = K / 8;
     const int rs = t / tl.tpr, ct = t % tl.tpr, wpr = tl.tpr / 32, wir = ct / 32;
-    const int nm = GATED ? 2 : 1;
-    for (int r = g.r0; r < g.r1; r += R) {
-      const int n = min(R, g.r1 - r);
+    const int q = row_of_lane<RPT * NM>(lane);
+    const bool writer = (lane & (32 / (RPT * NM) - 1)) == 0;
+    int rl = 0;  // first row of the segment within the instruction
+#pragma unroll 1
+    for (int sg = 0; sg < g.nseg; ++sg) {
+      const int nr = g.seg_rows(sg);
+#pragma unroll 1
+    for (int rr = 0; rr < nr; rr += R) {
+      const int n = min(R, nr - rr);
       const uint16_t* w0 = reinterpret_cast<const uint16_t*>(wait_full());
+      if (tr && kc == 0 && sg == 0 && rr == 0) tr[5] = globaltimer();
       const uint16_t* w1 = w0 + (size_t)R * K;
-      for (int i = rs; i < n; i += tl.rpp) {
-        float a0 = 0.f, a1 = 0.f;
+      float acc[RPT * NM];
 #pragma unroll
-        for (int j = 0; j < NVT; ++j) {
-          const int v = ct + j * tl.tpr;
-          if (v < vt) {
-            a0 = dot8(*reinterpret_cast<const uint4*>(w0 + (size_t)i * K + v * 8), xr[j], a0);
-            if (GATED) a1 = dot8(*reinterpret_cast<const uint4*>(w1 + (size_t)i * K + v * 8), xr[j], a1);
+      for (int k = 0; k < RPT; ++k) {
+        const int i = rs + k * tl.rpp;
+        float a0 = 0.f, a1 = 0.f;
+        if (i < n) {
+#pragma unroll
+          for (int j = 0; j < NVT; ++j) {
+            const int v = ct + j * tl.tpr;
+            if (v < vt) {
+              a0 = dot8(*reinterpret_cast<const uint4*>(w0 + (size_t)i * K + v * 8), xr[j], a0);
+              if (GATED) a1 = dot8(*reinterpret_cast<const uint4*>(w1 + (size_t)i * K + v * 8), xr[j], a1);
+            }
           }
         }
-        a0 = warp_sum(a0);
-        if (GATED) a1 = warp_sum(a1);
-        if (lane == 0) {
-          const int rl = r - g.r0 + i;
-          red[(rl * nm) * wpr + wir] = a0;
-          if (GATED) red[(rl * nm + 1) * wpr + wir] = a1;
+        acc[k] = a0;
+        if (GATED) acc[RPT + k] = a1;
+      }
+      const float sum = warp_reduce_multi<RPT * NM>(acc, lane);
+      if (writer) {
+        const int k = q % RPT, which = q / RPT;
+        const int i = rs + k * tl.rpp;
+        if (i < n) {
+          float* dst = red + ((rl + rr + i) * NM + which) * wpr + wir;
+          *dst = (kc ? *dst : 0.f) + sum;  // the same thread owns this slot in every slice pass
         }
       }
       release();
     }
+      rl += nr;
+    }
+    if (tr) tr[6] = globaltimer();
     consumer_bar();
   }
 
-  template <int NVT>
-  __device__ __forceinline__ void gemv_run(const mk_instr& in, int op, int layer) {
+  template <int NVT, int RPT, bool NORM, bool GATED>
+  __device__ __forceinline__ bool gemv_run(const mk_instr& in, int op, int layer) {
     const Gemv g = gemv_geo(p, in, op, layer);
     const int BH = p.B * p.H;
     // input vector and prologue
@@ -557,17 +738,25 @@ struct Consumer {
       src = p.xres + (size_t)(2 * p.L) * BH;
       gain = p.final_norm;
     }
-    float xr[NVT][8];
-    load_x<NVT>(src, gain, g.K, g.tile, xr);
-    if (op == OP_GATEUP)
-      gemv_stream<NVT, true>(g, xr);
-    else
-      gemv_stream<NVT, false>(g, xr);
+    uint4 graw[NVT];
+    load_gain<NVT, NORM>(gain, g.Kc, g.tile, graw);
+    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
+    if (tr) tr[1] = globaltimer();
+    // residual rows for the epilogue, fetched before the weights stream
+    float resid = 0.f;
+    if ((op == OP_OPROJ || op == OP_DOWN) && t < g.r1 - g.r0)
+      resid = __ldcg(p.xres + (size_t)(2 * layer + (op == OP_DOWN ? 1 : 0)) * BH + g.r0 + t);
+    for (int kc = 0; kc < g.ks; ++kc) {  // ks > 1 only without a norm prologue
+      float xr[NVT][8];
+      load_x<NVT, NORM>(src + (size_t)kc * g.Kc, graw, g.Kc, g.tile, xr);
+      if (tr && kc == 0) tr[4] = globaltimer();
+      gemv_stream<NVT, RPT, GATED>(g, xr, kc);
+    }
     // epilogue: fixed-order sum of the per-warp partials, then the op's output
     const int wpr = g.tile.tpr / 32, n = g.r1 - g.r0;
     for (int i = t; i < n; i += kConsumerThreads) {
       const int row = g.r0 + i;
-      if (op == OP_GATEUP) {
+      if (GATED) {
         float gs = 0.f, us = 0.f;
         for (int w = 0; w < wpr; ++w) {
           gs += red[(i * 2) * wpr + w];
@@ -579,30 +768,47 @@ struct Consumer {
       float y = 0.f;
       for (int w = 0; w < wpr; ++w) y += red[i * wpr + w];
       if (op == OP_QKV) {
-        const int qd = p.nq * p.hd, kvd = p.nkv * p.hd;
-        const int off = in.c == 0 ? 0 : (in.c == 1 ? qd : qd + kvd);
-        p.qkv[off + row] = y;
+        p.qkv[row] = y;  // q | k | v concatenated, like the instruction's rows
       } else if (op == OP_OPROJ) {
-        p.xres[(size_t)(2 * layer + 1) * BH + row] = __ldcg(p.xres + (size_t)(2 * layer) * BH + row) + y;
+        p.xres[(size_t)(2 * layer + 1) * BH + row] = resid + y;
       } else if (op == OP_DOWN) {
-        p.xres[(size_t)(2 * layer + 2) * BH + row] = __ldcg(p.xres + (size_t)(2 * layer + 1) * BH + row) + y;
+        p.xres[(size_t)(2 * layer + 2) * BH + row] = resid + y;
       } else {
         p.logits[row] = y;
       }
     }
+    return true;
   }
 
-  __device__ void gemv(const mk_instr& in, int op, int layer) {
+  // gemv_tile caps rows per thread at 16 / (NVT * matrices), at most 8.
+  template <int NVT, bool NORM, bool GATED>
+  __device__ __forceinline__ bool gemv_nv(const mk_instr& in, int op, int layer, int rpt) {
+    constexpr int CAP = 16 / (NVT * (GATED ? 2 : 1)) > 8 ? 8 : 16 / (NVT * (GATED ? 2 : 1));
+    if (rpt <= 1 || CAP == 1) return gemv_run<NVT, 1, NORM, GATED>(in, op, layer);
+    if (rpt <= 2 || CAP == 2) return gemv_run<NVT, 2, NORM, GATED>(in, op, layer);
+    if (rpt <= 4 || CAP == 4) return gemv_run<NVT, (CAP < 4 ? CAP : 4), NORM, GATED>(in, op, layer);
+    return gemv_run<NVT, CAP, NORM, GATED>(in, op, layer);
+  }
+
+  template <bool NORM, bool GATED>
+  __device__ __forceinline__ bool gemv_nvsel(const mk_instr& in, int op, int layer, int nv, int rpt) {
+    if (nv <= 1) return gemv_nv<1, NORM, GATED>(in, op, layer, rpt);
+    if (nv <= 2) return gemv_nv<2, NORM, GATED>(in, op, layer, rpt);
+    if (NORM || nv <= 4) return gemv_nv<4, NORM, GATED>(in, op, layer, rpt);
+    return gemv_nv<(NORM ? 4 : 8), NORM, GATED>(in, op, layer, rpt);
+  }
+
+  // Ops with an RMSNorm prologue read the hidden vector (K = hidden, at most
+  // 4 vectors per thread, checked at creation); o_proj and down read attn / act.
+  __device__ __forceinline__ bool gemv(const mk_instr& in, int op, int layer) {
+    const bool norm = op == OP_QKV || op == OP_GATEUP || op == OP_LMHEAD;
     const int K = op == OP_OPROJ ? p.nq * p.hd : (op == OP_DOWN ? p.I : p.H);
-    const int nv = gemv_tile(K, op == OP_GATEUP ? 2 : 1).nv;
-    if (nv <= 1)
-      gemv_run<1>(in, op, layer);
-    else if (nv <= 2)
-      gemv_run<2>(in, op, layer);
-    else if (nv <= 4)
-      gemv_run<4>(in, op, layer);
-    else
-      gemv_run<8>(in, op, layer);
+    const int nm = op == OP_GATEUP ? 2 : 1;
+    const GemvTile tl = gemv_tile(K / gemv_ksplit(K, nm), nm);
+    const int rpt = (tl.rows_per_stage + tl.rpp - 1) / tl.rpp;
+    if (op == OP_GATEUP) return gemv_nvsel<true, true>(in, op, layer, tl.nv, rpt);
+    if (norm) return gemv_nvsel<true, false>(in, op, layer, tl.nv, rpt);
+    return gemv_nvsel<false, false>(in, op, layer, tl.nv, rpt);
   }
 
   // ---- attention ---------------------------------------------------------------
@@ -612,24 +818,32 @@ struct Consumer {
   // result is an unnormalised partial (o, m, l) in log2 units; the last
   // chunk of the (sequence, KV head) to finish merges all partials.
   template <int HD, int G>
-  __device__ __forceinline__ void attn_run(const mk_instr& in, int layer, int sig_idx) {
+  __device__ __forceinline__ bool attn_run(const mk_instr& in, int layer, int sig_idx) {
     constexpr int LPP = HD / 8;    // lanes per position (16-byte vectors)
     constexpr int PPW = 32 / LPP;  // positions per warp pass
+    constexpr int NP = HD / 64;    // rotation pairs per lane
     const Attn a = attn_geo(p, in, layer, HD);
     const int qd = p.nq * HD, kvd = p.nkv * HD;
     const float* qkv = p.qkv + (size_t)a.b * (qd + 2 * kvd);
     const float qscale = 1.4426950408889634f * rsqrtf((float)HD);  // log2(e) / sqrt(hd)
     const int pl = lane / LPP, vi = lane % LPP;
+    // RoPE table entries do not depend on this step's activations: fetch
+    // them before the dependency wait.
+    float2 csr[NP];
+    if (a.active) {
+      const float2* cs = p.rope + (size_t)p.positions[a.b] * (HD / 2);
+#pragma unroll
+      for (int j = 0; j < NP; ++j) csr[j] = __ldg(cs + lane + 32 * j);
+    }
+    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
+    if (tr) tr[1] = globaltimer();
     if (a.active) {
       // -- prologue: q heads (qk-norm, RoPE, scale) and the new K/V row
-      const int pos = p.positions[a.b];
-      const float2* cs = p.rope + (size_t)pos * (HD / 2);
       const int tasks = G + (a.owns_new ? 2 : 0);
       for (int task = warp; task < tasks; task += kConsumerWarps) {
         const bool is_v = task == G + 1;
         const float* src = task < G ? qkv + (a.kvh * G + task) * HD
                                     : qkv + qd + (is_v ? kvd : 0) + a.kvh * HD;
-        constexpr int NP = HD / 64;  // rotation pairs per lane
         float lo[NP], hi[NP];
         float ss = 0.f;
 #pragma unroll
@@ -642,16 +856,16 @@ struct Consumer {
           if (p.qk_norm) {
             ss = warp_sum(ss);
             const float sc = 1.f / sqrtf(ss / (float)HD + p.eps);
-            const uint16_t* gn = task < G ? p.layers[layer].q_norm : p.layers[layer].k_norm;
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
+              const uint16_t* gn = task < G ? p.layers[layer].q_norm : p.layers[layer].k_norm;
               lo[j] = lo[j] * sc * bf16_bits_to_f32(gn[lane + 32 * j]);
               hi[j] = hi[j] * sc * bf16_bits_to_f32(gn[lane + 32 * j + HD / 2]);
             }
           }
 #pragma unroll
           for (int j = 0; j < NP; ++j) {
-            const float2 r = cs[lane + 32 * j];
+            const float2 r = csr[j];
             const float x0 = lo[j], x1 = hi[j];
             lo[j] = x0 * r.x - x1 * r.y;
             hi[j] = x1 * r.x + x0 * r.y;
@@ -678,6 +892,7 @@ struct Consumer {
         }
       }
       consumer_bar();
+      if (tr) tr[4] = globaltimer();
       // q stays in registers up to 4 heads per KV head; with 8 it is read
       // from shared memory (a broadcast across position groups) so that the
       // 8 x 8 running outputs fit the 168-register budget of a 9-warp CTA.
@@ -699,6 +914,7 @@ struct Consumer {
         const int np = min(a.P, a.n_cached - s * a.P);
         const uint16_t* Ks = reinterpret_cast<const uint16_t*>(wait_stage(k));
         const uint16_t* Vs = reinterpret_cast<const uint16_t*>(wait_stage(k + 1));
+        if (tr && s == 0) tr[5] = globaltimer();
         for (int tb = warp * PPW; tb < np; tb += kConsumerWarps * PPW) {
           const int tp = tb + pl;
           const bool valid = tp < np;
@@ -735,6 +951,7 @@ struct Consumer {
         release();  // K slot
         release();  // V slot
       }
+      if (tr) tr[6] = globaltimer();
       // -- the new token (warp 0, first position group)
       if (a.owns_new && warp == 0) {
         float kf[8], vf[8];
@@ -821,71 +1038,98 @@ struct Consumer {
     }
     consumer_bar();
     if (ctl->last) {
+      // (m, l) of every (head, chunk) into shared memory with one parallel
+      // pass, then each output element reads its chunks' o with independent loads
       const int nvalid = a.S / p.chunk + 1;  // chunks holding a position <= S
+      const size_t pg = ((size_t)a.b * p.nq + (size_t)a.kvh * G) * p.n_chunks;
+      for (int idx = t; idx < G * nvalid; idx += kConsumerThreads) {
+        const int h = idx / nvalid, c = idx % nvalid;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml) + pg + (size_t)h * p.n_chunks + c);
+        red[2 * idx] = ml.x;
+        red[2 * idx + 1] = ml.y;
+      }
+      consumer_bar();
       for (int idx = t; idx < G * HD; idx += kConsumerThreads) {
         const int h = idx / HD, d = idx % HD;
-        const size_t pi0 = ((size_t)a.b * p.nq + (size_t)a.kvh * G + h) * p.n_chunks;
+        const float* ml = red + 2 * h * nvalid;
         float M = -1e30f;
-        for (int c = 0; c < nvalid; ++c) M = fmaxf(M, __ldcg(p.part_ml + (pi0 + c) * 2));
+        for (int c = 0; c < nvalid; ++c) M = fmaxf(M, ml[2 * c]);
+        const float* po = p.part_o + (pg + (size_t)h * p.n_chunks) * HD + d;
         float den = 0.f, num = 0.f;
+#pragma unroll 8
         for (int c = 0; c < nvalid; ++c) {
-          const float w = exp2f(__ldcg(p.part_ml + (pi0 + c) * 2) - M);
-          den = fmaf(w, __ldcg(p.part_ml + (pi0 + c) * 2 + 1), den);
-          num = fmaf(w, __ldcg(p.part_o + (pi0 + c) * HD + d), num);
+          const float w = exp2f(ml[2 * c] - M);
+          den = fmaf(w, ml[2 * c + 1], den);
+          num = fmaf(w, __ldcg(po + (size_t)c * HD), num);
         }
         p.attn[(size_t)a.b * qd + (size_t)(a.kvh * G + h) * HD + d] = num / den;
       }
       signal(sig_idx);
     }
+    return true;
   }
 
-  __device__ void attn(const mk_instr& in, int layer, int sig_idx) {
+  __device__ __forceinline__ bool attn(const mk_instr& in, int layer, int sig_idx) {
     const int G = p.nq / p.nkv;
     if (p.hd == 128) {
       switch (G) {
-        case 1: attn_run<128, 1>(in, layer, sig_idx); break;
-        case 2: attn_run<128, 2>(in, layer, sig_idx); break;
-        case 4: attn_run<128, 4>(in, layer, sig_idx); break;
-        default: attn_run<128, 8>(in, layer, sig_idx); break;
+        case 1: return attn_run<128, 1>(in, layer, sig_idx);
+        case 2: return attn_run<128, 2>(in, layer, sig_idx);
+        case 4: return attn_run<128, 4>(in, layer, sig_idx);
+        default: return attn_run<128, 8>(in, layer, sig_idx);
       }
     } else {
       switch (G) {
-        case 1: attn_run<64, 1>(in, layer, sig_idx); break;
-        case 2: attn_run<64, 2>(in, layer, sig_idx); break;
-        case 4: attn_run<64, 4>(in, layer, sig_idx); break;
-        default: attn_run<64, 8>(in, layer, sig_idx); break;
+        case 1: return attn_run<64, 1>(in, layer, sig_idx);
+        case 2: return attn_run<64, 2>(in, layer, sig_idx);
+        case 4: return attn_run<64, 4>(in, layer, sig_idx);
+        default: return attn_run<64, 8>(in, layer, sig_idx);
       }
     }
   }
 };
 
-__device__ void run_consumers(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring, float* red) {
+__device__ __forceinline__ void run_consumers(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring, float* red) {
   Consumer cs(p, ctl, ring, red);
+  uint64_t* trace = p.trace && threadIdx.x == 0 ? p.trace + (size_t)p.offsets[blockIdx.x] * kTraceStamps : nullptr;
   for (int i = 0; i < n; ++i) {
     const mk_instr in = list[i];
     const int op = op_of(in.op_layer), layer = layer_of(in.op_layer);
-    if (!cs.wait_counter(in.wait_idx, in.wait_count)) {
-      ctl->dead = 1;
-      return;
-    }
+    cs.tr = trace ? trace + (size_t)i * kTraceStamps : nullptr;
+    if (trace) trace[i * kTraceStamps + 0] = globaltimer();
+    bool ok = true;
     switch (op) {
       case OP_EMBED:
-        cs.embed(in);
-        cs.signal(in.sig_idx);
+        ok = cs.wait_counter(in.wait_idx, in.wait_count);
+        if (ok) {
+          if (trace) trace[i * kTraceStamps + 1] = globaltimer();
+          cs.embed(in);
+          if (trace) trace[i * kTraceStamps + 2] = globaltimer();
+          cs.signal(in.sig_idx);
+        }
         break;
       case OP_QKV:
       case OP_OPROJ:
       case OP_GATEUP:
       case OP_DOWN:
       case OP_LMHEAD:
-        cs.gemv(in, op, layer);
-        cs.signal(in.sig_idx);
+        ok = cs.gemv(in, op, layer);  // waits on the instruction's counter inside
+        if (ok) {
+          if (trace) trace[i * kTraceStamps + 2] = globaltimer();
+          cs.signal(in.sig_idx);
+        }
         break;
       case OP_ATTN:
-        cs.attn(in, layer, in.sig_idx);
+        ok = cs.attn(in, layer, in.sig_idx);
+        if (trace) trace[i * kTraceStamps + 2] = globaltimer();
         break;
       default:
+        ok = cs.wait_counter(in.wait_idx, in.wait_count);
         break;
+    }
+    if (!ok) {
+      ctl->dead = 1;
+      return;
     }
   }
 }

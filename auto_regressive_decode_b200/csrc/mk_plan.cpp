@@ -29,12 +29,10 @@ struct mk_plan {
 namespace mk {
 
 static bool aligned_ok(int K, int n_mats) {
-  // a full row (or a gate+up row pair) must fit one ring slot, and each
-  // thread holds at most 8 input vectors
+  // a row (or a gate+up row pair), possibly cut into column slices, must fit
+  // one ring slot with at most 4 input vectors per thread
   if (K <= 0 || K % 8) return false;
-  if ((int64_t)K * 2 * n_mats > kStageBytes) return false;
-  GemvTile t = gemv_tile(K, n_mats);
-  return t.nv <= 8 && t.rows_per_stage >= 1;
+  return gemv_ksplit(K, n_mats) > 0;
 }
 
 int validate_desc(const mk_model_desc* d) {
@@ -54,6 +52,8 @@ int validate_desc(const mk_model_desc* d) {
   const int qd = d->n_q_heads * d->head_dim;
   if (!aligned_ok(d->hidden, 1) || !aligned_ok(d->hidden, 2) || !aligned_ok(qd, 1) || !aligned_ok(d->ffn_dim, 1))
     return MK_ERR_UNSUPPORTED;
+  // GEMVs with an RMSNorm prologue (K = hidden) read whole rows in one pass
+  if (gemv_ksplit(d->hidden, 1) != 1 || gemv_ksplit(d->hidden, 2) != 1) return MK_ERR_UNSUPPORTED;
   if ((int64_t)d->max_ctx * d->head_dim > (1ll << 31)) return MK_ERR_UNSUPPORTED;
   return MK_OK;
 }
@@ -120,6 +120,9 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
   p->targets.assign(n_counters(L), 0);
   p->chunk = default_chunk(d, n_sm);
   p->n_chunks = (d->max_ctx + p->chunk - 1) / p->chunk;
+  // the merging CTA stages (m, l) of every (query head of the group, chunk) in
+  // its kRedFloats-float reduction buffer
+  if (2 * (d->n_q_heads / d->n_kv_heads) * p->n_chunks > kRedFloats) return MK_ERR_UNSUPPORTED;
   Builder b{p};
 
   // x0 = embedding rows, hidden dimension split over the SMs
@@ -136,7 +139,8 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
   for (int l = 0; l < L; ++l) {
     const int cq = counter_index(l, C_QKV), ca = counter_index(l, C_ATTN), co = counter_index(l, C_OPROJ);
     const int cg = counter_index(l, C_GATEUP), cd = counter_index(l, C_DOWN);
-    int n_qkv = b.rows_op(OP_QKV, l, qd + 2 * kvd, {qd, qd + kvd}, prev_idx, prev_count, cq);
+    // rows of wq | wk | wv concatenated; an instruction may span matrices
+    int n_qkv = b.rows_op(OP_QKV, l, qd + 2 * kvd, {}, prev_idx, prev_count, cq);
     p->targets[cq] = n_qkv;
     for (int s = 0; s < d->batch; ++s)
       for (int h = 0; h < d->n_kv_heads; ++h)

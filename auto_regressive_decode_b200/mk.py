@@ -24,6 +24,7 @@ MK_STATE_ROUTER = 1
 MK_STATE_SELECTION = 2
 MK_STATE_SEL_WEIGHT = 3
 MK_STATE_EXPERT_COUNT = 4
+MK_STATE_TRACE = 5
 
 OP_NAMES = {0: "nop", 1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead",
             8: "router", 9: "exp_gateup", 10: "exp_down"}
@@ -245,3 +246,15 @@ def weight_structs(cfg, weights, k_cache, v_cache):
                    None if lm is None else lm.data_ptr(), layers)
     kv = mk_kv(k_cache.data_ptr(), v_cache.data_ptr())
     return model_desc(cfg), w, kv, (layers, weights, k_cache, v_cache)
+
+
+def decoder_trace(dec):
+    """int64 [n_instr][8] timestamps of the last step (handle created with MK_TRACE=1)."""
+    import torch
+    n = mk_state_bytes(dec.h, MK_STATE_TRACE)
+    if n == 0:
+        raise MkError(MK_ERR_INVALID_ARG, "handle was not created with MK_TRACE=1")
+    out = torch.empty(n // 8, dtype=torch.int64, device="cuda")
+    dec.read_state(MK_STATE_TRACE, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().reshape(-1, 8)

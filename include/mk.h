@@ -125,13 +125,21 @@ const char* mk_status_string(int status);
  *   MK_STATE_ROUTER      float[n_layers][batch][n_experts] router logits (MoE)
  *   MK_STATE_SELECTION   int32[n_layers][batch][top_k] chosen experts (MoE)
  *   MK_STATE_SEL_WEIGHT  float[n_layers][batch][top_k] their weights (MoE)
- *   MK_STATE_EXPERT_COUNT int32[n_layers] distinct experts used (MoE) */
+ *   MK_STATE_EXPERT_COUNT int32[n_layers] distinct experts used (MoE)
+ *   MK_STATE_TRACE       uint64[n_instr][8] per-instruction %globaltimer stamps
+ *                        (ns) of the last step, in mk_plan_copy order: consumer
+ *                        start, dependency satisfied, compute done, producer's
+ *                        first copy issued, prologue done, first stage landed,
+ *                        last stage consumed, producer's last copy issued.
+ *                        Only for handles created with the environment variable
+ *                        MK_TRACE=1 (0 bytes otherwise). */
 enum {
   MK_STATE_HIDDEN = 0,
   MK_STATE_ROUTER = 1,
   MK_STATE_SELECTION = 2,
   MK_STATE_SEL_WEIGHT = 3,
-  MK_STATE_EXPERT_COUNT = 4
+  MK_STATE_EXPERT_COUNT = 4,
+  MK_STATE_TRACE = 5
 };
 int mk_read_state(mk_handle* h, int which, void* dst, size_t bytes, void* stream);
 
