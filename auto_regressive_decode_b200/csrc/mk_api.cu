@@ -122,7 +122,8 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   h->epoch = 0;
   const int L = d.n_layers, B = d.batch, H = d.hidden, hd = d.head_dim, nq = d.n_q_heads, nkv = d.n_kv_heads;
   const size_t qd = (size_t)nq * hd, kvd = (size_t)nkv * hd;
-  h->n_tickets = (size_t)L * B * nkv;
+  const int group = nq / nkv;
+  h->n_tickets = (size_t)L * B * nkv * (group / mk::attn_heads_per_instr(group));
 
   Carve cv;
   const size_t o_xres = cv.take(sizeof(float) * (size_t)(2 * L + 1) * B * H);
@@ -225,6 +226,8 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   p.trace = tracing ? (uint64_t*)(base + o_trace) : nullptr;
   const char* l2_env = getenv("MK_L2_AHEAD_KB");  // diagnostic knob: L2 prefetch window per SM
   p.l2_ahead = l2_env ? (uint32_t)atoi(l2_env) * 1024u : mk::kDefaultL2AheadBytes;
+  const char* piece_env = getenv("MK_COPY_PIECE_KB");  // diagnostic knob: bytes per bulk copy
+  p.copy_piece = piece_env && atoi(piece_env) > 0 ? (uint32_t)atoi(piece_env) * 1024u : mk::kDefaultCopyPiece;
   *out = h;
   return MK_OK;
 }

@@ -47,6 +47,7 @@ struct Params {
   uint64_t timeout_ns;
   uint64_t* trace;          // [n_instr][kTraceStamps] timestamps, or nullptr
   uint32_t l2_ahead;        // bytes the producer prefetches into L2 beyond its ring (0 = off)
+  uint32_t copy_piece;      // bytes per bulk copy (a multiple of 16); a stage is split into pieces
 };
 
 // Dynamic shared memory of one CTA.

@@ -19,7 +19,7 @@ enum Op : int32_t {
   OP_NOP = 0,
   OP_EMBED = 1,    // a,b: hidden slice [a,b) of x0 = embed[token]
   OP_QKV = 2,      // a,b: rows of wq|wk|wv concatenated; RMSNorm(x_{2l}) prologue
-  OP_ATTN = 3,     // a: sequence, b: kv head, c: chunk; last chunk of (a,b) merges
+  OP_ATTN = 3,     // a: sequence, b: kv head, c: chunk, d: head group; last chunk of (a,b,d) merges
   OP_OPROJ = 4,    // a,b: rows of wo; x_{2l+1} = x_{2l} + wo . attn
   OP_GATEUP = 5,   // a,b: rows of w_gate/w_up; act = silu(g) * u; RMSNorm(x_{2l+1}) prologue
   OP_DOWN = 6,     // a,b: rows of w_down; x_{2l+2} = x_{2l+1} + w_down . act
@@ -45,6 +45,7 @@ constexpr int kMaxGroup = 8;                           // query heads per KV hea
 constexpr int kMaxHeadDim = 128;
 constexpr int kTraceStamps = 8;                        // per-instruction trace words
 constexpr uint32_t kDefaultL2AheadBytes = 0;  // L2 prefetch window beyond the ring (measured: no gain)
+constexpr uint32_t kDefaultCopyPiece = 32 * 1024;  // bytes per bulk copy
 
 // ---- dependency counters -----------------------------------------------------
 // Each counter is bumped once per producing instruction per step; a waiter
@@ -108,6 +109,11 @@ MK_HD int gemv_ksplit(int K, int n_mats) {
 }
 
 // ---- attention split -------------------------------------------------------------
+// Query heads one attention instruction handles: a KV head with more query
+// heads than this is split into head groups, each a separate instruction
+// over the same cache chunk (keeps the per-thread accumulators in registers).
+MK_HD int attn_heads_per_instr(int group) { return group > 4 ? 4 : group; }
+
 // Positions of K (or V) that fit one ring slot.
 MK_HD int attn_stage_positions(int head_dim) { return kStageBytes / (head_dim * 2); }
 

@@ -40,12 +40,14 @@ struct Ctl {
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
   int dead;       // this CTA gives up: every wait returns at once
+  int waiting;    // consumers are blocked on a dependency counter (producer may prefetch)
   int last;       // attention: this CTA merges (broadcast)
   int flag;       // generic broadcast
   float sred[kConsumerWarps * 2];
   float qs[kMaxGroup * kMaxHeadDim];
-  float knew[kMaxHeadDim];
-  float vnew[kMaxHeadDim];
+  float aml[kConsumerWarps * kMaxGroup * 2];  // attention: per-warp (m, l) of every head
+  alignas(16) uint16_t knew[kMaxHeadDim];     // the new token's K/V rows (bf16, as appended)
+  alignas(16) uint16_t vnew[kMaxHeadDim];
 };
 
 constexpr size_t kRingBytes = (size_t)kStages * kStageBytes;
@@ -156,12 +158,16 @@ __device__ __forceinline__ float warp_sum(float v) {
 // copy of that half), then plain xor levels finish the sum.  Afterwards lane l
 // holds the total of value index row_of_lane<R>(l) (lanes sharing the top
 // log2(R) bits hold the same total).
-template <int R>
-__device__ __forceinline__ float warp_reduce_multi(float (&v)[R], int lane) {
-  constexpr int LOG = R >= 16 ? 4 : R >= 8 ? 3 : R >= 4 ? 2 : R >= 2 ? 1 : 0;
+__host__ __device__ constexpr int ilog2c(int x) { return x <= 1 ? 0 : 1 + ilog2c(x / 2); }
+
+// The same over groups of LPP consecutive lanes (R <= LPP): afterwards lane l
+// holds the group total of value index (l % LPP) >> (log2 LPP - log2 R).
+template <int R, int LPP>
+__device__ __forceinline__ float group_reduce_multi(float (&v)[R], int lane) {
+  constexpr int LOG = ilog2c(R);
 #pragma unroll
   for (int lvl = 0; lvl < LOG; ++lvl) {
-    const int off = 16 >> lvl;
+    const int off = (LPP / 2) >> lvl;
     const int half = R >> (lvl + 1);
     const bool up = (lane & off) != 0;
 #pragma unroll
@@ -175,8 +181,13 @@ __device__ __forceinline__ float warp_reduce_multi(float (&v)[R], int lane) {
   }
   float s = v[0];
 #pragma unroll
-  for (int off = 16 >> LOG; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  for (int off = (LPP / 2) >> LOG; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   return s;
+}
+
+template <int R>
+__device__ __forceinline__ float warp_reduce_multi(float (&v)[R], int lane) {
+  return group_reduce_multi<R, 32>(v, lane);
 }
 
 template <int R>
@@ -199,16 +210,18 @@ __device__ __forceinline__ void unpack8(const uint4 w, float f[8]) {
   f[6] = bf16_lo(w.w); f[7] = bf16_hi(w.w);
 }
 
+// 8-term dot product in two interleaved FMA chains (shorter dependency chain).
 __device__ __forceinline__ float dot8(const uint4 w, const float x[8], float acc) {
+  float b = 0.f;
   acc = fmaf(bf16_lo(w.x), x[0], acc);
-  acc = fmaf(bf16_hi(w.x), x[1], acc);
+  b = fmaf(bf16_hi(w.x), x[1], b);
   acc = fmaf(bf16_lo(w.y), x[2], acc);
-  acc = fmaf(bf16_hi(w.y), x[3], acc);
+  b = fmaf(bf16_hi(w.y), x[3], b);
   acc = fmaf(bf16_lo(w.z), x[4], acc);
-  acc = fmaf(bf16_hi(w.z), x[5], acc);
+  b = fmaf(bf16_hi(w.z), x[5], b);
   acc = fmaf(bf16_lo(w.w), x[6], acc);
-  acc = fmaf(bf16_hi(w.w), x[7], acc);
-  return acc;
+  b = fmaf(bf16_hi(w.w), x[7], b);
+  return acc + b;
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
@@ -298,7 +311,7 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
 }
 
 struct Attn {
-  int b, kvh, c, S, p0, n_cached, nsub, P;
+  int b, kvh, c, hg, S, p0, n_cached, nsub, P;
   bool active, owns_new;
   size_t cache_base;  // element offset of (layer, b, kvh, position p0)
 };
@@ -308,6 +321,7 @@ __device__ __forceinline__ Attn attn_geo(const Params& p, const mk_instr& in, in
   a.b = in.a;
   a.kvh = in.b;
   a.c = in.c;
+  a.hg = in.d;
   a.S = p.seq_lens[a.b];
   a.p0 = a.c * p.chunk;
   const int p1 = min(a.p0 + p.chunk, p.T);
@@ -383,7 +397,8 @@ struct Cursor {
     if (op == OP_ATTN) {
       const int np = min(a.P, a.n_cached - sub * a.P);
       const uint32_t bytes = (uint32_t)np * pp->hd * 2u;
-      f((kv ? pp->vc : pp->kc) + a.cache_base + (size_t)sub * a.P * pp->hd, bytes, 0u);
+      const uint16_t* src = (kv ? pp->vc : pp->kc) + a.cache_base + (size_t)sub * a.P * pp->hd;
+      for (uint32_t o = 0; o < bytes; o += pp->copy_piece) f(src + o / 2, min(pp->copy_piece, bytes - o), o);
       return bytes;
     }
     const int R = g.tile.rows_per_stage;
@@ -395,7 +410,10 @@ struct Cursor {
       const uint16_t* src = (m ? g.wup : g.seg_ptr(sg)) + off;
       const uint32_t base = (uint32_t)m * R * seg;
       if (g.ks == 1) {
-        f(src, bytes, base);
+        // several concurrent bulk copies per stage keep more requests in flight
+        const uint32_t piece = pp->copy_piece;
+        for (uint32_t o = 0; o < bytes; o += piece)
+          f(src + o / 2, min(piece, bytes - o), base + o);
       } else {
         for (int r = 0; r < nr; ++r) f(src + (size_t)r * g.K, seg, base + r * seg);
       }
@@ -438,10 +456,12 @@ struct Producer {
     if (k >= (uint32_t)kStages) {
       const uint32_t parity = ((k / kStages) - 1) & 1;
       if (!mbar_try_wait(&ctl->empty[slot], parity)) {
-        prefetch_ahead();
         const uint64_t t0 = globaltimer();
         uint32_t spins = 0;
         while (!mbar_try_wait(&ctl->empty[slot], parity)) {
+          // only while the consumers wait on another SM: steady streaming is
+          // left alone (prefetches share the copy engine with the ring)
+          if (*(volatile int*)&ctl->waiting) prefetch_ahead();
           if (*(volatile int*)&ctl->dead) return false;
           if ((++spins & 63) == 0) {
             if (ld_relaxed_i32(p.status) != 0) return false;
@@ -559,6 +579,7 @@ struct Consumer {
       const uint32_t target = p.epoch * (uint32_t)count;
       const uint32_t* c = p.counters + idx;
       if ((int32_t)(ld_acquire(c) - target) < 0) {
+        *(volatile int*)&ctl->waiting = 1;
         const uint64_t t0 = globaltimer();
         while (true) {
           if ((int32_t)(ld_acquire(c) - target) >= 0) break;
@@ -573,6 +594,7 @@ struct Consumer {
           }
           __nanosleep(40);
         }
+        *(volatile int*)&ctl->waiting = 0;
       }
     }
     if (t == 0 && *(volatile int*)&ctl->dead) fail = true;
@@ -686,19 +708,25 @@ struct Consumer {
 #pragma unroll
       for (int k = 0; k < RPT; ++k) {
         const int i = rs + k * tl.rpp;
-        float a0 = 0.f, a1 = 0.f;
-        if (i < n) {
+        // one FMA chain per input vector (independent), summed at the end
+        float a0[NVT], a1[NVT];
 #pragma unroll
-          for (int j = 0; j < NVT; ++j) {
-            const int v = ct + j * tl.tpr;
-            if (v < vt) {
-              a0 = dot8(*reinterpret_cast<const uint4*>(w0 + (size_t)i * K + v * 8), xr[j], a0);
-              if (GATED) a1 = dot8(*reinterpret_cast<const uint4*>(w1 + (size_t)i * K + v * 8), xr[j], a1);
-            }
+        for (int j = 0; j < NVT; ++j) {
+          a0[j] = 0.f;
+          a1[j] = 0.f;
+          const int v = ct + j * tl.tpr;
+          if (i < n && v < vt) {
+            a0[j] = dot8(*reinterpret_cast<const uint4*>(w0 + (size_t)i * K + v * 8), xr[j], 0.f);
+            if (GATED) a1[j] = dot8(*reinterpret_cast<const uint4*>(w1 + (size_t)i * K + v * 8), xr[j], 0.f);
           }
         }
-        acc[k] = a0;
-        if (GATED) acc[RPT + k] = a1;
+#pragma unroll
+        for (int j = 1; j < NVT; ++j) {
+          a0[0] += a0[j];
+          if (GATED) a1[0] += a1[j];
+        }
+        acc[k] = a0[0];
+        if (GATED) acc[RPT + k] = a1[0];
       }
       const float sum = warp_reduce_multi<RPT * NM>(acc, lane);
       if (writer) {
@@ -825,6 +853,9 @@ struct Consumer {
     const Attn a = attn_geo(p, in, layer, HD);
     const int qd = p.nq * HD, kvd = p.nkv * HD;
     const float* qkv = p.qkv + (size_t)a.b * (qd + 2 * kvd);
+    // G = query heads of this instruction: head group hg of KV head kvh
+    const int group = p.nq / p.nkv, nhg = group / G;
+    const int q0 = a.kvh * group + a.hg * G;  // first query head
     const float qscale = 1.4426950408889634f * rsqrtf((float)HD);  // log2(e) / sqrt(hd)
     const int pl = lane / LPP, vi = lane % LPP;
     // RoPE table entries do not depend on this step's activations: fetch
@@ -842,8 +873,7 @@ struct Consumer {
       const int tasks = G + (a.owns_new ? 2 : 0);
       for (int task = warp; task < tasks; task += kConsumerWarps) {
         const bool is_v = task == G + 1;
-        const float* src = task < G ? qkv + (a.kvh * G + task) * HD
-                                    : qkv + qd + (is_v ? kvd : 0) + a.kvh * HD;
+        const float* src = task < G ? qkv + (q0 + task) * HD : qkv + qd + (is_v ? kvd : 0) + a.kvh * HD;
         float lo[NP], hi[NP];
         float ss = 0.f;
 #pragma unroll
@@ -878,104 +908,123 @@ struct Consumer {
             ctl->qs[task * HD + lane + 32 * j + HD / 2] = hi[j] * qscale;
           }
         } else {
-          // append the new row (bf16) at index S and keep its rounded value
+          // the new row (bf16): kept for this instruction's own use, and
+          // appended at index S by head group 0 (every group computes the
+          // same bits)
           uint16_t* cache = (is_v ? p.vc : p.kc) + a.cache_base + (size_t)(a.S - a.p0) * HD;
-          float* keep = is_v ? ctl->vnew : ctl->knew;
+          uint16_t* keep = is_v ? ctl->vnew : ctl->knew;
 #pragma unroll
           for (int j = 0; j < NP; ++j) {
             const uint16_t b0 = f32_to_bf16_bits(lo[j]), b1 = f32_to_bf16_bits(hi[j]);
-            cache[lane + 32 * j] = b0;
-            cache[lane + 32 * j + HD / 2] = b1;
-            keep[lane + 32 * j] = bf16_bits_to_f32(b0);
-            keep[lane + 32 * j + HD / 2] = bf16_bits_to_f32(b1);
+            if (a.hg == 0) {
+              cache[lane + 32 * j] = b0;
+              cache[lane + 32 * j + HD / 2] = b1;
+            }
+            keep[lane + 32 * j] = b0;
+            keep[lane + 32 * j + HD / 2] = b1;
           }
         }
       }
       consumer_bar();
       if (tr) tr[4] = globaltimer();
-      // q stays in registers up to 4 heads per KV head; with 8 it is read
-      // from shared memory (a broadcast across position groups) so that the
-      // 8 x 8 running outputs fit the 168-register budget of a 9-warp CTA.
-      constexpr bool kQRegs = G <= 4;
-      float q[kQRegs ? G : 1][8], o[G][8], m[G], l[G];
+      // Each group of LPP lanes owns 8 dimensions per lane and walks blocks
+      // of TB consecutive positions.  One transposed reduction leaves every
+      // (position, head) score of the block on its own lane (R = TB * G
+      // values), so each exponential is computed once; p and the rescale
+      // factors are then broadcast for the P.V update.
+      constexpr int TB = LPP / G < 4 ? LPP / G : 4;
+      constexpr int R = TB * G;
+      constexpr int SH = ilog2c(LPP) - ilog2c(R);  // lane -> value index shift
+      const int gbase = lane & ~(LPP - 1);
+      const int my_t = (vi >> SH) / G;  // this lane's position in a block (its head is (vi >> SH) % G)
+      float q[G][8], o[G][8];
+      float m_l = -1e30f, l_l = 0.f;  // running max / sum of this lane's head
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        m[h] = -1e30f;
-        l[h] = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          if (kQRegs) q[kQRegs ? h : 0][e] = ctl->qs[h * HD + vi * 8 + e];
+          q[h][e] = ctl->qs[h * HD + vi * 8 + e];
           o[h][e] = 0.f;
         }
       }
-      auto qv = [&](int h, int e) -> float { return kQRegs ? q[kQRegs ? h : 0][e] : ctl->qs[h * HD + vi * 8 + e]; };
+      // one block of TB positions starting at row t0 of Kb/Vb (rows >= np are absent)
+      auto block = [&](const uint16_t* Kb, const uint16_t* Vb, int t0, int np) {
+        float acc[R];
+#pragma unroll
+        for (int tt = 0; tt < TB; ++tt) {
+          float kf[8];
+          if (t0 + tt < np) {
+            unpack8(*reinterpret_cast<const uint4*>(Kb + (size_t)(t0 + tt) * HD + vi * 8), kf);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) kf[e] = 0.f;
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) d = fmaf(q[h][e], kf[e], d);
+            acc[tt * G + h] = d;
+          }
+        }
+        // every lane takes part in the reduction (full-mask shuffles), then
+        // lanes whose position is absent drop their score
+        const float red_sc = group_reduce_multi<R, LPP>(acc, lane);
+        const bool valid = t0 + my_t < np;
+        const float sc = valid ? red_sc : -1e30f;
+        float bm = sc;
+#pragma unroll
+        for (int off = G << SH; off < LPP; off <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+        const float mn = fmaxf(m_l, bm);
+        const float corr = exp2f(m_l - mn);
+        const float pv = valid ? exp2f(sc - mn) : 0.f;
+        float ps = pv;
+#pragma unroll
+        for (int off = G << SH; off < LPP; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        l_l = l_l * corr + ps;
+        m_l = mn;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float c = __shfl_sync(0xffffffffu, corr, gbase + ((h) << SH));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[h][e] *= c;
+        }
+#pragma unroll
+        for (int tt = 0; tt < TB; ++tt) {
+          float vf[8];
+          if (t0 + tt < np) {
+            unpack8(*reinterpret_cast<const uint4*>(Vb + (size_t)(t0 + tt) * HD + vi * 8), vf);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) vf[e] = 0.f;
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float pr = __shfl_sync(0xffffffffu, pv, gbase + ((tt * G + h) << SH));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e]);
+          }
+        }
+      };
       // -- cached positions, streamed K stage then V stage
       for (int s = 0; s < a.nsub; ++s) {
         const int np = min(a.P, a.n_cached - s * a.P);
         const uint16_t* Ks = reinterpret_cast<const uint16_t*>(wait_stage(k));
         const uint16_t* Vs = reinterpret_cast<const uint16_t*>(wait_stage(k + 1));
         if (tr && s == 0) tr[5] = globaltimer();
-        for (int tb = warp * PPW; tb < np; tb += kConsumerWarps * PPW) {
-          const int tp = tb + pl;
-          const bool valid = tp < np;
-          float kf[8], vf[8];
-          if (valid) {
-            unpack8(*reinterpret_cast<const uint4*>(Ks + (size_t)tp * HD + vi * 8), kf);
-            unpack8(*reinterpret_cast<const uint4*>(Vs + (size_t)tp * HD + vi * 8), vf);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) kf[e] = vf[e] = 0.f;
-          }
-          float sc[G];
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float d = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) d = fmaf(qv(h, e), kf[e], d);
-#pragma unroll
-            for (int off = LPP / 2; off; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-            sc[h] = d;
-          }
-          if (valid) {
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const float mn = fmaxf(m[h], sc[h]);
-              const float corr = exp2f(m[h] - mn), pr = exp2f(sc[h] - mn);
-              l[h] = l[h] * corr + pr;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) o[h][e] = fmaf(o[h][e], corr, pr * vf[e]);
-              m[h] = mn;
-            }
-          }
-        }
+        for (int tb = warp * PPW * TB; tb < np; tb += kConsumerWarps * PPW * TB) block(Ks, Vs, tb + pl * TB, np);
         release();  // K slot
         release();  // V slot
       }
       if (tr) tr[6] = globaltimer();
       // -- the new token (warp 0, first position group)
-      if (a.owns_new && warp == 0) {
-        float kf[8], vf[8];
+      if (a.owns_new && warp == 0) block(ctl->knew, ctl->vnew, pl * TB, 1);
+      // every lane gets (m, l) of every head of its group
+      float m[G], l[G];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          kf[e] = ctl->knew[vi * 8 + e];
-          vf[e] = ctl->vnew[vi * 8 + e];
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float d = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) d = fmaf(qv(h, e), kf[e], d);
-#pragma unroll
-          for (int off = LPP / 2; off; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-          if (pl == 0) {
-            const float mn = fmaxf(m[h], d);
-            const float corr = exp2f(m[h] - mn), pr = exp2f(d - mn);
-            l[h] = l[h] * corr + pr;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[h][e] = fmaf(o[h][e], corr, pr * vf[e]);
-            m[h] = mn;
-          }
-        }
+      for (int h = 0; h < G; ++h) {
+        m[h] = __shfl_sync(0xffffffffu, m_l, gbase + (h << SH));
+        l[h] = __shfl_sync(0xffffffffu, l_l, gbase + (h << SH));
       }
       // -- merge the position groups of each warp
 #pragma unroll
@@ -995,33 +1044,41 @@ struct Consumer {
           m[h] = mn;
         }
       }
-      // -- merge the warps through shared memory, one head at a time
-      const size_t pbase = ((size_t)a.b * p.nq + (size_t)a.kvh * G) * p.n_chunks + a.c;
+      // -- merge the warps through shared memory, HR heads per round
+      constexpr int HR = kRedFloats / (kConsumerWarps * HD) < G ? kRedFloats / (kConsumerWarps * HD) : G;
+      const size_t pbase = ((size_t)a.b * p.nq + q0) * p.n_chunks + a.c;
+      if (pl == 0 && vi == 0) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < G; ++h) {
+          ctl->aml[(warp * kMaxGroup + h) * 2] = m[h];
+          ctl->aml[(warp * kMaxGroup + h) * 2 + 1] = l[h];
+        }
+      }
+#pragma unroll
+      for (int h0 = 0; h0 < G; h0 += HR) {
         if (pl == 0) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) red[warp * (HD + 2) + vi * 8 + e] = o[h][e];
-          if (vi == 0) {
-            red[warp * (HD + 2) + HD] = m[h];
-            red[warp * (HD + 2) + HD + 1] = l[h];
+          for (int hh = 0; hh < HR; ++hh) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) red[(warp * HR + hh) * HD + vi * 8 + e] = o[h0 + hh][e];
           }
         }
         consumer_bar();
-        if (t < HD) {
+        for (int id = t; id < HR * HD; id += kConsumerThreads) {
+          const int hh = id / HD, d = id % HD, h = h0 + hh;
           float M = -1e30f;
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * (HD + 2) + HD]);
+          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ctl->aml[(w * kMaxGroup + h) * 2]);
           float den = 0.f, num = 0.f;
 #pragma unroll
           for (int w = 0; w < kConsumerWarps; ++w) {
-            const float c = exp2f(red[w * (HD + 2) + HD] - M);
-            den = fmaf(c, red[w * (HD + 2) + HD + 1], den);
-            num = fmaf(c, red[w * (HD + 2) + t], num);
+            const float c = exp2f(ctl->aml[(w * kMaxGroup + h) * 2] - M);
+            den = fmaf(c, ctl->aml[(w * kMaxGroup + h) * 2 + 1], den);
+            num = fmaf(c, red[(w * HR + hh) * HD + d], num);
           }
           const size_t pi = pbase + (size_t)h * p.n_chunks;
-          p.part_o[pi * HD + t] = num;
-          if (t == 0) {
+          p.part_o[pi * HD + d] = num;
+          if (d == 0) {
             p.part_ml[pi * 2] = M;
             p.part_ml[pi * 2 + 1] = den;
           }
@@ -1033,7 +1090,8 @@ struct Consumer {
     consumer_bar();
     if (t == 0) {
       __threadfence();
-      const uint32_t old = atom_acq_rel_add(p.tickets + ((size_t)layer * p.B + a.b) * p.nkv + a.kvh, 1u);
+      const uint32_t old =
+          atom_acq_rel_add(p.tickets + (((size_t)layer * p.B + a.b) * p.nkv + a.kvh) * nhg + a.hg, 1u);
       ctl->last = (old + 1u == p.epoch * (uint32_t)p.n_chunks);
     }
     consumer_bar();
@@ -1041,7 +1099,7 @@ struct Consumer {
       // (m, l) of every (head, chunk) into shared memory with one parallel
       // pass, then each output element reads its chunks' o with independent loads
       const int nvalid = a.S / p.chunk + 1;  // chunks holding a position <= S
-      const size_t pg = ((size_t)a.b * p.nq + (size_t)a.kvh * G) * p.n_chunks;
+      const size_t pg = ((size_t)a.b * p.nq + q0) * p.n_chunks;
       for (int idx = t; idx < G * nvalid; idx += kConsumerThreads) {
         const int h = idx / nvalid, c = idx % nvalid;
         const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml) + pg + (size_t)h * p.n_chunks + c);
@@ -1062,7 +1120,7 @@ struct Consumer {
           den = fmaf(w, ml[2 * c + 1], den);
           num = fmaf(w, __ldcg(po + (size_t)c * HD), num);
         }
-        p.attn[(size_t)a.b * qd + (size_t)(a.kvh * G + h) * HD + d] = num / den;
+        p.attn[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = num / den;
       }
       signal(sig_idx);
     }
@@ -1070,21 +1128,18 @@ struct Consumer {
   }
 
   __device__ __forceinline__ bool attn(const mk_instr& in, int layer, int sig_idx) {
-    const int G = p.nq / p.nkv;
+    const int G = attn_heads_per_instr(p.nq / p.nkv);
     if (p.hd == 128) {
       switch (G) {
         case 1: return attn_run<128, 1>(in, layer, sig_idx);
         case 2: return attn_run<128, 2>(in, layer, sig_idx);
-        case 4: return attn_run<128, 4>(in, layer, sig_idx);
-        default: return attn_run<128, 8>(in, layer, sig_idx);
+        default: return attn_run<128, 4>(in, layer, sig_idx);
       }
-    } else {
-      switch (G) {
-        case 1: return attn_run<64, 1>(in, layer, sig_idx);
-        case 2: return attn_run<64, 2>(in, layer, sig_idx);
-        case 4: return attn_run<64, 4>(in, layer, sig_idx);
-        default: return attn_run<64, 8>(in, layer, sig_idx);
-      }
+    }
+    switch (G) {
+      case 1: return attn_run<64, 1>(in, layer, sig_idx);
+      case 2: return attn_run<64, 2>(in, layer, sig_idx);
+      default: return attn_run<64, 4>(in, layer, sig_idx);
     }
   }
 };
@@ -1147,6 +1202,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
     }
     ctl->dead = 0;
     ctl->last = 0;
+    ctl->waiting = 0;
     // a sticky error from an earlier step, or out-of-range inputs: do nothing
     int bad = ld_relaxed_i32(p.status) != 0;
     for (int b = 0; b < p.B && !bad; ++b) {

@@ -125,7 +125,8 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
     return o;
   };
   const size_t o_cnt = take(sizeof(uint32_t) * (size_t)n_cnt);
-  const size_t o_tk = take(sizeof(uint32_t) * (size_t)L * B * nkv);
+  const int group = nq / nkv;
+  const size_t o_tk = take(sizeof(uint32_t) * (size_t)L * B * nkv * (group / mk::attn_heads_per_instr(group)));
   const size_t o_st = take(sizeof(int) * 4);
   const size_t zero_bytes = off;
   const size_t o_xres = take(sizeof(float) * (size_t)(2 * L + 1) * B * H);
@@ -208,6 +209,7 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   p.logits = out_logits;
   p.epoch = 1;  // counters were just cleared
   p.l2_ahead = mk::kDefaultL2AheadBytes;
+  p.copy_piece = mk::kDefaultCopyPiece;
   if (mk::launch_step(p, n_sm, s) != cudaSuccess) {
     cudaGetLastError();
     return MK_ERR_CUDA;

@@ -122,7 +122,7 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
   p->n_chunks = (d->max_ctx + p->chunk - 1) / p->chunk;
   // the merging CTA stages (m, l) of every (query head of the group, chunk) in
   // its kRedFloats-float reduction buffer
-  if (2 * (d->n_q_heads / d->n_kv_heads) * p->n_chunks > kRedFloats) return MK_ERR_UNSUPPORTED;
+  if (2 * attn_heads_per_instr(d->n_q_heads / d->n_kv_heads) * p->n_chunks > kRedFloats) return MK_ERR_UNSUPPORTED;
   Builder b{p};
 
   // x0 = embedding rows, hidden dimension split over the SMs
@@ -142,13 +142,15 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
     // rows of wq | wk | wv concatenated; an instruction may span matrices
     int n_qkv = b.rows_op(OP_QKV, l, qd + 2 * kvd, {}, prev_idx, prev_count, cq);
     p->targets[cq] = n_qkv;
+    const int group = d->n_q_heads / d->n_kv_heads, nhg = group / attn_heads_per_instr(group);
     for (int s = 0; s < d->batch; ++s)
       for (int h = 0; h < d->n_kv_heads; ++h)
-        for (int c = 0; c < p->n_chunks; ++c) {
-          b.emit((int)(attn_rr % n_sm), OP_ATTN, l, cq, n_qkv, ca, s, h, c);
-          ++attn_rr;
-        }
-    p->targets[ca] = d->batch * d->n_kv_heads;  // one bump per merged (sequence, KV head)
+        for (int hg = 0; hg < nhg; ++hg)
+          for (int c = 0; c < p->n_chunks; ++c) {
+            b.emit((int)(attn_rr % n_sm), OP_ATTN, l, cq, n_qkv, ca, s, h, c, hg);
+            ++attn_rr;
+          }
+    p->targets[ca] = d->batch * d->n_kv_heads * nhg;  // one bump per merged (sequence, KV head, head group)
     int n_o = b.rows_op(OP_OPROJ, l, H, {}, ca, p->targets[ca], co);
     p->targets[co] = n_o;
     int n_gu = b.rows_op(OP_GATEUP, l, d->ffn_dim, {}, co, n_o, cg);
