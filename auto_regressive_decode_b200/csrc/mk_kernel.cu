@@ -224,6 +224,35 @@ __device__ __forceinline__ float dot8(const uint4 w, const float x[8], float acc
   return acc + b;
 }
 
+// Packed fp32 pairs (sm_100 fma.rn.f32x2: two IEEE fp32 FMAs per instruction).
+__device__ __forceinline__ unsigned long long pack2(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ float sum2(unsigned long long a) {
+  float x, y;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(a));
+  return x + y;
+}
+
+// 8 bf16 weights times 8 packed fp32 inputs, accumulated as fp32 pairs.
+__device__ __forceinline__ unsigned long long dot8x2(const uint4 w, const unsigned long long xp[4],
+                                                     unsigned long long acc) {
+  acc = ffma2(pack2(bf16_lo(w.x), bf16_hi(w.x)), xp[0], acc);
+  acc = ffma2(pack2(bf16_lo(w.y), bf16_hi(w.y)), xp[1], acc);
+  acc = ffma2(pack2(bf16_lo(w.z), bf16_hi(w.z)), xp[2], acc);
+  acc = ffma2(pack2(bf16_lo(w.w), bf16_hi(w.w)), xp[3], acc);
+  return acc;
+}
+
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
   __nv_bfloat16 b = __float2bfloat16_rn(f);
   return *reinterpret_cast<uint16_t*>(&b);
@@ -592,7 +621,6 @@ struct Consumer {
             fail = true;
             break;
           }
-          __nanosleep(40);
         }
         *(volatile int*)&ctl->waiting = 0;
       }
@@ -601,12 +629,13 @@ struct Consumer {
     return !consumer_bar_or(fail);
   }
 
+  // The named barrier orders every consumer thread's stores of this
+  // instruction before thread 0's release reduction; a gpu-scope release is
+  // cumulative over what is ordered before it, so an SM that acquires the
+  // counter sees all of them.
   __device__ __forceinline__ void signal(int idx) {
     consumer_bar();
-    if (t == 0 && idx >= 0) {
-      __threadfence();
-      red_release_add(p.counters + idx, 1u);
-    }
+    if (t == 0 && idx >= 0) red_release_add(p.counters + idx, 1u);
   }
 
   // Block-wide sum over the 256 consumer threads (result in every thread).
@@ -694,6 +723,11 @@ struct Consumer {
     const int rs = t / tl.tpr, ct = t % tl.tpr, wpr = tl.tpr / 32, wir = ct / 32;
     const int q = row_of_lane<RPT * NM>(lane);
     const bool writer = (lane & (32 / (RPT * NM) - 1)) == 0;
+    unsigned long long xp[NVT][4];  // the input slice as fp32 pairs
+#pragma unroll
+    for (int j = 0; j < NVT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) xp[j][e] = pack2(xr[j][2 * e], xr[j][2 * e + 1]);
     int rl = 0;  // first row of the segment within the instruction
 #pragma unroll 1
     for (int sg = 0; sg < g.nseg; ++sg) {
@@ -708,25 +742,17 @@ struct Consumer {
 #pragma unroll
       for (int k = 0; k < RPT; ++k) {
         const int i = rs + k * tl.rpp;
-        // one FMA chain per input vector (independent), summed at the end
-        float a0[NVT], a1[NVT];
+        unsigned long long a0 = 0ull, a1 = 0ull;  // (+0.0f, +0.0f) pairs
 #pragma unroll
         for (int j = 0; j < NVT; ++j) {
-          a0[j] = 0.f;
-          a1[j] = 0.f;
           const int v = ct + j * tl.tpr;
           if (i < n && v < vt) {
-            a0[j] = dot8(*reinterpret_cast<const uint4*>(w0 + (size_t)i * K + v * 8), xr[j], 0.f);
-            if (GATED) a1[j] = dot8(*reinterpret_cast<const uint4*>(w1 + (size_t)i * K + v * 8), xr[j], 0.f);
+            a0 = dot8x2(*reinterpret_cast<const uint4*>(w0 + (size_t)i * K + v * 8), xp[j], a0);
+            if (GATED) a1 = dot8x2(*reinterpret_cast<const uint4*>(w1 + (size_t)i * K + v * 8), xp[j], a1);
           }
         }
-#pragma unroll
-        for (int j = 1; j < NVT; ++j) {
-          a0[0] += a0[j];
-          if (GATED) a1[0] += a1[j];
-        }
-        acc[k] = a0[0];
-        if (GATED) acc[RPT + k] = a1[0];
+        acc[k] = sum2(a0);
+        if (GATED) acc[RPT + k] = sum2(a1);
       }
       const float sum = warp_reduce_multi<RPT * NM>(acc, lane);
       if (writer) {
