@@ -162,6 +162,14 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
   }
   const int c_lm = counter_lmhead(L);
   p->targets[c_lm] = b.rows_op(OP_LMHEAD, L, d->vocab, {}, prev_idx, prev_count, c_lm);
+  // Host-made fault for tests of the failure path (never set in normal use):
+  // MK_FAULT_INJECT=wait makes SM 0's first instruction wait on a counter no
+  // instruction ever raises far enough, so every bounded wait must run out.
+  const char* fault = getenv("MK_FAULT_INJECT");
+  if (fault && strcmp(fault, "wait") == 0 && !p->lists[0].empty()) {
+    p->lists[0][0].wait_idx = c_lm;
+    p->lists[0][0].wait_count = p->targets[c_lm] + 1;
+  }
   return MK_OK;
 }
 

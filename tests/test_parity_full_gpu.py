@@ -1,0 +1,58 @@
+"""Parity at the full dense 8B shape (batch 1, context 4096), in the configuration bench.py times.
+
+The whole step runs on the GPU; the oracle then recomputes sampled layers one by
+one from the GPU's own input to each layer (its dumped residual), and the LM
+head from the GPU's final residual, so each check is independent of the
+others.  Tolerances as in tests/gpu_harness.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fixtures as fx
+import oracle as ora
+from fixtures.device import device_caches, device_model
+from tests.gpu_harness import TOL_HIDDEN, TOL_KV, TOL_LOGITS_ABS, bits
+from tests.helpers import bf16_f64, host_model, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+SAMPLED_LAYERS = (0, 13, 31)
+
+
+def test_dense_8b_sampled_layers_and_logits():
+    import auto_regressive_decode_b200.mk as mk
+    cfg = fx.CONFIGS["dense-8b"]
+    S0 = fx.context_lengths(cfg)
+    tok = fx.tokens(cfg)[0]
+    w = device_model(cfg)
+    kc, vc = device_caches(cfg, S0)
+    dec = mk.Decoder(cfg, w, kc, vc)
+    logits = torch.empty((1, cfg.vocab), dtype=torch.float32, device="cuda")
+    d_tok = torch.from_numpy(tok.copy()).cuda()
+    d_len = torch.from_numpy(S0.copy()).cuda()
+    dec.step(d_tok, d_len, d_len, logits)
+    assert dec.status() == mk.MK_OK
+    hid = dec.hidden_states().cpu().numpy().astype(np.float64)
+    lg = logits.cpu().numpy().astype(np.float64)[0]
+    S = int(S0[0])
+    k_new = {l: bf16_f64(bits(kc[l, 0, :, S].contiguous())) for l in SAMPLED_LAYERS}
+    v_new = {l: bf16_f64(bits(vc[l, 0, :, S].contiguous())) for l in SAMPLED_LAYERS}
+    dec.close()
+    del w, kc, vc
+    torch.cuda.empty_cache()
+
+    g, ls = host_model(cfg, layers=SAMPLED_LAYERS)
+    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls)
+    assert np.array_equal(hid[0, 0], bf16_f64(g["embed"][tok[0]]))
+    for l in SAMPLED_LAYERS:
+        okc = fx.kv_prefill(cfg, l, 0, S0)
+        ovc = fx.kv_prefill(cfg, l, 1, S0)
+        out = model.layer_forward(l, hid[2 * l].copy(), okc, ovc, S0, S0)
+        assert rel_l2(hid[2 * l + 1], out["h_attn"]) <= TOL_HIDDEN, l
+        assert rel_l2(hid[2 * l + 2], out["h_mlp"]) <= TOL_HIDDEN, l
+        assert rel_l2(k_new[l], bf16_f64(okc[0, :, S])) <= TOL_KV, l
+        assert rel_l2(v_new[l], bf16_f64(ovc[0, :, S])) <= TOL_KV, l
+    ref = model.lm_head(hid[2 * cfg.n_layers, 0])
+    assert float(np.max(np.abs(lg - ref))) <= TOL_LOGITS_ABS
+    assert int(np.argmax(lg)) == int(np.argmax(ref))

@@ -1,0 +1,155 @@
+"""Contract tests of the host scheduler (per-SM instruction lists and dependency counters), no GPU.
+
+The lists must cover every output row / attention chunk exactly once, every
+counter's per-step target must equal the number of its producers, waits may
+only point at earlier ops, and a simulation of the counter protocol (each SM
+executes its list in order, an instruction runs once its counter reached its
+target) must run every instruction to completion: no cyclic wait.
+"""
+import collections
+
+import numpy as np
+import pytest
+
+import fixtures as fx
+
+mk = pytest.importorskip("auto_regressive_decode_b200.mk")
+
+OP_EMBED, OP_QKV, OP_ATTN, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LMHEAD = 1, 2, 3, 4, 5, 6, 7
+ORDER = {OP_EMBED: 0, OP_QKV: 1, OP_ATTN: 2, OP_OPROJ: 3, OP_GATEUP: 4, OP_DOWN: 5, OP_LMHEAD: 6}
+
+CASES = [("tiny", 148), ("tiny", 7), ("tiny", 1), ("dense-0.6b", 148), ("dense-8b", 148), ("dense-8b", 132)]
+
+
+def plan_of(name, n_sm, **kw):
+    cfg = fx.CONFIGS[name].replace(**kw)
+    return cfg, mk.Plan(mk.model_desc(cfg), n_sm)
+
+
+def rows_of(cfg, op):
+    return {OP_QKV: cfg.q_dim + 2 * cfg.kv_dim, OP_OPROJ: cfg.hidden, OP_GATEUP: cfg.ffn_dim, OP_DOWN: cfg.hidden,
+            OP_LMHEAD: cfg.vocab, OP_EMBED: cfg.hidden}[op]
+
+
+@pytest.mark.parametrize("name,n_sm", CASES)
+def test_rows_and_chunks_covered_once(name, n_sm):
+    cfg, p = plan_of(name, n_sm)
+    cover = collections.defaultdict(list)
+    attn = collections.Counter()
+    for row in p.instrs:
+        op, layer = p.op(row), p.layer(row)
+        if op == OP_ATTN:
+            attn[(layer, int(row[4]), int(row[5]), int(row[6]), int(row[7]))] += 1
+        else:
+            cover[(layer, op)].append((int(row[4]), int(row[5])))
+            assert 0 < row[5] - row[4] <= 256
+    for (layer, op), segs in cover.items():
+        segs.sort()
+        assert segs[0][0] == 0 and segs[-1][1] == rows_of(cfg, op)
+        assert all(a[1] == b[0] for a, b in zip(segs, segs[1:])), (layer, op)
+    group = cfg.n_q_heads // cfg.n_kv_heads
+    nhg = group // min(group, 4)
+    assert len(attn) == cfg.n_layers * cfg.batch * cfg.n_kv_heads * nhg * p.n_chunks
+    assert set(attn.values()) == {1}
+    assert p.chunk * p.n_chunks >= cfg.max_ctx > p.chunk * (p.n_chunks - 1)
+
+
+@pytest.mark.parametrize("name,n_sm", CASES)
+def test_counter_targets_and_wait_order(name, n_sm):
+    cfg, p = plan_of(name, n_sm)
+    producers = collections.Counter(int(r[3]) for r in p.instrs if int(r[3]) >= 0 and p.op(r) != OP_ATTN)
+    merges = collections.Counter()
+    op_of_counter = {}
+    for r in p.instrs:
+        if int(r[3]) >= 0:
+            op_of_counter[int(r[3])] = (p.layer(r) if p.op(r) != OP_EMBED else -1, ORDER[p.op(r)])
+        if p.op(r) == OP_ATTN:
+            merges[int(r[3])] = 0
+    group = cfg.n_q_heads // cfg.n_kv_heads
+    nhg = group // min(group, 4)
+    for c, t in enumerate(p.targets):
+        if c in merges:
+            assert t == cfg.batch * cfg.n_kv_heads * nhg
+        elif c in producers:
+            assert t == producers[c], c
+    for r in p.instrs:
+        w = int(r[1])
+        if w < 0:
+            assert p.op(r) == OP_EMBED
+            continue
+        assert int(r[2]) == p.targets[w]
+        me = (p.layer(r) if p.op(r) != OP_EMBED else -1, ORDER[p.op(r)])
+        assert op_of_counter[w] < me, "waits only on an earlier op"
+    # each SM's list is ordered by (layer, op): waits never point forward in a list
+    for s in range(n_sm):
+        keys = [(p.layer(r) if p.op(r) != OP_EMBED else -1, ORDER[p.op(r)]) for r in p.sm_list(s)]
+        assert keys == sorted(keys)
+
+
+def simulate(p, cfg, order_seed=0):
+    """Counter protocol on the host: SMs progress in a random order; returns instructions executed."""
+    rng = np.random.default_rng(order_seed)
+    counters = np.zeros(len(p.targets), dtype=np.int64)
+    tickets = collections.Counter()
+    pos = [0] * p.n_sm
+    done = 0
+    total = len(p.instrs)
+    while done < total:
+        progressed = False
+        for s in rng.permutation(p.n_sm):
+            lst = p.sm_list(s)
+            while pos[s] < len(lst):
+                r = lst[pos[s]]
+                w = int(r[1])
+                if w >= 0 and counters[w] < int(r[2]):
+                    break
+                if p.op(r) == OP_ATTN:
+                    key = (p.layer(r), int(r[4]), int(r[5]), int(r[7]))
+                    tickets[key] += 1
+                    if tickets[key] == p.n_chunks:
+                        counters[int(r[3])] += 1
+                elif int(r[3]) >= 0:
+                    counters[int(r[3])] += 1
+                pos[s] += 1
+                done += 1
+                progressed = True
+        if not progressed:
+            return done
+    assert (counters == np.asarray(p.targets)).all()
+    return done
+
+
+@pytest.mark.parametrize("name,n_sm", [("tiny", 148), ("tiny", 3), ("dense-0.6b", 148), ("dense-8b", 148)])
+def test_counter_protocol_completes(name, n_sm):
+    cfg, p = plan_of(name, n_sm)
+    for seed in range(2):
+        assert simulate(p, cfg, seed) == len(p.instrs)
+
+
+def test_weight_bytes_balanced_over_sms():
+    cfg, p = plan_of("dense-8b", 148)
+    per_sm = np.zeros(148)
+    K = {OP_QKV: cfg.hidden, OP_OPROJ: cfg.q_dim, OP_GATEUP: 2 * cfg.hidden, OP_DOWN: cfg.ffn_dim, OP_LMHEAD: cfg.hidden}
+    for s in range(148):
+        for r in p.sm_list(s):
+            if p.op(r) in K:
+                per_sm[s] += (int(r[5]) - int(r[4])) * K[p.op(r)] * 2
+    assert per_sm.max() / per_sm.mean() < 1.02
+
+
+def test_fault_injection_hook_makes_an_unsatisfiable_wait(monkeypatch):
+    monkeypatch.setenv("MK_FAULT_INJECT", "wait")
+    cfg, p = plan_of("tiny", 148)
+    first = p.sm_list(0)[0]
+    assert int(first[2]) > p.targets[int(first[1])]
+    assert simulate(p, cfg) < len(p.instrs)
+
+
+def test_invalid_and_unsupported_shapes():
+    base = fx.CONFIGS["tiny"]
+    bad = [base.replace(n_q_heads=3), base.replace(head_dim=96), base.replace(hidden=252)]
+    for cfg in bad:
+        with pytest.raises(mk.MkError):
+            mk.Plan(mk.model_desc(cfg), 148)
+    with pytest.raises(mk.MkError):
+        mk.Plan(mk.model_desc(base), 0)
