@@ -95,10 +95,10 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) return MK_ERR_CUDA;
   if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return MK_ERR_CUDA;
-  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes()) return MK_ERR_UNSUPPORTED;
+  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes(d.batch > 1)) return MK_ERR_UNSUPPORTED;
   if (mk::kernel_prepare() != cudaSuccess) return MK_ERR_CUDA;
   int per_sm = 0;
-  if (mk::kernel_occupancy(&per_sm) != cudaSuccess) return MK_ERR_CUDA;
+  if (mk::kernel_occupancy(&per_sm, d.batch > 1) != cudaSuccess) return MK_ERR_CUDA;
   if (per_sm < 1) return MK_ERR_UNSUPPORTED;
 
   mk_plan* plan = nullptr;

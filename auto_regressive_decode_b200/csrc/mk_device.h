@@ -51,9 +51,9 @@ struct Params {
 };
 
 // Dynamic shared memory of one CTA.
-size_t kernel_smem_bytes();
-cudaError_t kernel_prepare();  // set the function's shared-memory limit
-cudaError_t kernel_occupancy(int* blocks_per_sm);
+size_t kernel_smem_bytes(bool batched);
+cudaError_t kernel_prepare();  // set both kernels' shared-memory limits
+cudaError_t kernel_occupancy(int* blocks_per_sm, bool batched);
 cudaError_t launch_step(const Params& p, int n_blocks, cudaStream_t stream);
 
 }  // namespace mk

@@ -37,7 +37,9 @@ constexpr int kConsumerWarps = 8;                      // compute warps
 constexpr int kConsumerThreads = kConsumerWarps * 32;  // 256
 constexpr int kThreads = kConsumerThreads + 32;        // + one producer warp
 constexpr int kStageBytes = 32 * 1024;                 // one ring slot
-constexpr int kStages = 6;                             // ring depth (192 KB)
+constexpr int kStages = 6;                             // ring depth (192 KB), batch-1 kernel
+constexpr int kStagesBatched = 4;                      // ring depth of the batch > 1 kernel (128 KB)
+constexpr int kXsPitchBytes = 4096 * 2 + 16;           // batch > 1: one sequence's bf16 input slice (padded)
 constexpr int kMaxRows = 256;                          // rows per GEMV instruction
 constexpr int kRedFloats = 4096;                       // cross-warp reduction buffer
 constexpr int kMaxBatch = 8;
@@ -105,6 +107,20 @@ MK_HD int gemv_ksplit(int K, int n_mats) {
     const GemvTile t = gemv_tile(K / ks, n_mats);
     if (t.nv <= 8 && t.rows_per_stage >= 1) return ks;
   }
+  return 0;
+}
+
+// ---- batch > 1 GEMV (tensor cores) -------------------------------------------------
+// Stages hold up to 8 weight rows (16 for the gate/up pair) of one column
+// chunk, each row at a pitch of chunk*2 + 16 bytes (conflict-free fragment
+// loads); the bf16 inputs of all sequences hold one column slice of at most
+// kBatchedSlice columns at a time.
+constexpr int kBatchedMaxRows = 64;   // rows per batched GEMV instruction (8 tiles of 8)
+constexpr int kBatchedSlice = 4096;   // input columns per slice
+MK_HD int bgemv_chunk(int n_mats) { return n_mats == 2 ? 960 : 1984; }
+MK_HD int bgemv_slices(int K) {
+  for (int ks = 1; ks <= 16; ++ks)
+    if (K % ks == 0 && (K / ks) % 16 == 0 && K / ks <= kBatchedSlice) return ks;
   return 0;
 }
 

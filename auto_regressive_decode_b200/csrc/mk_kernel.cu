@@ -50,9 +50,16 @@ struct Ctl {
   alignas(16) uint16_t vnew[kMaxHeadDim];
 };
 
-constexpr size_t kRingBytes = (size_t)kStages * kStageBytes;
-constexpr size_t kRedBytes = (size_t)kRedFloats * sizeof(float);
-constexpr size_t kSmemBytes = kRingBytes + kRedBytes + sizeof(Ctl);
+// Shared memory: the ring, then (batched kernel only) the bf16 input-vector
+// slice for the tensor-core GEMV, then the reduction buffer and Ctl.
+template <bool BATCHED>
+struct Smem {
+  static constexpr int kNst = BATCHED ? kStagesBatched : kStages;
+  static constexpr size_t kRing = (size_t)kNst * kStageBytes;
+  static constexpr size_t kXs = BATCHED ? (size_t)kMaxBatch * kXsPitchBytes : 0;
+  static constexpr size_t kRed = (size_t)kRedFloats * sizeof(float);
+  static constexpr size_t kTotal = kRing + kXs + kRed + sizeof(Ctl);
+};
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -210,6 +217,11 @@ __device__ __forceinline__ void unpack8(const uint4 w, float f[8]) {
   f[6] = bf16_lo(w.w); f[7] = bf16_hi(w.w);
 }
 
+__device__ __forceinline__ uint16_t f32_to_bf16_bits_fwd(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+
 // 8-term dot product in two interleaved FMA chains (shorter dependency chain).
 __device__ __forceinline__ float dot8(const uint4 w, const float x[8], float acc) {
   float b = 0.f;
@@ -253,6 +265,20 @@ __device__ __forceinline__ unsigned long long dot8x2(const uint4 w, const unsign
   return acc;
 }
 
+// D += A(16x16, row) * B(16x8, col), bf16 in, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return (uint32_t)f32_to_bf16_bits_fwd(lo) | ((uint32_t)f32_to_bf16_bits_fwd(hi) << 16);
+}
+
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
   __nv_bfloat16 b = __float2bfloat16_rn(f);
   return *reinterpret_cast<uint16_t*>(&b);
@@ -279,7 +305,17 @@ struct Gemv {
   int K, r0, r1;
   int ks, Kc;                       // column slices per row, slice width (K = ks * Kc)
   GemvTile tile;                    // tiling of one slice
+  // batch > 1 (tensor cores): bks slices of bKs columns, chunks of bKc
+  // columns per stage (bnchunk per slice), 8-row tiles (bntiles)
+  int bks, bKs, bKc, bnchunk, bntiles;
   __device__ __forceinline__ const uint16_t* seg_ptr(int s) const { return s == 0 ? sw0 : (s == 1 ? sw1 : sw2); }
+  // first element of row r0 + rel (rel < r1 - r0), whichever matrix holds it
+  __device__ __forceinline__ const uint16_t* row_ptr(int rel) const {
+    if (rel < sn0) return sw0 + (size_t)rel * K;
+    rel -= sn0;
+    if (rel < sn1) return sw1 + (size_t)rel * K;
+    return sw2 + (size_t)(rel - sn1) * K;
+  }
   __device__ __forceinline__ int seg_rows(int s) const { return s == 0 ? sn0 : (s == 1 ? sn1 : sn2); }
 };
 
@@ -336,6 +372,13 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
   g.ks = gemv_ksplit(g.K, g.wup ? 2 : 1);
   g.Kc = g.K / g.ks;
   g.tile = gemv_tile(g.Kc, g.wup ? 2 : 1);
+  if (p.B > 1) {
+    g.bks = bgemv_slices(g.K);
+    g.bKs = g.K / g.bks;
+    g.bKc = bgemv_chunk(g.wup ? 2 : 1);
+    g.bnchunk = (g.bKs + g.bKc - 1) / g.bKc;
+    g.bntiles = (g.r1 - g.r0 + 7) / 8;
+  }
   return g;
 }
 
@@ -410,6 +453,16 @@ struct Cursor {
       if (!kv && ++sub >= a.nsub) seek(i + 1);
       return;
     }
+    if (pp->B > 1) {  // batched GEMV: (slice kc, tile sg, chunk rr)
+      if (++rr >= g.bnchunk) {
+        rr = 0;
+        if (++sg >= g.bntiles) {
+          sg = 0;
+          if (++kc >= g.bks) seek(i + 1);
+        }
+      }
+      return;
+    }
     rr += g.tile.rows_per_stage;
     if (rr >= g.seg_rows(sg)) {
       rr = 0;
@@ -429,6 +482,18 @@ struct Cursor {
       const uint16_t* src = (kv ? pp->vc : pp->kc) + a.cache_base + (size_t)sub * a.P * pp->hd;
       for (uint32_t o = 0; o < bytes; o += pp->copy_piece) f(src + o / 2, min(pp->copy_piece, bytes - o), o);
       return bytes;
+    }
+    if (pp->B > 1) {
+      // up to 8 rows (tile sg) of column chunk rr of slice kc, one copy per row
+      const int nr = min(8, g.r1 - g.r0 - sg * 8);
+      const int width = min(g.bKc, g.bKs - rr * g.bKc);
+      const uint32_t pitch = (uint32_t)width * 2u + 16u, bytes = (uint32_t)width * 2u;
+      const size_t col = (size_t)kc * g.bKs + (size_t)rr * g.bKc;
+      for (int r = 0; r < nr; ++r) {
+        f(g.row_ptr(sg * 8 + r) + col, bytes, (uint32_t)r * pitch);
+        if (g.wup) f(g.wup + (size_t)(sg * 8 + r) * g.K + col, bytes, (uint32_t)(8 + r) * pitch);
+      }
+      return (uint32_t)nr * bytes * (g.wup ? 2u : 1u);
     }
     const int R = g.tile.rows_per_stage;
     const int nr = min(R, g.seg_rows(sg) - rr);
@@ -452,12 +517,17 @@ struct Cursor {
 
   __device__ __forceinline__ uint32_t stage_bytes() const {
     if (op == OP_ATTN) return (uint32_t)min(a.P, a.n_cached - sub * a.P) * pp->hd * 2u;
+    if (pp->B > 1)
+      return (uint32_t)min(8, g.r1 - g.r0 - sg * 8) * (uint32_t)min(g.bKc, g.bKs - rr * g.bKc) * 2u *
+             (g.wup ? 2u : 1u);
     const uint32_t b = (uint32_t)min(g.tile.rows_per_stage, g.seg_rows(sg) - rr) * (uint32_t)g.Kc * 2u;
     return g.wup ? 2 * b : b;
   }
 };
 
+template <bool BATCHED>
 struct Producer {
+  static constexpr int NST = Smem<BATCHED>::kNst;
   const Params& p;
   Ctl* ctl;
   uint8_t* ring;
@@ -481,9 +551,9 @@ struct Producer {
 
   // Claim the next slot (waiting until the consumers released it).
   __device__ __forceinline__ bool claim(uint8_t** dst, unsigned long long** bar) {
-    const int slot = k % kStages;
-    if (k >= (uint32_t)kStages) {
-      const uint32_t parity = ((k / kStages) - 1) & 1;
+    const int slot = k % NST;
+    if (k >= (uint32_t)NST) {
+      const uint32_t parity = ((k / NST) - 1) & 1;
       if (!mbar_try_wait(&ctl->empty[slot], parity)) {
         const uint64_t t0 = globaltimer();
         uint32_t spins = 0;
@@ -509,18 +579,19 @@ struct Producer {
 
   // After giving up: wait (bounded) for the copies still in flight.
   __device__ __forceinline__ void drain() {
-    const uint32_t first = k > (uint32_t)kStages ? k - kStages : 0;
+    const uint32_t first = k > (uint32_t)NST ? k - NST : 0;
     for (uint32_t j = first; j < k; ++j) {
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&ctl->full[j % kStages], (j / kStages) & 1)) {
+      while (!mbar_try_wait(&ctl->full[j % NST], (j / NST) & 1)) {
         if (globaltimer() - t0 > p.timeout_ns) break;
       }
     }
   }
 };
 
+template <bool BATCHED>
 __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
-  Producer pr(p, ctl, ring, list, n);
+  Producer<BATCHED> pr(p, ctl, ring, list, n);
   uint64_t* trace = p.trace ? p.trace + (size_t)p.offsets[blockIdx.x] * kTraceStamps : nullptr;
   Cursor cur(p, list, n);
   cur.seek(0);
@@ -559,7 +630,9 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
 // ---------------------------------------------------------------------------
 // Consumer warps
 // ---------------------------------------------------------------------------
+template <bool BATCHED>
 struct Consumer {
+  static constexpr int NST = Smem<BATCHED>::kNst;
   const Params& p;
   Ctl* ctl;
   uint8_t* ring;
@@ -578,8 +651,8 @@ struct Consumer {
   __device__ __forceinline__ const uint8_t* wait_full() { return wait_stage(k); }
 
   __device__ __forceinline__ const uint8_t* wait_stage(uint32_t kk) {
-    const int slot = kk % kStages;
-    const uint32_t parity = (kk / kStages) & 1;
+    const int slot = kk % NST;
+    const uint32_t parity = (kk / NST) & 1;
     if (!mbar_try_wait(&ctl->full[slot], parity)) {
       const uint64_t t0 = globaltimer();
       uint32_t spins = 0;
@@ -597,7 +670,7 @@ struct Consumer {
 
   __device__ __forceinline__ void release() {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->empty[k % kStages]);
+    if (lane == 0) mbar_arrive(&ctl->empty[k % NST]);
     ++k;
   }
 
@@ -854,7 +927,162 @@ struct Consumer {
 
   // Ops with an RMSNorm prologue read the hidden vector (K = hidden, at most
   // 4 vectors per thread, checked at creation); o_proj and down read attn / act.
+  // ---- GEMV, batch > 1: tensor cores ---------------------------------------
+  // mma.m16n8k16: A = the bf16 inputs of the batch (rows b < B of 16), B = 8
+  // weight rows of the stage, D[b][row] accumulated in fp32.  Warps share a
+  // stage's k-steps; per 8-row tile the partials are summed across warps in a
+  // fixed order, per column slice into oacc (shared memory).
+  template <bool NORM, bool GATED>
+  __device__ __forceinline__ bool gemv_mma(const mk_instr& in, int op, int layer) {
+    constexpr int NM = GATED ? 2 : 1;
+    const Gemv g = gemv_geo(p, in, op, layer);
+    const int B = p.B, BH = B * p.H, nrows = g.r1 - g.r0;
+    const float* src;
+    const uint16_t* gain = nullptr;
+    int ld;  // elements per sequence in src
+    if (op == OP_QKV) {
+      src = p.xres + (size_t)(2 * layer) * BH, gain = p.layers[layer].attn_norm, ld = p.H;
+    } else if (op == OP_OPROJ) {
+      src = p.attn, ld = p.nq * p.hd;
+    } else if (op == OP_GATEUP) {
+      src = p.xres + (size_t)(2 * layer + 1) * BH, gain = p.layers[layer].mlp_norm, ld = p.H;
+    } else if (op == OP_DOWN) {
+      src = p.act, ld = p.I;
+    } else {
+      src = p.xres + (size_t)(2 * p.L) * BH, gain = p.final_norm, ld = p.H;
+    }
+    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
+    if (tr) tr[1] = globaltimer();
+    float* red2 = red;               // [2][8 warps][NM*64] tile partials
+    float* oacc = red + 2 * 8 * 128;  // [64 rows][16] (gate: b, up: 8 + b)
+    float* scale = ctl->sred;         // [8] RMS scale per sequence
+    if (NORM) {
+      // per-sequence RMS over the whole vector (K = hidden): one block pass
+      float ss[kMaxBatch];
+#pragma unroll
+      for (int b = 0; b < kMaxBatch; ++b) {
+        ss[b] = 0.f;
+        if (b < B) {
+          for (int i = t; i < g.K / 4; i += kConsumerThreads) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * ld) + i);
+            ss[b] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+          }
+        }
+        ss[b] = warp_sum(ss[b]);
+      }
+      if (lane == 0)
+#pragma unroll
+        for (int b = 0; b < kMaxBatch; ++b) ctl->aml[warp * kMaxBatch + b] = ss[b];
+      consumer_bar();
+      if (t < B) {
+        float tot = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) tot += ctl->aml[w * kMaxBatch + t];
+        scale[t] = 1.f / sqrtf(tot / (float)g.K + p.eps);
+      }
+    }
+    uint8_t* xs = ring + (size_t)NST * kStageBytes;
+    const uint32_t xpitch = (uint32_t)g.bKs * 2u + 16u;
+    const int gq = lane >> 2, cq = lane & 3;
+    if (tr) tr[4] = globaltimer();
+    int buf = 0;
+    for (int sl = 0; sl < g.bks; ++sl) {
+      consumer_bar();  // previous slice's fragments read; scales visible
+      // bf16 input slice of every sequence: xs[b][k], k < bKs
+      const int nvec = g.bKs / 8;
+      for (int idx = t; idx < B * nvec; idx += kConsumerThreads) {
+        const int b = idx / nvec, v = idx % nvec;
+        const size_t col = (size_t)sl * g.bKs + (size_t)v * 8;
+        const float4 x0 = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * ld + col));
+        const float4 x1 = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * ld + col) + 1);
+        float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        if (NORM) {
+          float gf[8];
+          unpack8(__ldg(reinterpret_cast<const uint4*>(gain + col)), gf);
+          const float sc = scale[b];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xv[e] = xv[e] * sc * gf[e];
+        }
+        uint4 o;
+        o.x = pack_bf16x2(xv[0], xv[1]);
+        o.y = pack_bf16x2(xv[2], xv[3]);
+        o.z = pack_bf16x2(xv[4], xv[5]);
+        o.w = pack_bf16x2(xv[6], xv[7]);
+        *reinterpret_cast<uint4*>(xs + (size_t)b * xpitch + (size_t)v * 16) = o;
+      }
+      consumer_bar();
+      for (int tile = 0; tile < g.bntiles; ++tile) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f}, du[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < g.bnchunk; ++j) {
+          const int width = min(g.bKc, g.bKs - j * g.bKc);
+          const uint32_t pitch = (uint32_t)width * 2u + 16u;
+          const uint8_t* st = wait_full();
+          if (tr && sl == 0 && tile == 0 && j == 0) tr[5] = globaltimer();
+          const uint8_t* wrow = st + (size_t)gq * pitch + cq * 4;
+          const uint8_t* xrow = xs + (size_t)gq * xpitch + (size_t)j * g.bKc * 2 + cq * 4;
+          for (int ks = warp; ks < width / 16; ks += kConsumerWarps) {
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(xrow + ks * 32);
+            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(xrow + ks * 32 + 16);
+            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wrow + ks * 32);
+            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wrow + ks * 32 + 16);
+            mma16816(d, a0, 0u, a2, 0u, b0, b1);
+            if (GATED) {
+              const uint32_t u0 = *reinterpret_cast<const uint32_t*>(wrow + 8 * pitch + ks * 32);
+              const uint32_t u1 = *reinterpret_cast<const uint32_t*>(wrow + 8 * pitch + ks * 32 + 16);
+              mma16816(du, a0, 0u, a2, 0u, u0, u1);
+            }
+          }
+          release();
+        }
+        // D[b = gq][rows 2cq, 2cq+1] of this warp
+        float* pw = red2 + (buf * kConsumerWarps + warp) * 128;
+        pw[gq * 8 + 2 * cq] = d[0];
+        pw[gq * 8 + 2 * cq + 1] = d[1];
+        if (GATED) {
+          pw[64 + gq * 8 + 2 * cq] = du[0];
+          pw[64 + gq * 8 + 2 * cq + 1] = du[1];
+        }
+        consumer_bar();
+        if (t < 64 * NM) {
+          const int which = t >> 6, b = (t & 63) >> 3, rr = t & 7;
+          float v = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) v += red2[(buf * kConsumerWarps + w) * 128 + which * 64 + b * 8 + rr];
+          float* o = oacc + (tile * 8 + rr) * 16 + which * 8 + b;
+          *o = (sl ? *o : 0.f) + v;
+        }
+        buf ^= 1;
+      }
+    }
+    if (tr) tr[6] = globaltimer();
+    consumer_bar();
+    const int qkvw = p.nq * p.hd + 2 * p.nkv * p.hd;
+    for (int idx = t; idx < nrows * B; idx += kConsumerThreads) {
+      const int rr = idx / B, b = idx % B, row = g.r0 + rr;
+      const float y = oacc[rr * 16 + b];
+      if (GATED) {
+        const float u = oacc[rr * 16 + 8 + b];
+        p.act[(size_t)b * p.I + row] = y / (1.f + expf(-y)) * u;
+      } else if (op == OP_QKV) {
+        p.qkv[(size_t)b * qkvw + row] = y;
+      } else if (op == OP_OPROJ) {
+        const size_t o = (size_t)b * p.H + row;
+        p.xres[(size_t)(2 * layer + 1) * BH + o] = __ldcg(p.xres + (size_t)(2 * layer) * BH + o) + y;
+      } else if (op == OP_DOWN) {
+        const size_t o = (size_t)b * p.H + row;
+        p.xres[(size_t)(2 * layer + 2) * BH + o] = __ldcg(p.xres + (size_t)(2 * layer + 1) * BH + o) + y;
+      } else {
+        p.logits[(size_t)b * p.V + row] = y;
+      }
+    }
+    return true;
+  }
+
   __device__ __forceinline__ bool gemv(const mk_instr& in, int op, int layer) {
+    if constexpr (BATCHED) {
+      if (op == OP_GATEUP) return gemv_mma<true, true>(in, op, layer);
+      if (op == OP_QKV || op == OP_LMHEAD) return gemv_mma<true, false>(in, op, layer);
+      return gemv_mma<false, false>(in, op, layer);
+    }
     const bool norm = op == OP_QKV || op == OP_GATEUP || op == OP_LMHEAD;
     const int K = op == OP_OPROJ ? p.nq * p.hd : (op == OP_DOWN ? p.I : p.H);
     const int nm = op == OP_GATEUP ? 2 : 1;
@@ -1170,8 +1398,10 @@ struct Consumer {
   }
 };
 
-__device__ __forceinline__ void run_consumers(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring, float* red) {
-  Consumer cs(p, ctl, ring, red);
+template <bool BATCHED>
+__device__ __forceinline__ void run_consumers(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring,
+                                              float* red) {
+  Consumer<BATCHED> cs(p, ctl, ring, red);
   uint64_t* trace = p.trace && threadIdx.x == 0 ? p.trace + (size_t)p.offsets[blockIdx.x] * kTraceStamps : nullptr;
   for (int i = 0; i < n; ++i) {
     const mk_instr in = list[i];
@@ -1215,14 +1445,16 @@ __device__ __forceinline__ void run_consumers(const Params& p, const mk_instr* l
   }
 }
 
+template <bool BATCHED>
 __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_constant__ Params p) {
+  using SM = Smem<BATCHED>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
-  float* red = reinterpret_cast<float*>(smem + kRingBytes);
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + kRingBytes + kRedBytes);
+  float* red = reinterpret_cast<float*>(smem + SM::kRing + SM::kXs);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + SM::kRing + SM::kXs + SM::kRed);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < SM::kNst; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], kConsumerWarps);
     }
@@ -1247,29 +1479,39 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
   const int n = p.offsets[blockIdx.x + 1] - p.offsets[blockIdx.x];
   const mk_instr* list = p.instrs + p.offsets[blockIdx.x];
   if (threadIdx.x >= kConsumerThreads) {
-    if (threadIdx.x == kConsumerThreads) run_producer(p, list, n, ctl, ring);
+    if (threadIdx.x == kConsumerThreads) run_producer<BATCHED>(p, list, n, ctl, ring);
   } else {
-    run_consumers(p, list, n, ctl, ring, red);
+    run_consumers<BATCHED>(p, list, n, ctl, ring, red);
   }
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-size_t kernel_smem_bytes() { return kSmemBytes; }
+size_t kernel_smem_bytes(bool batched) { return batched ? Smem<true>::kTotal : Smem<false>::kTotal; }
 
 cudaError_t kernel_prepare() {
-  return cudaFuncSetAttribute(mk_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(mk_persistent<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Smem<false>::kTotal);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(mk_persistent<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)Smem<true>::kTotal);
 }
 
-cudaError_t kernel_occupancy(int* blocks_per_sm) {
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_persistent, kThreads, kSmemBytes);
+cudaError_t kernel_occupancy(int* blocks_per_sm, bool batched) {
+  return batched ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_persistent<true>, kThreads,
+                                                                 Smem<true>::kTotal)
+                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_persistent<false>, kThreads,
+                                                                 Smem<false>::kTotal);
 }
 
 cudaError_t launch_step(const Params& p, int n_blocks, cudaStream_t stream) {
   void* args[] = {const_cast<Params*>(&p)};
-  return cudaLaunchCooperativeKernel((const void*)mk_persistent, dim3(n_blocks), dim3(kThreads), args, kSmemBytes,
-                                     stream);
+  if (p.B > 1)
+    return cudaLaunchCooperativeKernel((const void*)mk_persistent<true>, dim3(n_blocks), dim3(kThreads), args,
+                                       Smem<true>::kTotal, stream);
+  return cudaLaunchCooperativeKernel((const void*)mk_persistent<false>, dim3(n_blocks), dim3(kThreads), args,
+                                     Smem<false>::kTotal, stream);
 }
 
 }  // namespace mk

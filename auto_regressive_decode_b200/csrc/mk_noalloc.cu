@@ -98,9 +98,9 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-      mk::kernel_occupancy(&per_sm) != cudaSuccess)
+      mk::kernel_occupancy(&per_sm, d.batch > 1) != cudaSuccess)
     return MK_ERR_CUDA;
-  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes() || per_sm < 1) return MK_ERR_UNSUPPORTED;
+  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes(d.batch > 1) || per_sm < 1) return MK_ERR_UNSUPPORTED;
 
   mk_plan* plan = nullptr;
   rc = mk_plan_create(desc, n_sm, &plan);

@@ -46,7 +46,7 @@ int validate_desc(const mk_model_desc* d) {
   const int g = d->n_q_heads / d->n_kv_heads;
   if (g != 1 && g != 2 && g != 4 && g != 8) return MK_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128) return MK_ERR_UNSUPPORTED;
-  if (d->batch > 1) return MK_ERR_UNSUPPORTED;  // batch > 1 needs the tensor-core projections
+  if (d->batch > kMaxBatch) return MK_ERR_UNSUPPORTED;
   if (d->n_experts) return MK_ERR_UNSUPPORTED;   // MoE lowering not built yet
   if (d->ffn_dim <= 0) return MK_ERR_INVALID_ARG;
   const int qd = d->n_q_heads * d->head_dim;
@@ -55,6 +55,12 @@ int validate_desc(const mk_model_desc* d) {
   // GEMVs with an RMSNorm prologue (K = hidden) read whole rows in one pass
   if (gemv_ksplit(d->hidden, 1) != 1 || gemv_ksplit(d->hidden, 2) != 1) return MK_ERR_UNSUPPORTED;
   if ((int64_t)d->max_ctx * d->head_dim > (1ll << 31)) return MK_ERR_UNSUPPORTED;
+  if (d->batch > 1) {
+    // tensor-core GEMVs: k-steps of 16 and input slices of at most kBatchedSlice columns
+    const int ks[3] = {d->hidden, qd, d->ffn_dim};
+    for (int K : ks)
+      if (K % 16 || bgemv_slices(K) == 0) return MK_ERR_UNSUPPORTED;
+  }
   return MK_OK;
 }
 
@@ -81,10 +87,11 @@ struct Builder {
   int rows_op(int op, int layer, int N, const std::vector<int>& cuts, int wait_idx, int wait_count, int sig_idx) {
     int n = 0;
     const int n_sm = p->n_sm;
+    const int max_rows = p->d.batch > 1 ? kBatchedMaxRows : kMaxRows;
     for (int s = 0; s < n_sm; ++s) {
       int r0 = (int)((int64_t)N * s / n_sm), r1 = (int)((int64_t)N * (s + 1) / n_sm);
       while (r0 < r1) {
-        int e = std::min(r1, r0 + kMaxRows);
+        int e = std::min(r1, r0 + max_rows);
         int seg = 0, base = 0;
         for (size_t k = 0; k < cuts.size(); ++k) {
           if (r0 >= cuts[k]) { seg = (int)k + 1; base = cuts[k]; }

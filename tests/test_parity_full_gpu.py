@@ -56,3 +56,49 @@ def test_dense_8b_sampled_layers_and_logits():
     ref = model.lm_head(hid[2 * cfg.n_layers, 0])
     assert float(np.max(np.abs(lg - ref))) <= TOL_LOGITS_ABS
     assert int(np.argmax(lg)) == int(np.argmax(ref))
+
+
+def test_dense_13b_batch8_ragged_sampled_layers_and_logits():
+    """13B shape, batch 8 with ragged contexts in [256, 4096]: tensor-core projections."""
+    import auto_regressive_decode_b200.mk as mk
+    cfg = fx.CONFIGS["dense-13b-b8"]
+    S0 = fx.context_lengths(cfg)
+    tok = fx.tokens(cfg)[0]
+    w = device_model(cfg)
+    kc, vc = device_caches(cfg, S0)
+    dec = mk.Decoder(cfg, w, kc, vc)
+    logits = torch.empty((cfg.batch, cfg.vocab), dtype=torch.float32, device="cuda")
+    d_tok = torch.from_numpy(tok.copy()).cuda()
+    d_len = torch.from_numpy(S0.copy()).cuda()
+    dec.step(d_tok, d_len, d_len, logits)
+    assert dec.status() == mk.MK_OK
+    hid = dec.hidden_states().cpu().numpy().astype(np.float64)
+    lg = logits.cpu().numpy().astype(np.float64)
+    layers = (0, 39)
+    new_rows = {}
+    for l in layers:
+        for b in range(cfg.batch):
+            S = int(S0[b])
+            new_rows[(l, b)] = (bf16_f64(bits(kc[l, b, :, S].contiguous())), bf16_f64(bits(vc[l, b, :, S].contiguous())))
+    dec.close()
+    del w, kc, vc
+    torch.cuda.empty_cache()
+
+    g, ls = host_model(cfg, layers=layers)
+    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls)
+    for l in layers:
+        okc = fx.kv_prefill(cfg, l, 0, S0)
+        ovc = fx.kv_prefill(cfg, l, 1, S0)
+        out = model.layer_forward(l, hid[2 * l].copy(), okc, ovc, S0, S0)
+        assert rel_l2(hid[2 * l + 1], out["h_attn"]) <= TOL_HIDDEN, l
+        assert rel_l2(hid[2 * l + 2], out["h_mlp"]) <= TOL_HIDDEN, l
+        for b in range(cfg.batch):
+            S = int(S0[b])
+            assert rel_l2(new_rows[(l, b)][0], bf16_f64(okc[b, :, S])) <= TOL_KV
+            assert rel_l2(new_rows[(l, b)][1], bf16_f64(ovc[b, :, S])) <= TOL_KV
+    top1 = 0
+    for b in range(cfg.batch):
+        ref = model.lm_head(hid[2 * cfg.n_layers, b])
+        assert float(np.max(np.abs(lg[b] - ref))) <= TOL_LOGITS_ABS
+        top1 += int(np.argmax(lg[b]) == np.argmax(ref))
+    assert top1 == cfg.batch

@@ -40,3 +40,24 @@ def test_tiny_last_cache_slot():
 
 def test_dense_0_6b_first_steps():
     assert_parity(run_teacher_forced(fx.CONFIGS["dense-0.6b"], steps=3))
+
+
+# ---- batch > 1 (tensor-core projections) -------------------------------------------------------
+
+@pytest.mark.parametrize("kw,gains", [
+    ({"batch": 4, "ctx": 0, "ctx_lo": 3, "ctx_hi": 60, "steps": 3}, "random"),
+    ({"batch": 8, "ctx": 0, "steps": 2}, "ones"),                                    # empty caches
+    ({"batch": 2, "n_q_heads": 8, "n_kv_heads": 1, "qk_norm": True, "tied_embeddings": True}, "random"),
+    ({"batch": 3, "ctx": 0, "ctx_lo": 250, "ctx_hi": 260, "steps": 3}, "ones"),    # chunk boundary, ragged
+])
+def test_tiny_batched(kw, gains):
+    cfg = fx.CONFIGS["tiny"].replace(**kw)
+    assert_parity(run_teacher_forced(cfg, steps=kw.get("steps", 3), gains=gains))
+
+
+def test_batched_multi_slice_multi_chunk():
+    # MHA, head_dim 128; the down projection (K = 4608) runs as 2 input slices of
+    # 2 column chunks each, the other projections as 1 slice / 1 chunk
+    cfg = fx.ModelConfig("mid-b8", n_layers=3, hidden=640, n_q_heads=5, n_kv_heads=5, head_dim=128, ffn_dim=4608,
+                         vocab=2000, batch=8, ctx_lo=10, ctx_hi=300, steps=3)
+    assert_parity(run_teacher_forced(cfg, gains="random"))
