@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["mk_kernel.cu", "mk_api.cu", "mk_plan.cpp", "mk_noalloc.cu"]
+SOURCES = ["mk_kernel.cu", "mk_api.cu", "mk_plan.cpp", "mk_noalloc.cu", "mk_tmap.cu"]
 HEADERS = ["mk_internal.h", "mk_device.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-Xcompiler", "-fPIC",

@@ -139,6 +139,8 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const size_t o_off = cv.take(sizeof(int32_t) * offsets.size());
   const size_t o_lay = cv.take(sizeof(mk::LayerPtrs) * (size_t)L);
   const size_t o_rope = cv.take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
+  const size_t n_tmaps = B > 1 ? (size_t)mk::kTmapsPerLayer * L + 1 : 0;
+  const size_t o_tmap = n_tmaps ? cv.take(128 * n_tmaps) : 0;
   const char* trace_env = getenv("MK_TRACE");
   const bool tracing = trace_env && atoi(trace_env) > 0;
   const size_t o_trace = tracing ? cv.take(sizeof(uint64_t) * mk::kTraceStamps * instrs.size()) : 0;
@@ -175,7 +177,17 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
       rope[(size_t)pos * (hd / 2) + i] = make_float2((float)cos(ang), (float)sin(ang));
     }
 
+  std::vector<uint8_t> tmaps(128 * n_tmaps);
+  if (n_tmaps) {
+    const cudaError_t te = mk::encode_weight_tmaps(d, *w, tmaps.data());
+    if (te != cudaSuccess) {
+      cudaFree(h->region);
+      delete h;
+      return te == cudaErrorInvalidValue ? MK_ERR_UNSUPPORTED : MK_ERR_CUDA;
+    }
+  }
   bool ok = cudaMemset(base, 0, h->region_bytes) == cudaSuccess &&
+            (!n_tmaps || cudaMemcpy(base + o_tmap, tmaps.data(), tmaps.size(), cudaMemcpyHostToDevice) == cudaSuccess) &&
             cudaMemcpy(base + o_ins, instrs.data(), sizeof(mk_instr) * instrs.size(), cudaMemcpyHostToDevice) ==
                 cudaSuccess &&
             cudaMemcpy(base + o_off, offsets.data(), sizeof(int32_t) * offsets.size(), cudaMemcpyHostToDevice) ==
@@ -211,6 +223,7 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   p.kc = (uint16_t*)kv->k;
   p.vc = (uint16_t*)kv->v;
   p.rope = (const float2*)(base + o_rope);
+  p.tmaps = n_tmaps ? base + o_tmap : nullptr;
   p.xres = (float*)(base + o_xres);
   p.qkv = (float*)(base + o_qkv);
   p.attn = (float*)(base + o_attn);

@@ -38,8 +38,7 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;  // 256
 constexpr int kThreads = kConsumerThreads + 32;        // + one producer warp
 constexpr int kStageBytes = 32 * 1024;                 // one ring slot
 constexpr int kStages = 6;                             // ring depth (192 KB), batch-1 kernel
-constexpr int kStagesBatched = 4;                      // ring depth of the batch > 1 kernel (128 KB)
-constexpr int kXsPitchBytes = 4096 * 2 + 16;           // batch > 1: one sequence's bf16 input slice (padded)
+constexpr int kStagesBatched = 6;                      // ring depth of the batch > 1 kernel
 constexpr int kMaxRows = 256;                          // rows per GEMV instruction
 constexpr int kRedFloats = 4096;                       // cross-warp reduction buffer
 constexpr int kMaxBatch = 8;
@@ -111,18 +110,21 @@ MK_HD int gemv_ksplit(int K, int n_mats) {
 }
 
 // ---- batch > 1 GEMV (tensor cores) -------------------------------------------------
-// Stages hold up to 8 weight rows (16 for the gate/up pair) of one column
-// chunk, each row at a pitch of chunk*2 + 16 bytes (conflict-free fragment
-// loads); the bf16 inputs of all sequences hold one column slice of at most
-// kBatchedSlice columns at a time.
-constexpr int kBatchedMaxRows = 64;   // rows per batched GEMV instruction (8 tiles of 8)
-constexpr int kBatchedSlice = 4096;   // input columns per slice
-MK_HD int bgemv_chunk(int n_mats) { return n_mats == 2 ? 960 : 1984; }
-MK_HD int bgemv_slices(int K) {
-  for (int ks = 1; ks <= 16; ++ks)
-    if (K % ks == 0 && (K / ks) % 16 == 0 && K / ks <= kBatchedSlice) return ks;
-  return 0;
-}
+// A stage is one tile of 16 A-operand rows (16 weight rows, or 8 gate rows over
+// the same 8 up rows) for one chunk of kBChunk input columns, moved as two TMA
+// boxes of kBBoxRows rows each.  A weight matrix [N][K] is viewed by its tensor
+// map as a 3-D tensor (64 columns, N rows, K/64 column blocks), so that a box
+// lands as [column block][row][64] with 128-byte rows swizzled (16-byte chunk
+// c of line L stored at chunk c ^ (L & 7)): the eight row reads of an ldmatrix
+// phase hit distinct bank groups.  An instruction streams chunk by chunk, and
+// tile by tile within a chunk; row ranges are cut at multiples of kBBoxRows.
+constexpr int kBChunk = 1024;                        // input columns per stage
+constexpr int kBBoxRows = 8;                         // weight rows per TMA box
+constexpr int kBBoxBytes = kBBoxRows * kBChunk * 2;  // 16 KB
+constexpr int kBatchedMaxRows = 128;                 // rows per instruction: 8 tiles of 16
+constexpr int kBatchedMaxRowsGated = 96;             // gate/up: 12 tiles of 8 neurons
+constexpr int kTmapsPerLayer = 7;                    // wq wk wv wo w_gate w_up w_down (+ one LM head map)
+MK_HD int btile_rows(bool gated) { return gated ? 8 : 16; }
 
 // ---- attention split -------------------------------------------------------------
 // Query heads one attention instruction handles: a KV head with more query

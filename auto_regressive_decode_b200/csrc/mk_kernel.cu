@@ -50,15 +50,18 @@ struct Ctl {
   alignas(16) uint16_t vnew[kMaxHeadDim];
 };
 
-// Shared memory: the ring, then (batched kernel only) the bf16 input-vector
-// slice for the tensor-core GEMV, then the reduction buffer and Ctl.
+// Shared memory: the ring of weight / KV stages (slots 1024-byte aligned, as
+// the swizzled TMA boxes of the batched GEMV need), the reduction buffer, Ctl.
 template <bool BATCHED>
 struct Smem {
   static constexpr int kNst = BATCHED ? kStagesBatched : kStages;
-  static constexpr size_t kRing = (size_t)kNst * kStageBytes;
-  static constexpr size_t kXs = BATCHED ? (size_t)kMaxBatch * kXsPitchBytes : 0;
+  static constexpr size_t kSlot = (size_t)kStageBytes;
+  static_assert(2 * kBBoxBytes == kStageBytes, "a batched GEMV stage is two boxes");
+  static constexpr size_t kRing = (size_t)kNst * kSlot;
   static constexpr size_t kRed = (size_t)kRedFloats * sizeof(float);
-  static constexpr size_t kTotal = kRing + kXs + kRed + sizeof(Ctl);
+  static constexpr size_t kTotal = kRing + kRed + sizeof(Ctl);
+  static_assert(kNst <= kStages, "Ctl holds kStages barrier pairs");
+  static_assert(kTotal <= 227 * 1024, "dynamic shared memory of one CTA");
 };
 
 // ---------------------------------------------------------------------------
@@ -100,6 +103,17 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
 }
 
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// One box of a 3-D tensor map (coordinates c0, c1, c2) into shared memory,
+// completing on `bar`.
+__device__ __forceinline__ void tma_box3(void* dst, const void* map, int c0, int c1, int c2, unsigned long long* bar,
+                                         uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar)), "l"(pol)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar,
                                          uint64_t pol) {
   asm volatile(
@@ -275,8 +289,21 @@ __device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, u
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Two fp32 values rounded to nearest-even bf16, `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return (uint32_t)f32_to_bf16_bits_fwd(lo) | ((uint32_t)f32_to_bf16_bits_fwd(hi) << 16);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Four 8x8 b16 matrices from shared memory; lane l supplies the address of
+// row (l & 7) of matrix (l >> 3) and receives element pair (l >> 2, 2 * (l & 3))
+// of every matrix: exactly an m16n8k16 A fragment when the matrices are
+// (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15).
+__device__ __forceinline__ void ldmatrix_x4(uint32_t a[4], uint32_t saddr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(saddr));
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
@@ -305,9 +332,9 @@ struct Gemv {
   int K, r0, r1;
   int ks, Kc;                       // column slices per row, slice width (K = ks * Kc)
   GemvTile tile;                    // tiling of one slice
-  // batch > 1 (tensor cores): bks slices of bKs columns, chunks of bKc
-  // columns per stage (bnchunk per slice), 8-row tiles (bntiles)
-  int bks, bKs, bKc, bnchunk, bntiles;
+  // batch > 1 (tensor cores): bnch chunks of kBChunk columns, bnt tiles of
+  // btile_rows() output rows
+  int bnch, bnt;
   __device__ __forceinline__ const uint16_t* seg_ptr(int s) const { return s == 0 ? sw0 : (s == 1 ? sw1 : sw2); }
   // first element of row r0 + rel (rel < r1 - r0), whichever matrix holds it
   __device__ __forceinline__ const uint16_t* row_ptr(int rel) const {
@@ -373,11 +400,9 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
   g.Kc = g.K / g.ks;
   g.tile = gemv_tile(g.Kc, g.wup ? 2 : 1);
   if (p.B > 1) {
-    g.bks = bgemv_slices(g.K);
-    g.bKs = g.K / g.bks;
-    g.bKc = bgemv_chunk(g.wup ? 2 : 1);
-    g.bnchunk = (g.bKs + g.bKc - 1) / g.bKc;
-    g.bntiles = (g.r1 - g.r0 + 7) / 8;
+    const int tr = btile_rows(g.wup != nullptr);
+    g.bnch = (g.K + kBChunk - 1) / kBChunk;
+    g.bnt = (g.r1 - g.r0 + tr - 1) / tr;
   }
   return g;
 }
@@ -421,9 +446,9 @@ struct Cursor {
   const mk_instr* list;
   int n;
   int i;  // instruction index; >= n when every stage has been walked
-  int op;
+  int op, layer;
   Gemv g;
-  int kc, sg, rr;  // GEMV: slice, segment, first row within the segment
+  int kc, sg, rr;  // GEMV: slice (batched: chunk), segment (batched: tile), first row within the segment
   Attn a;
   int sub, kv;     // attention: sub-chunk, K (0) or V (1)
 
@@ -434,7 +459,7 @@ struct Cursor {
     for (i = j; i < n; ++i) {
       const mk_instr in = list[i];
       op = op_of(in.op_layer);
-      const int layer = layer_of(in.op_layer);
+      layer = layer_of(in.op_layer);
       if (op == OP_ATTN) {
         a = attn_geo(*pp, in, layer, pp->hd);
         sub = kv = 0;
@@ -453,13 +478,10 @@ struct Cursor {
       if (!kv && ++sub >= a.nsub) seek(i + 1);
       return;
     }
-    if (pp->B > 1) {  // batched GEMV: (slice kc, tile sg, chunk rr)
-      if (++rr >= g.bnchunk) {
-        rr = 0;
-        if (++sg >= g.bntiles) {
-          sg = 0;
-          if (++kc >= g.bks) seek(i + 1);
-        }
+    if (pp->B > 1) {  // batched GEMV: chunk kc, tile sg within it
+      if (++sg >= g.bnt) {
+        sg = 0;
+        if (++kc >= g.bnch) seek(i + 1);
       }
       return;
     }
@@ -483,18 +505,6 @@ struct Cursor {
       for (uint32_t o = 0; o < bytes; o += pp->copy_piece) f(src + o / 2, min(pp->copy_piece, bytes - o), o);
       return bytes;
     }
-    if (pp->B > 1) {
-      // up to 8 rows (tile sg) of column chunk rr of slice kc, one copy per row
-      const int nr = min(8, g.r1 - g.r0 - sg * 8);
-      const int width = min(g.bKc, g.bKs - rr * g.bKc);
-      const uint32_t pitch = (uint32_t)width * 2u + 16u, bytes = (uint32_t)width * 2u;
-      const size_t col = (size_t)kc * g.bKs + (size_t)rr * g.bKc;
-      for (int r = 0; r < nr; ++r) {
-        f(g.row_ptr(sg * 8 + r) + col, bytes, (uint32_t)r * pitch);
-        if (g.wup) f(g.wup + (size_t)(sg * 8 + r) * g.K + col, bytes, (uint32_t)(8 + r) * pitch);
-      }
-      return (uint32_t)nr * bytes * (g.wup ? 2u : 1u);
-    }
     const int R = g.tile.rows_per_stage;
     const int nr = min(R, g.seg_rows(sg) - rr);
     const uint32_t seg = (uint32_t)g.Kc * 2u;
@@ -515,11 +525,41 @@ struct Cursor {
     return g.wup ? 2 * bytes : bytes;
   }
 
+  // Batched GEMV stage: f(tensor map, row, column block, shared-memory
+  // offset) per TMA box: the two 8-row halves of 16-row tile sg (the second
+  // only if the tile has more than 8 rows), or gate over up rows of 8-row tile
+  // sg, at column chunk kc.  Returns the stage's bytes.
+  template <typename F>
+  __device__ __forceinline__ uint32_t boxes(F&& f) const {
+    const Params& p = *pp;
+    const int kb = kc * (kBChunk / 64);
+    if (g.wup) {
+      const uint8_t* m = p.tmaps + ((size_t)layer * kTmapsPerLayer + 4) * 128;
+      const int row = g.r0 + sg * 8;
+      f(m, row, kb, 0u);
+      f(m + 128, row, kb, (uint32_t)kBBoxBytes);
+      return 2u * kBBoxBytes;
+    }
+    const int nh = g.r1 - g.r0 - sg * 16 > 8 ? 2 : 1;
+    for (int h = 0; h < nh; ++h) {
+      int row = g.r0 + sg * 16 + h * 8, m;
+      if (op == OP_QKV) {
+        const int qd = p.nq * p.hd, kvd = p.nkv * p.hd;
+        m = row < qd ? 0 : (row < qd + kvd ? 1 : 2);
+        row -= m == 0 ? 0 : (m == 1 ? qd : qd + kvd);
+      } else {
+        m = op == OP_OPROJ ? 3 : 6;
+      }
+      const uint8_t* map = op == OP_LMHEAD ? p.tmaps + (size_t)p.L * kTmapsPerLayer * 128
+                                           : p.tmaps + ((size_t)layer * kTmapsPerLayer + m) * 128;
+      f(map, row, kb, (uint32_t)(h * kBBoxBytes));
+    }
+    return (uint32_t)nh * kBBoxBytes;
+  }
+
   __device__ __forceinline__ uint32_t stage_bytes() const {
     if (op == OP_ATTN) return (uint32_t)min(a.P, a.n_cached - sub * a.P) * pp->hd * 2u;
-    if (pp->B > 1)
-      return (uint32_t)min(8, g.r1 - g.r0 - sg * 8) * (uint32_t)min(g.bKc, g.bKs - rr * g.bKc) * 2u *
-             (g.wup ? 2u : 1u);
+    if (pp->B > 1) return (g.wup || g.r1 - g.r0 - sg * 16 > 8) ? 2u * kBBoxBytes : (uint32_t)kBBoxBytes;
     const uint32_t b = (uint32_t)min(g.tile.rows_per_stage, g.seg_rows(sg) - rr) * (uint32_t)g.Kc * 2u;
     return g.wup ? 2 * b : b;
   }
@@ -541,11 +581,14 @@ struct Producer {
     pol = evict_first_policy();
   }
 
-  // While blocked on the ring: prefetch the next stages into L2, up to Params::l2_ahead bytes.
+  // While blocked on the ring: prefetch the next stages into L2, up to
+  // Params::l2_ahead bytes (batch-1 kernel only).
   __device__ __forceinline__ void prefetch_ahead() {
-    while (pf_ahead < p.l2_ahead && pf.i < pf.n) {
-      pf_ahead += pf.copies([&](const uint16_t* src, uint32_t bytes, uint32_t) { prefetch_l2(src, bytes); });
-      pf.advance();
+    if constexpr (!BATCHED) {
+      while (pf_ahead < p.l2_ahead && pf.i < pf.n) {
+        pf_ahead += pf.copies([&](const uint16_t* src, uint32_t bytes, uint32_t) { prefetch_l2(src, bytes); });
+        pf.advance();
+      }
     }
   }
 
@@ -572,7 +615,7 @@ struct Producer {
         }
       }
     }
-    *dst = ring + (size_t)slot * kStageBytes;
+    *dst = ring + (size_t)slot * Smem<BATCHED>::kSlot;
     *bar = &ctl->full[slot];
     return true;
   }
@@ -589,6 +632,7 @@ struct Producer {
   }
 };
 
+// One thread (lane 0 of the producer warp) issues every copy.
 template <bool BATCHED>
 __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
   Producer<BATCHED> pr(p, ctl, ring, list, n);
@@ -610,7 +654,13 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
     if (!(ok = pr.claim(&dst, &bar))) break;
     const uint32_t bytes = cur.stage_bytes();
     mbar_arrive_expect_tx(bar, bytes);
-    cur.copies([&](const uint16_t* src, uint32_t b, uint32_t off) { bulk_g2s(dst + off, src, b, bar, pr.pol); });
+    if (BATCHED && cur.op != OP_ATTN) {
+      cur.boxes([&](const uint8_t* map, int row, int kb, uint32_t off) {
+        tma_box3(dst + off, map, 0, row, kb, bar, pr.pol);
+      });
+    } else {
+      cur.copies([&](const uint16_t* src, uint32_t b, uint32_t off) { bulk_g2s(dst + off, src, b, bar, pr.pol); });
+    }
     ++pr.k;
     cur.advance();
     if (pr.pf_ahead > bytes) {
@@ -665,7 +715,7 @@ struct Consumer {
         }
       }
     }
-    return ring + (size_t)slot * kStageBytes;
+    return ring + (size_t)slot * Smem<BATCHED>::kSlot;
   }
 
   __device__ __forceinline__ void release() {
@@ -925,18 +975,23 @@ struct Consumer {
     return gemv_nv<(NORM ? 4 : 8), NORM, GATED>(in, op, layer, rpt);
   }
 
-  // Ops with an RMSNorm prologue read the hidden vector (K = hidden, at most
-  // 4 vectors per thread, checked at creation); o_proj and down read attn / act.
   // ---- GEMV, batch > 1: tensor cores ---------------------------------------
-  // mma.m16n8k16: A = the bf16 inputs of the batch (rows b < B of 16), B = 8
-  // weight rows of the stage, D[b][row] accumulated in fp32.  Warps share a
-  // stage's k-steps; per 8-row tile the partials are summed across warps in a
-  // fixed order, per column slice into oacc (shared memory).
+  // mma.m16n8k16 with A = a stage tile of 16 weight rows (ldmatrix from the
+  // ring), B = the bf16 inputs of the batch (n = sequence, columns b >= B are
+  // zero), D[row][b] in fp32 registers.  Warps split each chunk's k-steps
+  // between them and keep every tile's partial sums in registers for the
+  // whole instruction; one cross-warp reduction in a fixed order ends it.
+  // The inputs of a chunk are fragments in registers, loaded (fp32, from L2)
+  // one chunk ahead.  RMSNorm: the gain is applied to the inputs, and the
+  // per-sequence 1/rms factor, whose sum of squares accumulates from the same
+  // loads, scales the outputs in the epilogue (it is constant along K).
   template <bool NORM, bool GATED>
-  __device__ __forceinline__ bool gemv_mma(const mk_instr& in, int op, int layer) {
-    constexpr int NM = GATED ? 2 : 1;
+  __device__ __forceinline__ bool gemv_tc(const mk_instr& in, int op, int layer) {
+    constexpr int TR = GATED ? 8 : 16;  // output rows per tile
+    constexpr int MAXT = (GATED ? kBatchedMaxRowsGated : kBatchedMaxRows) / TR;
+    constexpr int KPW = kBChunk / 16 / kConsumerWarps;  // k-steps per warp per chunk
     const Gemv g = gemv_geo(p, in, op, layer);
-    const int B = p.B, BH = B * p.H, nrows = g.r1 - g.r0;
+    const int B = p.B, BH = B * p.H, nrows = g.r1 - g.r0, ntiles = g.bnt;
     const float* src;
     const uint16_t* gain = nullptr;
     int ld;  // elements per sequence in src
@@ -953,125 +1008,143 @@ struct Consumer {
     }
     if (!wait_counter(in.wait_idx, in.wait_count)) return false;
     if (tr) tr[1] = globaltimer();
-    float* red2 = red;               // [2][8 warps][NM*64] tile partials
-    float* oacc = red + 2 * 8 * 128;  // [64 rows][16] (gate: b, up: 8 + b)
-    float* scale = ctl->sred;         // [8] RMS scale per sequence
-    if (NORM) {
-      // per-sequence RMS over the whole vector (K = hidden): one block pass
-      float ss[kMaxBatch];
+    const int gq = lane >> 2, cq = lane & 3;
+    const bool bval = gq < B;  // this lane's B-fragment column (sequence gq) exists
+    const float* xrow = src + (size_t)(bval ? gq : 0) * ld;
+    float acc[MAXT][4];
 #pragma unroll
-      for (int b = 0; b < kMaxBatch; ++b) {
-        ss[b] = 0.f;
-        if (b < B) {
-          for (int i = t; i < g.K / 4; i += kConsumerThreads) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * ld) + i);
-            ss[b] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    for (int t2 = 0; t2 < MAXT; ++t2) acc[t2][0] = acc[t2][1] = acc[t2][2] = acc[t2][3] = 0.f;
+    float ss = 0.f;
+    float2 xr[KPW][2];
+    uint32_t gr[KPW][2];
+    uint32_t xf[KPW][2];
+    // raw inputs (and gains) of chunk j: k = 16 ks + 2 cq (+1) and + 8 (+1)
+    auto load = [&](int j) {
+      const int nks = min(kBChunk, g.K - j * kBChunk) / 16;
+#pragma unroll
+      for (int kk = 0; kk < KPW; ++kk) {
+        const int ks = warp + kk * kConsumerWarps;
+        const int k = j * kBChunk + ks * 16 + 2 * cq;
+        if (bval && ks < nks) {
+          xr[kk][0] = __ldcg(reinterpret_cast<const float2*>(xrow + k));
+          xr[kk][1] = __ldcg(reinterpret_cast<const float2*>(xrow + k + 8));
+          if (NORM) {
+            gr[kk][0] = __ldg(reinterpret_cast<const unsigned int*>(gain + k));
+            gr[kk][1] = __ldg(reinterpret_cast<const unsigned int*>(gain + k + 8));
+          }
+        } else {
+          xr[kk][0] = xr[kk][1] = make_float2(0.f, 0.f);
+          if (NORM) gr[kk][0] = gr[kk][1] = 0u;
+        }
+      }
+    };
+    load(0);
+    // ldmatrix row address of this lane within a stage: A-row R = lane & 15
+    // lives in box R >> 3 as row r = R & 7; k-step ks = warp + 8 kk reads
+    // column block (warp >> 2) + 2 kk, 16-byte chunk ((warp & 3) << 1) | (lane >> 4),
+    // stored at chunk position (chunk ^ r) of its 128-byte line.
+    const uint32_t rr7 = (uint32_t)(lane & 7), ch = ((uint32_t)(warp & 3) << 1) | (uint32_t)(lane >> 4);
+    const uint32_t lrow = (uint32_t)((lane >> 3) & 1) * kBBoxBytes + (uint32_t)(warp >> 2) * 1024u + rr7 * 128u +
+                          ((ch ^ rr7) << 4);
+    for (int j = 0; j < g.bnch; ++j) {
+      const int nks = min(kBChunk, g.K - j * kBChunk) / 16;
+#pragma unroll
+      for (int kk = 0; kk < KPW; ++kk) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 x = xr[kk][h];
+          if (NORM) {
+            ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
+            xf[kk][h] = pack_bf16x2(x.x * bf16_lo(gr[kk][h]), x.y * bf16_hi(gr[kk][h]));
+          } else {
+            xf[kk][h] = pack_bf16x2(x.x, x.y);
           }
         }
-        ss[b] = warp_sum(ss[b]);
       }
-      if (lane == 0)
+      if (tr && j == 0) tr[4] = globaltimer();
+      if (j + 1 < g.bnch) load(j + 1);
 #pragma unroll
-        for (int b = 0; b < kMaxBatch; ++b) ctl->aml[warp * kMaxBatch + b] = ss[b];
-      consumer_bar();
-      if (t < B) {
-        float tot = 0.f;
-        for (int w = 0; w < kConsumerWarps; ++w) tot += ctl->aml[w * kMaxBatch + t];
-        scale[t] = 1.f / sqrtf(tot / (float)g.K + p.eps);
-      }
-    }
-    uint8_t* xs = ring + (size_t)NST * kStageBytes;
-    const uint32_t xpitch = (uint32_t)g.bKs * 2u + 16u;
-    const int gq = lane >> 2, cq = lane & 3;
-    if (tr) tr[4] = globaltimer();
-    int buf = 0;
-    for (int sl = 0; sl < g.bks; ++sl) {
-      consumer_bar();  // previous slice's fragments read; scales visible
-      // bf16 input slice of every sequence: xs[b][k], k < bKs
-      const int nvec = g.bKs / 8;
-      for (int idx = t; idx < B * nvec; idx += kConsumerThreads) {
-        const int b = idx / nvec, v = idx % nvec;
-        const size_t col = (size_t)sl * g.bKs + (size_t)v * 8;
-        const float4 x0 = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * ld + col));
-        const float4 x1 = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * ld + col) + 1);
-        float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        if (NORM) {
-          float gf[8];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(gain + col)), gf);
-          const float sc = scale[b];
+      for (int t2 = 0; t2 < MAXT; ++t2) {
+        if (t2 < ntiles) {
+          const uint32_t st = smem_addr(wait_full()) + lrow;
+          if (tr && j == 0 && t2 == 0) tr[5] = globaltimer();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xv[e] = xv[e] * sc * gf[e];
-        }
-        uint4 o;
-        o.x = pack_bf16x2(xv[0], xv[1]);
-        o.y = pack_bf16x2(xv[2], xv[3]);
-        o.z = pack_bf16x2(xv[4], xv[5]);
-        o.w = pack_bf16x2(xv[6], xv[7]);
-        *reinterpret_cast<uint4*>(xs + (size_t)b * xpitch + (size_t)v * 16) = o;
-      }
-      consumer_bar();
-      for (int tile = 0; tile < g.bntiles; ++tile) {
-        float d[4] = {0.f, 0.f, 0.f, 0.f}, du[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < g.bnchunk; ++j) {
-          const int width = min(g.bKc, g.bKs - j * g.bKc);
-          const uint32_t pitch = (uint32_t)width * 2u + 16u;
-          const uint8_t* st = wait_full();
-          if (tr && sl == 0 && tile == 0 && j == 0) tr[5] = globaltimer();
-          const uint8_t* wrow = st + (size_t)gq * pitch + cq * 4;
-          const uint8_t* xrow = xs + (size_t)gq * xpitch + (size_t)j * g.bKc * 2 + cq * 4;
-          for (int ks = warp; ks < width / 16; ks += kConsumerWarps) {
-            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(xrow + ks * 32);
-            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(xrow + ks * 32 + 16);
-            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wrow + ks * 32);
-            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wrow + ks * 32 + 16);
-            mma16816(d, a0, 0u, a2, 0u, b0, b1);
-            if (GATED) {
-              const uint32_t u0 = *reinterpret_cast<const uint32_t*>(wrow + 8 * pitch + ks * 32);
-              const uint32_t u1 = *reinterpret_cast<const uint32_t*>(wrow + 8 * pitch + ks * 32 + 16);
-              mma16816(du, a0, 0u, a2, 0u, u0, u1);
+          for (int kk = 0; kk < KPW; ++kk) {
+            const int ks = warp + kk * kConsumerWarps;
+            if (ks < nks) {
+              uint32_t a[4];
+              ldmatrix_x4(a, st + (uint32_t)kk * 2048u);
+              mma16816(acc[t2], a[0], a[1], a[2], a[3], xf[kk][0], xf[kk][1]);
             }
           }
           release();
         }
-        // D[b = gq][rows 2cq, 2cq+1] of this warp
-        float* pw = red2 + (buf * kConsumerWarps + warp) * 128;
-        pw[gq * 8 + 2 * cq] = d[0];
-        pw[gq * 8 + 2 * cq + 1] = d[1];
-        if (GATED) {
-          pw[64 + gq * 8 + 2 * cq] = du[0];
-          pw[64 + gq * 8 + 2 * cq + 1] = du[1];
-        }
-        consumer_bar();
-        if (t < 64 * NM) {
-          const int which = t >> 6, b = (t & 63) >> 3, rr = t & 7;
-          float v = 0.f;
-#pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) v += red2[(buf * kConsumerWarps + w) * 128 + which * 64 + b * 8 + rr];
-          float* o = oacc + (tile * 8 + rr) * 16 + which * 8 + b;
-          *o = (sl ? *o : 0.f) + v;
-        }
-        buf ^= 1;
       }
     }
     if (tr) tr[6] = globaltimer();
-    consumer_bar();
+    if (NORM) {
+      // per-warp sum of squares of sequence gq (lanes cq = 0..3 hold disjoint columns)
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      if (cq == 0) ctl->aml[warp * kMaxBatch + gq] = ss;
+    }
+    // Cross-warp reduction, four tiles per round: warp w's partials of a tile
+    // at red[w * 512 + q * 128 + lane * 4 + e]; thread (q, l, i) then sums
+    // accumulator elements i and i + 2 of lane l over the warps.
+    const int q = t >> 6, l = (t >> 1) & 31, i = t & 1;
+    const int lgq = l >> 2, b = 2 * (l & 3) + i;
+    float sc = 1.f;
     const int qkvw = p.nq * p.hd + 2 * p.nkv * p.hd;
-    for (int idx = t; idx < nrows * B; idx += kConsumerThreads) {
-      const int rr = idx / B, b = idx % B, row = g.r0 + rr;
-      const float y = oacc[rr * 16 + b];
-      if (GATED) {
-        const float u = oacc[rr * 16 + 8 + b];
-        p.act[(size_t)b * p.I + row] = y / (1.f + expf(-y)) * u;
-      } else if (op == OP_QKV) {
-        p.qkv[(size_t)b * qkvw + row] = y;
-      } else if (op == OP_OPROJ) {
-        const size_t o = (size_t)b * p.H + row;
-        p.xres[(size_t)(2 * layer + 1) * BH + o] = __ldcg(p.xres + (size_t)(2 * layer) * BH + o) + y;
-      } else if (op == OP_DOWN) {
-        const size_t o = (size_t)b * p.H + row;
-        p.xres[(size_t)(2 * layer + 2) * BH + o] = __ldcg(p.xres + (size_t)(2 * layer + 1) * BH + o) + y;
-      } else {
-        p.logits[(size_t)b * p.V + row] = y;
+#pragma unroll
+    for (int t0 = 0; t0 < MAXT; t0 += 4) {
+      if (t0 < ntiles) {
+        if (t0 > 0) consumer_bar();  // the previous round's sums are read
+#pragma unroll
+        for (int dq = 0; dq < 4; ++dq)
+          if (t0 + dq < MAXT && t0 + dq < ntiles)
+            *reinterpret_cast<float4*>(red + warp * 512 + dq * 128 + lane * 4) =
+                make_float4(acc[t0 + dq][0], acc[t0 + dq][1], acc[t0 + dq][2], acc[t0 + dq][3]);
+        consumer_bar();
+        if (NORM && t0 == 0 && b < B) {
+          float tot = 0.f;
+          for (int w = 0; w < kConsumerWarps; ++w) tot += ctl->aml[w * kMaxBatch + b];
+          sc = 1.f / sqrtf(tot / (float)g.K + p.eps);
+        }
+        const int tile = t0 + q;
+        if (tile < ntiles && b < B) {
+          float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            v0 += red[w * 512 + q * 128 + l * 4 + i];
+            v1 += red[w * 512 + q * 128 + l * 4 + 2 + i];
+          }
+          v0 *= sc;
+          v1 *= sc;
+          if (GATED) {
+            const int row = tile * TR + lgq;  // v0 = gate, v1 = up of neuron row
+            if (row < nrows) p.act[(size_t)b * p.I + g.r0 + row] = v0 / (1.f + expf(-v0)) * v1;
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int rr = tile * TR + lgq + 8 * h;
+              if (rr < nrows) {
+                const float y = h ? v1 : v0;
+                const int row = g.r0 + rr;
+                if (op == OP_QKV) {
+                  p.qkv[(size_t)b * qkvw + row] = y;
+                } else if (op == OP_OPROJ) {
+                  const size_t o = (size_t)b * p.H + row;
+                  p.xres[(size_t)(2 * layer + 1) * BH + o] = __ldcg(p.xres + (size_t)(2 * layer) * BH + o) + y;
+                } else if (op == OP_DOWN) {
+                  const size_t o = (size_t)b * p.H + row;
+                  p.xres[(size_t)(2 * layer + 2) * BH + o] = __ldcg(p.xres + (size_t)(2 * layer + 1) * BH + o) + y;
+                } else {
+                  p.logits[(size_t)b * p.V + row] = y;
+                }
+              }
+            }
+          }
+        }
       }
     }
     return true;
@@ -1079,9 +1152,9 @@ struct Consumer {
 
   __device__ __forceinline__ bool gemv(const mk_instr& in, int op, int layer) {
     if constexpr (BATCHED) {
-      if (op == OP_GATEUP) return gemv_mma<true, true>(in, op, layer);
-      if (op == OP_QKV || op == OP_LMHEAD) return gemv_mma<true, false>(in, op, layer);
-      return gemv_mma<false, false>(in, op, layer);
+      if (op == OP_GATEUP) return gemv_tc<true, true>(in, op, layer);
+      if (op == OP_QKV || op == OP_LMHEAD) return gemv_tc<true, false>(in, op, layer);
+      return gemv_tc<false, false>(in, op, layer);
     }
     const bool norm = op == OP_QKV || op == OP_GATEUP || op == OP_LMHEAD;
     const int K = op == OP_OPROJ ? p.nq * p.hd : (op == OP_DOWN ? p.I : p.H);
@@ -1450,8 +1523,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
   using SM = Smem<BATCHED>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
-  float* red = reinterpret_cast<float*>(smem + SM::kRing + SM::kXs);
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + SM::kRing + SM::kXs + SM::kRed);
+  float* red = reinterpret_cast<float*>(smem + SM::kRing);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + SM::kRing + SM::kRed);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SM::kNst; ++s) {
@@ -1469,6 +1542,11 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
         set_status(p, MK_ERR_RANGE, b);
         bad = 1;
       }
+    }
+    // the swizzled TMA boxes of the batched GEMV need 1024-byte aligned slots
+    if (!bad && BATCHED && (smem_addr(ring) & 1023u) != 0) {
+      set_status(p, MK_ERR_UNSUPPORTED, -3);
+      bad = 1;
     }
     ctl->flag = bad;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");

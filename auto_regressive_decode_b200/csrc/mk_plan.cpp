@@ -56,10 +56,10 @@ int validate_desc(const mk_model_desc* d) {
   if (gemv_ksplit(d->hidden, 1) != 1 || gemv_ksplit(d->hidden, 2) != 1) return MK_ERR_UNSUPPORTED;
   if ((int64_t)d->max_ctx * d->head_dim > (1ll << 31)) return MK_ERR_UNSUPPORTED;
   if (d->batch > 1) {
-    // tensor-core GEMVs: k-steps of 16 and input slices of at most kBatchedSlice columns
+    // tensor-core GEMVs: the weight tensor maps view K as blocks of 64 columns
     const int ks[3] = {d->hidden, qd, d->ffn_dim};
     for (int K : ks)
-      if (K % 16 || bgemv_slices(K) == 0) return MK_ERR_UNSUPPORTED;
+      if (K % 64) return MK_ERR_UNSUPPORTED;
   }
   return MK_OK;
 }
@@ -87,9 +87,15 @@ struct Builder {
   int rows_op(int op, int layer, int N, const std::vector<int>& cuts, int wait_idx, int wait_count, int sig_idx) {
     int n = 0;
     const int n_sm = p->n_sm;
-    const int max_rows = p->d.batch > 1 ? kBatchedMaxRows : kMaxRows;
+    const int max_rows =
+        p->d.batch > 1 ? (op == OP_GATEUP ? kBatchedMaxRowsGated : kBatchedMaxRows) : kMaxRows;
+    // batch > 1: row ranges start at multiples of kBBoxRows (a TMA box
+    // never reaches into another SM's rows or across wq | wk | wv)
+    const int unit = p->d.batch > 1 ? kBBoxRows : 1;
+    const int64_t NU = (N + unit - 1) / unit;
     for (int s = 0; s < n_sm; ++s) {
-      int r0 = (int)((int64_t)N * s / n_sm), r1 = (int)((int64_t)N * (s + 1) / n_sm);
+      int r0 = (int)std::min<int64_t>(N, NU * s / n_sm * unit);
+      int r1 = (int)std::min<int64_t>(N, NU * (s + 1) / n_sm * unit);
       while (r0 < r1) {
         int e = std::min(r1, r0 + max_rows);
         int seg = 0, base = 0;

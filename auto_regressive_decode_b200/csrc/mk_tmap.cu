@@ -1,0 +1,74 @@
+// TMA tensor maps of the weight matrices, for the batch > 1 tensor-core GEMV.
+//
+// A row-major bf16 matrix W[N][K] (K a multiple of 64) is described as the
+// 3-D tensor (64, N, K/64) with strides (2 B, 2K B, 128 B): element
+// (c, r, kb) is W[r][64 kb + c].  A box of (64, kBBoxRows, kBChunk/64) then
+// brings kBBoxRows rows of one kBChunk-column chunk into shared memory as
+// [column block][row][64 columns], with the 128-byte swizzle (16-byte chunk
+// c of 128-byte line L at position c ^ (L & 7)).  Coordinates past K/64 read
+// as zeros (the tail chunk of a K that is not a multiple of kBChunk).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include "mk_device.h"
+
+namespace mk {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool encode_one(EncodeTiledFn enc, const void* w, int rows, int K, uint8_t* out) {
+  static_assert(sizeof(CUtensorMap) == 128, "tensor map size");
+  if (!w || rows <= 0 || K % 64) return false;
+  CUtensorMap m;
+  const cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(K / 64)};
+  const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+  const cuuint32_t box[3] = {64, (cuuint32_t)kBBoxRows, (cuuint32_t)(kBChunk / 64)};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  const CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  memcpy(out, &m, sizeof(m));
+  return true;
+}
+
+}  // namespace
+
+cudaError_t encode_weight_tmaps(const mk_model_desc& d, const mk_weights& w, uint8_t* out) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const int H = d.hidden, qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim, I = d.ffn_dim;
+  for (int l = 0; l < d.n_layers; ++l) {
+    const mk_layer_weights& lw = w.layers[l];
+    uint8_t* o = out + (size_t)l * kTmapsPerLayer * 128;
+    const bool ok = encode_one(enc, lw.wq, qd, H, o) && encode_one(enc, lw.wk, kvd, H, o + 128) &&
+                    encode_one(enc, lw.wv, kvd, H, o + 256) && encode_one(enc, lw.wo, H, qd, o + 384) &&
+                    encode_one(enc, lw.w_gate, I, H, o + 512) && encode_one(enc, lw.w_up, I, H, o + 640) &&
+                    encode_one(enc, lw.w_down, H, I, o + 768);
+    if (!ok) return cudaErrorInvalidValue;
+  }
+  const void* lm = d.tied_embeddings ? w.embed : w.lm_head;
+  if (!encode_one(enc, lm, d.vocab, H, out + (size_t)d.n_layers * kTmapsPerLayer * 128))
+    return cudaErrorInvalidValue;
+  return cudaSuccess;
+}
+
+}  // namespace mk

@@ -44,6 +44,7 @@ def test_dense_0_6b_first_steps():
 
 # ---- batch > 1 (tensor-core projections) -------------------------------------------------------
 
+# the batched GEMV reads K in blocks of 64 columns: tiny's ffn width 688 becomes 704
 @pytest.mark.parametrize("kw,gains", [
     ({"batch": 4, "ctx": 0, "ctx_lo": 3, "ctx_hi": 60, "steps": 3}, "random"),
     ({"batch": 8, "ctx": 0, "steps": 2}, "ones"),                                    # empty caches
@@ -51,13 +52,14 @@ def test_dense_0_6b_first_steps():
     ({"batch": 3, "ctx": 0, "ctx_lo": 250, "ctx_hi": 260, "steps": 3}, "ones"),    # chunk boundary, ragged
 ])
 def test_tiny_batched(kw, gains):
-    cfg = fx.CONFIGS["tiny"].replace(**kw)
+    cfg = fx.CONFIGS["tiny"].replace(ffn_dim=704, **kw)
     assert_parity(run_teacher_forced(cfg, steps=kw.get("steps", 3), gains=gains))
 
 
-def test_batched_multi_slice_multi_chunk():
-    # MHA, head_dim 128; the down projection (K = 4608) runs as 2 input slices of
-    # 2 column chunks each, the other projections as 1 slice / 1 chunk
+def test_batched_multi_chunk():
+    # MHA, head_dim 128; the down projection (K = 4608) streams 5 column chunks,
+    # the last one half empty (its TMA boxes read zeros past K); hidden = 640
+    # leaves 24 of each chunk's 64 k-steps idle
     cfg = fx.ModelConfig("mid-b8", n_layers=3, hidden=640, n_q_heads=5, n_kv_heads=5, head_dim=128, ffn_dim=4608,
                          vocab=2000, batch=8, ctx_lo=10, ctx_hi=300, steps=3)
     assert_parity(run_teacher_forced(cfg, gains="random"))

@@ -153,3 +153,37 @@ def test_invalid_and_unsupported_shapes():
             mk.Plan(mk.model_desc(cfg), 148)
     with pytest.raises(mk.MkError):
         mk.Plan(mk.model_desc(base), 0)
+
+
+def test_batched_shapes_need_64_column_blocks():
+    # the tensor-core GEMV views K (hidden, q width, ffn width) as blocks of 64 columns
+    base = fx.CONFIGS["tiny"].replace(batch=4)
+    with pytest.raises(mk.MkError):
+        mk.Plan(mk.model_desc(base), 148)                  # ffn 688
+    mk.Plan(mk.model_desc(base.replace(ffn_dim=704)), 148)
+    mk.Plan(mk.model_desc(fx.CONFIGS["tiny"]), 148)          # batch 1 reads rows whole: 688 is fine
+
+
+@pytest.mark.parametrize("name,kw,n_sm", [("dense-13b-b8", {}, 148), ("dense-13b-b8", {}, 132),
+                                          ("tiny", {"batch": 4, "ffn_dim": 704}, 148),
+                                          ("tiny", {"batch": 4, "ffn_dim": 704}, 5)])
+def test_batched_row_ranges_on_box_boundaries(name, kw, n_sm):
+    # a TMA box is 8 rows: every batched GEMV instruction starts on a multiple of 8
+    # and stays within one of wq | wk | wv; row caps 128 (96 for gate/up)
+    cfg, p = plan_of(name, n_sm, **kw)
+    qd, kvd = cfg.q_dim, cfg.kv_dim
+    for r in p.instrs:
+        op = p.op(r)
+        if op in (OP_QKV, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LMHEAD):
+            r0, r1 = int(r[4]), int(r[5])
+            assert r0 % 8 == 0 and r1 > r0
+            assert r1 - r0 <= (96 if op == OP_GATEUP else 128)
+            assert r1 % 8 == 0 or r1 == rows_of(cfg, op)
+    # balanced: no SM streams more than one 8-row box more than the mean per op
+    for op in (OP_QKV, OP_DOWN):
+        per = collections.Counter()
+        for s in range(n_sm):
+            for r in p.sm_list(s):
+                if p.op(r) == op and p.layer(r) == 0:
+                    per[s] += int(r[5]) - int(r[4])
+        assert max(per.values()) <= rows_of(cfg, op) / n_sm + 8
