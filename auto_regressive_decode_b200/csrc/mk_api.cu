@@ -139,7 +139,7 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const size_t o_off = cv.take(sizeof(int32_t) * offsets.size());
   const size_t o_lay = cv.take(sizeof(mk::LayerPtrs) * (size_t)L);
   const size_t o_rope = cv.take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
-  const size_t n_tmaps = B > 1 ? (size_t)mk::kTmapsPerLayer * L + 1 : 0;
+  const size_t n_tmaps = B > 1 ? (size_t)mk::kTmapsPerLayer * L + 3 : 0;
   const size_t o_tmap = n_tmaps ? cv.take(128 * n_tmaps) : 0;
   const char* trace_env = getenv("MK_TRACE");
   const bool tracing = trace_env && atoi(trace_env) > 0;
@@ -179,7 +179,7 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
 
   std::vector<uint8_t> tmaps(128 * n_tmaps);
   if (n_tmaps) {
-    const cudaError_t te = mk::encode_weight_tmaps(d, *w, tmaps.data());
+    const cudaError_t te = mk::encode_tmaps(d, *w, *kv, tmaps.data());
     if (te != cudaSuccess) {
       cudaFree(h->region);
       delete h;
@@ -237,8 +237,6 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   p.offsets = (const int32_t*)(base + o_off);
   p.timeout_ns = d.wait_timeout_ns ? d.wait_timeout_ns : kDefaultTimeoutNs;
   p.trace = tracing ? (uint64_t*)(base + o_trace) : nullptr;
-  const char* l2_env = getenv("MK_L2_AHEAD_KB");  // diagnostic knob: L2 prefetch window per SM
-  p.l2_ahead = l2_env ? (uint32_t)atoi(l2_env) * 1024u : mk::kDefaultL2AheadBytes;
   const char* piece_env = getenv("MK_COPY_PIECE_KB");  // diagnostic knob: bytes per bulk copy
   p.copy_piece = piece_env && atoi(piece_env) > 0 ? (uint32_t)atoi(piece_env) * 1024u : mk::kDefaultCopyPiece;
   *out = h;

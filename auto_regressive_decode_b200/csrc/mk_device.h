@@ -27,7 +27,8 @@ struct Params {
   uint16_t* vc;
   const float2* rope;       // [T][hd/2] (cos, sin)
   // batch > 1: TMA tensor maps (CUtensorMap, 128 bytes each) of every weight
-  // matrix: [layer][wq wk wv wo w_gate w_up w_down], then the LM head
+  // matrix: [layer][wq wk wv wo w_gate w_up w_down], then the LM head, the K
+  // cache and the V cache
   const uint8_t* tmaps;
   // library scratch (device)
   float* xres;              // [2L+1][B][H]
@@ -49,14 +50,14 @@ struct Params {
   uint32_t epoch;
   uint64_t timeout_ns;
   uint64_t* trace;          // [n_instr][kTraceStamps] timestamps, or nullptr
-  uint32_t l2_ahead;        // bytes the producer prefetches into L2 beyond its ring (0 = off)
   uint32_t copy_piece;      // bytes per bulk copy (a multiple of 16); a stage is split into pieces
 };
 
-// Encode the 3-D tensor maps of the batched GEMV (one per weight matrix) into
-// host memory `out` (kTmapsPerLayer * L + 1 maps of 128 bytes).  Returns
-// cudaErrorInvalidValue when the driver rejects a map (alignment, sizes).
-cudaError_t encode_weight_tmaps(const mk_model_desc& d, const mk_weights& w, uint8_t* out);
+// Encode the 3-D tensor maps of the batch > 1 kernel (one per weight matrix,
+// then the K and V caches) into host memory `out` (kTmapsPerLayer * L + 3
+// maps of 128 bytes).  Returns cudaErrorInvalidValue when the driver rejects a
+// map (alignment, sizes).
+cudaError_t encode_tmaps(const mk_model_desc& d, const mk_weights& w, const mk_kv& kv, uint8_t* out);
 
 // Dynamic shared memory of one CTA.
 size_t kernel_smem_bytes(bool batched);

@@ -45,7 +45,6 @@ constexpr int kMaxBatch = 8;
 constexpr int kMaxGroup = 8;                           // query heads per KV head
 constexpr int kMaxHeadDim = 128;
 constexpr int kTraceStamps = 8;                        // per-instruction trace words
-constexpr uint32_t kDefaultL2AheadBytes = 0;  // L2 prefetch window beyond the ring (measured: no gain)
 constexpr uint32_t kDefaultCopyPiece = 32 * 1024;  // bytes per bulk copy
 
 // ---- dependency counters -----------------------------------------------------
@@ -134,5 +133,68 @@ MK_HD int attn_heads_per_instr(int group) { return group > 4 ? 4 : group; }
 
 // Positions of K (or V) that fit one ring slot.
 MK_HD int attn_stage_positions(int head_dim) { return kStageBytes / (head_dim * 2); }
+
+// ---- attention schedule (computed on the device from each step's seq_lens) --------
+// A row is (sequence b, KV head, head group); its work is the positions
+// 0..S_b (S_b cached ones and the new token) in units of `unit` positions,
+// u_b = S_b / unit + 1 units.  Rows are ordered (b, KV head, head group) and
+// the U units of all rows are dealt to n = min(n_slots, U) slots as contiguous
+// runs [U j / n, U (j + 1) / n): every slot streams the same number of units
+// (to within one), whatever the lengths.  A slot's run is cut into pieces at row
+// boundaries; each piece writes a partial (o, m, l) and the last piece of a
+// row to finish merges the row's pieces in slot order.
+struct AttnSched {
+  int unit, n_slots, rows_per_seq, B;
+  int64_t U;
+  int u[kMaxBatch];          // units per row of sequence b
+  int64_t base[kMaxBatch + 1];  // first global unit of sequence b
+};
+
+struct AttnPiece {
+  int b, row;          // sequence, row within the sequence (KV head * head groups + head group)
+  int ua, ub;          // units [ua, ub) of the row
+  int slot_in_row;     // index of this piece among the row's pieces
+  int n_pieces;        // pieces of the row
+};
+
+MK_HD void attn_sched_init(AttnSched& s, const int32_t* seq_lens, int B, int rows_per_seq, int unit, int n_slots) {
+  s.unit = unit;
+  s.n_slots = n_slots;
+  s.rows_per_seq = rows_per_seq;
+  s.B = B;
+  s.base[0] = 0;
+  for (int b = 0; b < kMaxBatch; ++b) {
+    s.u[b] = b < B ? seq_lens[b] / unit + 1 : 0;
+    s.base[b + 1] = s.base[b] + (int64_t)rows_per_seq * s.u[b];
+  }
+  s.U = s.base[B];
+  // fewer units than slots: one unit each for the first U slots, none after,
+  // so that every slot in use holds at least one unit
+  if (s.U < s.n_slots) s.n_slots = (int)s.U;
+}
+
+// First global unit of slot j (U for j >= the slots in use).
+MK_HD int64_t attn_slot_begin(const AttnSched& s, int j) { return j >= s.n_slots ? s.U : s.U * j / s.n_slots; }
+
+// The slot holding global unit g (0 <= g < U).
+MK_HD int attn_slot_of(const AttnSched& s, int64_t g) { return (int)(((g + 1) * s.n_slots - 1) / s.U); }
+
+// The piece of slot j that starts at global unit g (g < end of slot j).
+MK_HD AttnPiece attn_piece_at(const AttnSched& s, int64_t g, int j) {
+  AttnPiece pc;
+  int b = 0;
+  while (b + 1 < s.B && s.base[b + 1] <= g) ++b;
+  const int64_t off = g - s.base[b];
+  pc.b = b;
+  pc.row = (int)(off / s.u[b]);
+  pc.ua = (int)(off % s.u[b]);
+  const int64_t left = attn_slot_begin(s, j + 1) - g;
+  pc.ub = (int)((int64_t)(s.u[b] - pc.ua) < left ? s.u[b] : pc.ua + left);
+  const int64_t first = s.base[b] + (int64_t)pc.row * s.u[b];
+  const int s0 = attn_slot_of(s, first);
+  pc.slot_in_row = j - s0;
+  pc.n_pieces = attn_slot_of(s, first + s.u[b] - 1) - s0 + 1;
+  return pc;
+}
 
 }  // namespace mk

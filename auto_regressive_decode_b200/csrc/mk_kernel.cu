@@ -40,7 +40,6 @@ struct Ctl {
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
   int dead;       // this CTA gives up: every wait returns at once
-  int waiting;    // consumers are blocked on a dependency counter (producer may prefetch)
   int last;       // attention: this CTA merges (broadcast)
   int flag;       // generic broadcast
   float sred[kConsumerWarps * 2];
@@ -48,6 +47,7 @@ struct Ctl {
   float aml[kConsumerWarps * kMaxGroup * 2];  // attention: per-warp (m, l) of every head
   alignas(16) uint16_t knew[kMaxHeadDim];     // the new token's K/V rows (bf16, as appended)
   alignas(16) uint16_t vnew[kMaxHeadDim];
+  AttnSched psched;  // the producer's attention schedule of its current slot
 };
 
 // Shared memory: the ring of weight / KV stages (slots 1024-byte aligned, as
@@ -296,6 +296,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Four 8x8 b16 matrices from shared memory, transposed on the way: lane
+// (g, c) receives elements (2c, g) and (2c + 1, g) of every stored matrix.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t a[4], uint32_t saddr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(saddr));
+}
+
+// Transpose of an 8x8 b16 matrix held one element pair per lane (lane (g, c)
+// holds row g, columns 2c and 2c + 1) into the same layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // Four 8x8 b16 matrices from shared memory; lane l supplies the address of
 // row (l & 7) of matrix (l >> 3) and receives element pair (l >> 2, 2 * (l & 3))
 // of every matrix: exactly an m16n8k16 A fragment when the matrices are
@@ -407,36 +423,44 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
   return g;
 }
 
+// One attention piece: units [ua, ub) of row (b, kvh, hg), i.e. positions
+// [p0, min(ub * unit, S + 1)); the cached ones [p0, p0 + n_cached) stream
+// through the ring, the new token (position S) comes from this step's qkv.
 struct Attn {
-  int b, kvh, c, hg, S, p0, n_cached, nsub, P;
+  int b, kvh, hg, S, p0, n_cached, nsub, P;
+  int c, npieces;  // index of the piece within its row, pieces of the row
   bool active, owns_new;
   size_t cache_base;  // element offset of (layer, b, kvh, position p0)
 };
 
-__device__ __forceinline__ Attn attn_geo(const Params& p, const mk_instr& in, int layer, int head_dim) {
+__device__ __forceinline__ Attn attn_geo(const Params& p, const AttnPiece& pc, int layer, int head_dim) {
   Attn a;
-  a.b = in.a;
-  a.kvh = in.b;
-  a.c = in.c;
-  a.hg = in.d;
+  const int group = p.nq / p.nkv, nhg = group / attn_heads_per_instr(group);
+  a.b = pc.b;
+  a.kvh = pc.row / nhg;
+  a.hg = pc.row % nhg;
   a.S = p.seq_lens[a.b];
-  a.p0 = a.c * p.chunk;
-  const int p1 = min(a.p0 + p.chunk, p.T);
-  a.active = a.p0 <= a.S;
-  a.owns_new = a.active && a.S < p1;
+  a.p0 = pc.ua * p.chunk;
+  const int p1 = pc.ub * p.chunk;
+  a.active = true;
+  a.owns_new = a.S < p1;
   a.n_cached = max(0, min(p1, a.S) - a.p0);
   a.P = attn_stage_positions(head_dim);
   a.nsub = (a.n_cached + a.P - 1) / a.P;
+  a.c = pc.slot_in_row;
+  a.npieces = pc.n_pieces;
   a.cache_base = ((((size_t)layer * p.B + a.b) * p.nkv + a.kvh) * p.T + a.p0) * head_dim;
   return a;
+}
+
+__device__ __forceinline__ void attn_sched(const Params& p, const mk_instr& in, AttnSched& sc) {
+  const int group = p.nq / p.nkv;
+  attn_sched_init(sc, p.seq_lens, p.B, p.nkv * (group / attn_heads_per_instr(group)), p.chunk, in.b);
 }
 
 // ---------------------------------------------------------------------------
 // Producer warp (lane 0 issues everything)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 
 // Walks the stages of an SM's instruction list in order.  A GEMV stage is R
 // rows (one column slice) of one segment, plus the same rows of the up matrix
@@ -450,9 +474,13 @@ struct Cursor {
   Gemv g;
   int kc, sg, rr;  // GEMV: slice (batched: chunk), segment (batched: tile), first row within the segment
   Attn a;
-  int sub, kv;     // attention: sub-chunk, K (0) or V (1)
+  int sub, kv;     // attention: stage within the piece, K (0) or V (1)
+  AttnSched* sc;   // attention: this step's schedule (shared memory), slot aslot's units [ag, ag1)
+  int64_t ag, ag1;
+  int aslot, pieceu;  // slot, units of the current piece
 
-  __device__ Cursor(const Params& prm, const mk_instr* l, int nn) : pp(&prm), list(l), n(nn), i(0) {}
+  __device__ Cursor(const Params& prm, const mk_instr* l, int nn, AttnSched* sched)
+      : pp(&prm), list(l), n(nn), i(0), sc(sched) {}
 
   // Position on the first stage of instruction j or of the next one that has stages.
   __device__ __forceinline__ void seek(int j) {
@@ -461,9 +489,12 @@ struct Cursor {
       op = op_of(in.op_layer);
       layer = layer_of(in.op_layer);
       if (op == OP_ATTN) {
-        a = attn_geo(*pp, in, layer, pp->hd);
+        attn_sched(*pp, in, *sc);
+        aslot = in.a;
+        ag = attn_slot_begin(*sc, aslot);
+        ag1 = attn_slot_begin(*sc, aslot + 1);
         sub = kv = 0;
-        if (a.nsub > 0) return;
+        if (next_piece()) return;
       } else if (op >= OP_QKV && op <= OP_LMHEAD) {
         g = gemv_geo(*pp, in, op, layer);
         kc = sg = rr = 0;
@@ -472,10 +503,26 @@ struct Cursor {
     }
   }
 
+  // From unit ag on: the first piece of the slot that has cached positions.
+  __device__ __forceinline__ bool next_piece() {
+    while (ag < ag1) {
+      const AttnPiece pc = attn_piece_at(*sc, ag, aslot);
+      a = attn_geo(*pp, pc, layer, pp->hd);
+      pieceu = pc.ub - pc.ua;
+      if (a.nsub > 0) return true;
+      ag += pieceu;
+    }
+    return false;
+  }
+
   __device__ __forceinline__ void advance() {
     if (op == OP_ATTN) {
       kv ^= 1;
-      if (!kv && ++sub >= a.nsub) seek(i + 1);
+      if (!kv && ++sub >= a.nsub) {
+        sub = 0;
+        ag += pieceu;
+        if (!next_piece()) seek(i + 1);
+      }
       return;
     }
     if (pp->B > 1) {  // batched GEMV: chunk kc, tile sg within it
@@ -557,8 +604,18 @@ struct Cursor {
     return (uint32_t)nh * kBBoxBytes;
   }
 
+  // Batched attention stage: one box of P positions of the K (kv = 0) or V
+  // cache, rows past the chunk's cached positions included (the consumers
+  // mask them).
+  __device__ __forceinline__ void attn_box(const uint8_t** map, int* row) const {
+    const Params& p = *pp;
+    *map = p.tmaps + ((size_t)p.L * kTmapsPerLayer + 1 + kv) * 128;
+    *row = (int)(a.cache_base / (size_t)p.hd) + sub * a.P;
+  }
+
   __device__ __forceinline__ uint32_t stage_bytes() const {
-    if (op == OP_ATTN) return (uint32_t)min(a.P, a.n_cached - sub * a.P) * pp->hd * 2u;
+    if (op == OP_ATTN)
+      return pp->B > 1 ? (uint32_t)kStageBytes : (uint32_t)min(a.P, a.n_cached - sub * a.P) * pp->hd * 2u;
     if (pp->B > 1) return (g.wup || g.r1 - g.r0 - sg * 16 > 8) ? 2u * kBBoxBytes : (uint32_t)kBBoxBytes;
     const uint32_t b = (uint32_t)min(g.tile.rows_per_stage, g.seg_rows(sg) - rr) * (uint32_t)g.Kc * 2u;
     return g.wup ? 2 * b : b;
@@ -573,24 +630,8 @@ struct Producer {
   uint8_t* ring;
   uint64_t pol;
   uint32_t k = 0;  // stages issued
-  Cursor pf;       // L2 prefetch cursor, pf_ahead bytes past the issue cursor
-  uint32_t pf_ahead = 0;
 
-  __device__ Producer(const Params& pp, Ctl* c, uint8_t* r, const mk_instr* l, int nn)
-      : p(pp), ctl(c), ring(r), pf(pp, l, nn) {
-    pol = evict_first_policy();
-  }
-
-  // While blocked on the ring: prefetch the next stages into L2, up to
-  // Params::l2_ahead bytes (batch-1 kernel only).
-  __device__ __forceinline__ void prefetch_ahead() {
-    if constexpr (!BATCHED) {
-      while (pf_ahead < p.l2_ahead && pf.i < pf.n) {
-        pf_ahead += pf.copies([&](const uint16_t* src, uint32_t bytes, uint32_t) { prefetch_l2(src, bytes); });
-        pf.advance();
-      }
-    }
-  }
+  __device__ Producer(const Params& pp, Ctl* c, uint8_t* r) : p(pp), ctl(c), ring(r) { pol = evict_first_policy(); }
 
   // Claim the next slot (waiting until the consumers released it).
   __device__ __forceinline__ bool claim(uint8_t** dst, unsigned long long** bar) {
@@ -601,9 +642,6 @@ struct Producer {
         const uint64_t t0 = globaltimer();
         uint32_t spins = 0;
         while (!mbar_try_wait(&ctl->empty[slot], parity)) {
-          // only while the consumers wait on another SM: steady streaming is
-          // left alone (prefetches share the copy engine with the ring)
-          if (*(volatile int*)&ctl->waiting) prefetch_ahead();
           if (*(volatile int*)&ctl->dead) return false;
           if ((++spins & 63) == 0) {
             if (ld_relaxed_i32(p.status) != 0) return false;
@@ -635,11 +673,10 @@ struct Producer {
 // One thread (lane 0 of the producer warp) issues every copy.
 template <bool BATCHED>
 __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
-  Producer<BATCHED> pr(p, ctl, ring, list, n);
+  Producer<BATCHED> pr(p, ctl, ring);
   uint64_t* trace = p.trace ? p.trace + (size_t)p.offsets[blockIdx.x] * kTraceStamps : nullptr;
-  Cursor cur(p, list, n);
+  Cursor cur(p, list, n, &ctl->psched);
   cur.seek(0);
-  pr.pf = cur;
   bool ok = true;
   int last = -1;
   while (cur.i < n) {
@@ -654,7 +691,12 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
     if (!(ok = pr.claim(&dst, &bar))) break;
     const uint32_t bytes = cur.stage_bytes();
     mbar_arrive_expect_tx(bar, bytes);
-    if (BATCHED && cur.op != OP_ATTN) {
+    if (BATCHED && cur.op == OP_ATTN) {
+      const uint8_t* map;
+      int row;
+      cur.attn_box(&map, &row);
+      tma_box3(dst, map, 0, row, 0, bar, pr.pol);
+    } else if (BATCHED) {
       cur.boxes([&](const uint8_t* map, int row, int kb, uint32_t off) {
         tma_box3(dst + off, map, 0, row, kb, bar, pr.pol);
       });
@@ -663,12 +705,6 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
     }
     ++pr.k;
     cur.advance();
-    if (pr.pf_ahead > bytes) {
-      pr.pf_ahead -= bytes;
-    } else {
-      pr.pf = cur;
-      pr.pf_ahead = 0;
-    }
   }
   if (trace && last >= 0) trace[last * kTraceStamps + 7] = globaltimer();
   if (!ok) {
@@ -731,7 +767,6 @@ struct Consumer {
       const uint32_t target = p.epoch * (uint32_t)count;
       const uint32_t* c = p.counters + idx;
       if ((int32_t)(ld_acquire(c) - target) < 0) {
-        *(volatile int*)&ctl->waiting = 1;
         const uint64_t t0 = globaltimer();
         while (true) {
           if ((int32_t)(ld_acquire(c) - target) >= 0) break;
@@ -745,7 +780,6 @@ struct Consumer {
             break;
           }
         }
-        *(volatile int*)&ctl->waiting = 0;
       }
     }
     if (t == 0 && *(volatile int*)&ctl->dead) fail = true;
@@ -1167,17 +1201,223 @@ struct Consumer {
   }
 
   // ---- attention ---------------------------------------------------------------
-  // One (sequence, KV head, chunk of positions): q of the G query heads of
-  // the group against the chunk's cached K/V rows (streamed through the ring)
-  // and, in the chunk that holds it, the new token's own K/V row.  The
-  // result is an unnormalised partial (o, m, l) in log2 units; the last
-  // chunk of the (sequence, KV head) to finish merges all partials.
+  // Batch > 1: the cached positions of one chunk on tensor cores.  A stage is
+  // a TMA box of P positions, [64-column block][position][64] with the 128-byte
+  // swizzle.  Warp w owns key tiles of 16 positions of every stage:
+  //   S^T[key][head] = K[key][:] . q[head][:]   mma: A = K tile (ldmatrix),
+  //                                              B = q (bf16, heads >= G zero)
+  //   O^T[dim][head] += V[key][dim]^T P^T        mma: A = V tile (ldmatrix.trans),
+  //                                              B = P (movmatrix transposes S's layout)
+  // with its own online softmax (log2 units, q pre-scaled by log2(e)/sqrt(hd)).
+  // The warps' (m, l, o) are merged through shared memory into the chunk's
+  // partial, the same partial the CUDA-core path writes.
+  template <int HD, int G>
+  __device__ __forceinline__ void attn_tc(const Attn& a, int q0) {
+    constexpr int P = kStageBytes / (HD * 2);
+    constexpr int MT = P / 16 / kConsumerWarps;  // key tiles per warp per stage
+    constexpr int KS = HD / 16;                  // k-steps of the score mma
+    constexpr int DT = HD / 16;                  // dimension tiles of the P.V mma
+    constexpr uint32_t CBB = (uint32_t)P * 128u;  // bytes of one 64-column block of a stage
+    const int gq = lane >> 2, cq = lane & 3;
+    uint32_t qf[KS][2];
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      if (gq < G) {
+        const float* qh = ctl->qs + gq * HD + ks * 16 + 2 * cq;
+        qf[ks][0] = pack_bf16x2(qh[0], qh[1]);
+        qf[ks][1] = pack_bf16x2(qh[8], qh[9]);
+      } else {
+        qf[ks][0] = qf[ks][1] = 0u;
+      }
+    }
+    float o[DT][4];
+#pragma unroll
+    for (int dt = 0; dt < DT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+    float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;  // heads 2cq and 2cq + 1
+    const uint32_t r7 = (uint32_t)(lane & 7);
+    // ldmatrix rows: K tile row (lane & 15); V tile row (lane & 7) + 8 (lane >> 4)
+    const uint32_t krow = (uint32_t)(lane & 15) * 128u;
+    const uint32_t vrow = (uint32_t)((lane & 7) + ((lane >> 4) << 3)) * 128u;
+    for (int s = 0; s < a.nsub; ++s) {
+      const int np = min(P, a.n_cached - s * P);
+      const uint32_t Ks = smem_addr(wait_stage(k));
+      uint8_t* Vp = const_cast<uint8_t*>(wait_stage(k + 1));
+      const uint32_t Vs = smem_addr(Vp);
+      if (tr && s == 0) tr[5] = globaltimer();
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int key0 = (warp * MT + mt) * 16;
+        if (key0 < np) {
+          float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const uint32_t ch = ((uint32_t)(ks & 3) << 1) | (uint32_t)(lane >> 4);
+            uint32_t af[4];
+            ldmatrix_x4(af, Ks + (uint32_t)(ks >> 2) * CBB + (uint32_t)key0 * 128u + krow + ((ch ^ r7) << 4));
+            mma16816(sc, af[0], af[1], af[2], af[3], qf[ks][0], qf[ks][1]);
+          }
+          // this lane: keys key0 + gq (sc[0..1]) and key0 + gq + 8 (sc[2..3]), heads 2cq, 2cq + 1
+          const bool v0 = key0 + gq < np, v1 = key0 + gq + 8 < np;
+          const float s00 = v0 ? sc[0] : -1e30f, s01 = v0 ? sc[1] : -1e30f;
+          const float s10 = v1 ? sc[2] : -1e30f, s11 = v1 ? sc[3] : -1e30f;
+          float x0 = fmaxf(s00, s10), x1 = fmaxf(s01, s11);
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
+            x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
+          }
+          const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+          const float c0 = exp2f(m0 - n0), c1 = exp2f(m1 - n1);
+          const float p00 = v0 ? exp2f(s00 - n0) : 0.f, p01 = v0 ? exp2f(s01 - n1) : 0.f;
+          const float p10 = v1 ? exp2f(s10 - n0) : 0.f, p11 = v1 ? exp2f(s11 - n1) : 0.f;
+          float y0 = p00 + p10, y1 = p01 + p11;
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            y0 += __shfl_xor_sync(0xffffffffu, y0, off);
+            y1 += __shfl_xor_sync(0xffffffffu, y1, off);
+          }
+          l0 = l0 * c0 + y0;
+          l1 = l1 * c1 + y1;
+          m0 = n0;
+          m1 = n1;
+#pragma unroll
+          for (int dt = 0; dt < DT; ++dt) {
+            o[dt][0] *= c0;
+            o[dt][1] *= c1;
+            o[dt][2] *= c0;
+            o[dt][3] *= c1;
+          }
+          const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p00, p01));  // P[keys 2cq, 2cq+1][head gq]
+          const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p10, p11));  // P[keys 8+2cq, 9+2cq][head gq]
+          if (key0 + 16 > np) {
+            // V rows past the cached positions may hold anything (0 * NaN is
+            // NaN): zero this tile's absent rows, in every 64-column block
+            for (int idx = lane; idx < 16 * (HD / 8); idx += 32) {
+              const int r = idx / (HD / 8), c16 = idx % (HD / 8);
+              if (key0 + r >= np)
+                *reinterpret_cast<uint4*>(Vp + (c16 >> 3) * CBB + (uint32_t)(key0 + r) * 128u + (c16 & 7) * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            // order the generic writes before the ring's next TMA write of this slot
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+          }
+#pragma unroll
+          for (int dt = 0; dt < DT; ++dt) {
+            const uint32_t ch = ((uint32_t)(dt & 3) << 1) | (uint32_t)((lane >> 3) & 1);
+            uint32_t af[4];
+            ldmatrix_x4_trans(af, Vs + (uint32_t)(dt >> 2) * CBB + (uint32_t)key0 * 128u + vrow + ((ch ^ r7) << 4));
+            mma16816(o[dt], af[0], af[1], af[2], af[3], pb0, pb1);
+          }
+        }
+      }
+      release();  // K slot
+      release();  // V slot
+    }
+    if (tr) tr[6] = globaltimer();
+    if (a.owns_new && warp == 0) {
+      // the new token: score of head (lane & 7), four lanes per head over
+      // interleaved dimensions, then folded into warp 0's running state
+      const int h = lane & 7, part = lane >> 3;
+      float d = 0.f;
+      if (h < G) {
+#pragma unroll 8
+        for (int e = 0; e < HD / 4; ++e)
+          d = fmaf(ctl->qs[h * HD + e * 4 + part], bf16_bits_to_f32(ctl->knew[e * 4 + part]), d);
+      }
+      d += __shfl_xor_sync(0xffffffffu, d, 8);
+      d += __shfl_xor_sync(0xffffffffu, d, 16);
+      const float sn0 = __shfl_sync(0xffffffffu, d, 2 * cq), sn1 = __shfl_sync(0xffffffffu, d, 2 * cq + 1);
+      const float n0 = fmaxf(m0, sn0), n1 = fmaxf(m1, sn1);
+      const float c0 = exp2f(m0 - n0), c1 = exp2f(m1 - n1);
+      const float e0 = exp2f(sn0 - n0), e1 = exp2f(sn1 - n1);
+      l0 = l0 * c0 + e0;
+      l1 = l1 * c1 + e1;
+      m0 = n0;
+      m1 = n1;
+#pragma unroll
+      for (int dt = 0; dt < DT; ++dt) {
+        const float va = bf16_bits_to_f32(ctl->vnew[dt * 16 + gq]), vb = bf16_bits_to_f32(ctl->vnew[dt * 16 + gq + 8]);
+        o[dt][0] = o[dt][0] * c0 + e0 * va;
+        o[dt][1] = o[dt][1] * c1 + e1 * va;
+        o[dt][2] = o[dt][2] * c0 + e0 * vb;
+        o[dt][3] = o[dt][3] * c1 + e1 * vb;
+      }
+    }
+    // -- merge the warps through shared memory, HR heads per round
+    constexpr int HR = kRedFloats / (kConsumerWarps * HD) < G ? kRedFloats / (kConsumerWarps * HD) : G;
+    const size_t pbase = ((size_t)a.b * p.nq + q0) * p.n_chunks + a.c;
+    if (gq == 0) {
+      ctl->aml[(warp * kMaxGroup + 2 * cq) * 2] = m0;
+      ctl->aml[(warp * kMaxGroup + 2 * cq) * 2 + 1] = l0;
+      ctl->aml[(warp * kMaxGroup + 2 * cq + 1) * 2] = m1;
+      ctl->aml[(warp * kMaxGroup + 2 * cq + 1) * 2 + 1] = l1;
+    }
+#pragma unroll
+    for (int h0 = 0; h0 < G; h0 += HR) {
+#pragma unroll
+      for (int dt = 0; dt < DT; ++dt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int hh = 2 * cq + (e & 1) - h0, dim = dt * 16 + gq + 8 * (e >> 1);
+          if (hh >= 0 && hh < HR) red[(warp * HR + hh) * HD + dim] = o[dt][e];
+        }
+      }
+      consumer_bar();
+      for (int id = t; id < HR * HD; id += kConsumerThreads) {
+        const int hh = id / HD, d = id % HD, h = h0 + hh;
+        float M = -1e30f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ctl->aml[(w * kMaxGroup + h) * 2]);
+        float den = 0.f, num = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float c = exp2f(ctl->aml[(w * kMaxGroup + h) * 2] - M);
+          den = fmaf(c, ctl->aml[(w * kMaxGroup + h) * 2 + 1], den);
+          num = fmaf(c, red[(w * HR + hh) * HD + d], num);
+        }
+        if (a.npieces == 1) {  // the whole row: the output itself
+          p.attn[(size_t)a.b * p.nq * HD + (size_t)(q0 + h) * HD + d] = num / den;
+        } else {
+          const size_t pi = pbase + (size_t)h * p.n_chunks;
+          p.part_o[pi * HD + d] = num;
+          if (d == 0) {
+            p.part_ml[pi * 2] = M;
+            p.part_ml[pi * 2 + 1] = den;
+          }
+        }
+      }
+      consumer_bar();
+    }
+  }
+
+  // One attention slot: this step's schedule gives the slot a run of units
+  // (equal for every slot), cut into pieces at row boundaries.
   template <int HD, int G>
   __device__ __forceinline__ bool attn_run(const mk_instr& in, int layer, int sig_idx) {
+    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
+    if (tr) tr[1] = globaltimer();
+    AttnSched sc;
+    attn_sched(p, in, sc);
+    const int j = in.a;
+    for (int64_t g = attn_slot_begin(sc, j), g1 = attn_slot_begin(sc, j + 1); g < g1;) {
+      const AttnPiece pc = attn_piece_at(sc, g, j);
+      g += pc.ub - pc.ua;
+      attn_piece<HD, G>(attn_geo(p, pc, layer, HD), layer, sig_idx);
+    }
+    return true;
+  }
+
+  // One piece of (sequence, KV head, head group): q of the G query heads of
+  // the group against the piece's cached K/V rows (streamed through the ring)
+  // and, in the piece that holds it, the new token's own K/V row.  The result
+  // is an unnormalised partial (o, m, l) in log2 units; the last piece of the
+  // row to finish merges all partials.
+  template <int HD, int G>
+  __device__ __forceinline__ void attn_piece(const Attn& a, int layer, int sig_idx) {
     constexpr int LPP = HD / 8;    // lanes per position (16-byte vectors)
     constexpr int PPW = 32 / LPP;  // positions per warp pass
     constexpr int NP = HD / 64;    // rotation pairs per lane
-    const Attn a = attn_geo(p, in, layer, HD);
     const int qd = p.nq * HD, kvd = p.nkv * HD;
     const float* qkv = p.qkv + (size_t)a.b * (qd + 2 * kvd);
     // G = query heads of this instruction: head group hg of KV head kvh
@@ -1185,16 +1425,12 @@ struct Consumer {
     const int q0 = a.kvh * group + a.hg * G;  // first query head
     const float qscale = 1.4426950408889634f * rsqrtf((float)HD);  // log2(e) / sqrt(hd)
     const int pl = lane / LPP, vi = lane % LPP;
-    // RoPE table entries do not depend on this step's activations: fetch
-    // them before the dependency wait.
     float2 csr[NP];
     if (a.active) {
       const float2* cs = p.rope + (size_t)p.positions[a.b] * (HD / 2);
 #pragma unroll
       for (int j = 0; j < NP; ++j) csr[j] = __ldg(cs + lane + 32 * j);
     }
-    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
-    if (tr) tr[1] = globaltimer();
     if (a.active) {
       // -- prologue: q heads (qk-norm, RoPE, scale) and the new K/V row
       const int tasks = G + (a.owns_new ? 2 : 0);
@@ -1254,178 +1490,194 @@ struct Consumer {
       }
       consumer_bar();
       if (tr) tr[4] = globaltimer();
-      // Each group of LPP lanes owns 8 dimensions per lane and walks blocks
-      // of TB consecutive positions.  One transposed reduction leaves every
-      // (position, head) score of the block on its own lane (R = TB * G
-      // values), so each exponential is computed once; p and the rescale
-      // factors are then broadcast for the P.V update.
-      constexpr int TB = LPP / G < 4 ? LPP / G : 4;
-      constexpr int R = TB * G;
-      constexpr int SH = ilog2c(LPP) - ilog2c(R);  // lane -> value index shift
-      const int gbase = lane & ~(LPP - 1);
-      const int my_t = (vi >> SH) / G;  // this lane's position in a block (its head is (vi >> SH) % G)
-      float q[G][8], o[G][8];
-      float m_l = -1e30f, l_l = 0.f;  // running max / sum of this lane's head
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          q[h][e] = ctl->qs[h * HD + vi * 8 + e];
-          o[h][e] = 0.f;
-        }
-      }
-      // one block of TB positions starting at row t0 of Kb/Vb (rows >= np are absent)
-      auto block = [&](const uint16_t* Kb, const uint16_t* Vb, int t0, int np) {
-        float acc[R];
-#pragma unroll
-        for (int tt = 0; tt < TB; ++tt) {
-          float kf[8];
-          if (t0 + tt < np) {
-            unpack8(*reinterpret_cast<const uint4*>(Kb + (size_t)(t0 + tt) * HD + vi * 8), kf);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) kf[e] = 0.f;
-          }
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float d = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) d = fmaf(q[h][e], kf[e], d);
-            acc[tt * G + h] = d;
-          }
-        }
-        // every lane takes part in the reduction (full-mask shuffles), then
-        // lanes whose position is absent drop their score
-        const float red_sc = group_reduce_multi<R, LPP>(acc, lane);
-        const bool valid = t0 + my_t < np;
-        const float sc = valid ? red_sc : -1e30f;
-        float bm = sc;
-#pragma unroll
-        for (int off = G << SH; off < LPP; off <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-        const float mn = fmaxf(m_l, bm);
-        const float corr = exp2f(m_l - mn);
-        const float pv = valid ? exp2f(sc - mn) : 0.f;
-        float ps = pv;
-#pragma unroll
-        for (int off = G << SH; off < LPP; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-        l_l = l_l * corr + ps;
-        m_l = mn;
+      if constexpr (!BATCHED) {
+        // Each group of LPP lanes owns 8 dimensions per lane and walks blocks
+        // of TB consecutive positions.  One transposed reduction leaves every
+        // (position, head) score of the block on its own lane (R = TB * G
+        // values), so each exponential is computed once; p and the rescale
+        // factors are then broadcast for the P.V update.
+        constexpr int TB = LPP / G < 4 ? LPP / G : 4;
+        constexpr int R = TB * G;
+        constexpr int SH = ilog2c(LPP) - ilog2c(R);  // lane -> value index shift
+        const int gbase = lane & ~(LPP - 1);
+        const int my_t = (vi >> SH) / G;  // this lane's position in a block (its head is (vi >> SH) % G)
+        float q[G][8], o[G][8];
+        float m_l = -1e30f, l_l = 0.f;  // running max / sum of this lane's head
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float c = __shfl_sync(0xffffffffu, corr, gbase + ((h) << SH));
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o[h][e] *= c;
-        }
-#pragma unroll
-        for (int tt = 0; tt < TB; ++tt) {
-          float vf[8];
-          if (t0 + tt < np) {
-            unpack8(*reinterpret_cast<const uint4*>(Vb + (size_t)(t0 + tt) * HD + vi * 8), vf);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) vf[e] = 0.f;
-          }
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pr = __shfl_sync(0xffffffffu, pv, gbase + ((tt * G + h) << SH));
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e]);
-          }
-        }
-      };
-      // -- cached positions, streamed K stage then V stage
-      for (int s = 0; s < a.nsub; ++s) {
-        const int np = min(a.P, a.n_cached - s * a.P);
-        const uint16_t* Ks = reinterpret_cast<const uint16_t*>(wait_stage(k));
-        const uint16_t* Vs = reinterpret_cast<const uint16_t*>(wait_stage(k + 1));
-        if (tr && s == 0) tr[5] = globaltimer();
-        for (int tb = warp * PPW * TB; tb < np; tb += kConsumerWarps * PPW * TB) block(Ks, Vs, tb + pl * TB, np);
-        release();  // K slot
-        release();  // V slot
-      }
-      if (tr) tr[6] = globaltimer();
-      // -- the new token (warp 0, first position group)
-      if (a.owns_new && warp == 0) block(ctl->knew, ctl->vnew, pl * TB, 1);
-      // every lane gets (m, l) of every head of its group
-      float m[G], l[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        m[h] = __shfl_sync(0xffffffffu, m_l, gbase + (h << SH));
-        l[h] = __shfl_sync(0xffffffffu, l_l, gbase + (h << SH));
-      }
-      // -- merge the position groups of each warp
-#pragma unroll
-      for (int off = LPP; off < 32; off <<= 1) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, m[h], off);
-          const float l2 = __shfl_xor_sync(0xffffffffu, l[h], off);
-          const float mn = fmaxf(m[h], m2);
-          const float c1 = exp2f(m[h] - mn), c2 = exp2f(m2 - mn);
-          l[h] = l[h] * c1 + l2 * c2;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float o2 = __shfl_xor_sync(0xffffffffu, o[h][e], off);
-            o[h][e] = o[h][e] * c1 + o2 * c2;
+            q[h][e] = ctl->qs[h * HD + vi * 8 + e];
+            o[h][e] = 0.f;
           }
-          m[h] = mn;
         }
-      }
-      // -- merge the warps through shared memory, HR heads per round
-      constexpr int HR = kRedFloats / (kConsumerWarps * HD) < G ? kRedFloats / (kConsumerWarps * HD) : G;
-      const size_t pbase = ((size_t)a.b * p.nq + q0) * p.n_chunks + a.c;
-      if (pl == 0 && vi == 0) {
+        // one block of TB positions starting at row t0 of Kb/Vb (rows >= np are absent)
+        auto block = [&](const uint16_t* Kb, const uint16_t* Vb, int t0, int np) {
+          float acc[R];
+#pragma unroll
+          for (int tt = 0; tt < TB; ++tt) {
+            float kf[8];
+            if (t0 + tt < np) {
+              unpack8(*reinterpret_cast<const uint4*>(Kb + (size_t)(t0 + tt) * HD + vi * 8), kf);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) kf[e] = 0.f;
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              float d = 0.f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) d = fmaf(q[h][e], kf[e], d);
+              acc[tt * G + h] = d;
+            }
+          }
+          // every lane takes part in the reduction (full-mask shuffles), then
+          // lanes whose position is absent drop their score
+          const float red_sc = group_reduce_multi<R, LPP>(acc, lane);
+          const bool valid = t0 + my_t < np;
+          const float sc = valid ? red_sc : -1e30f;
+          float bm = sc;
+#pragma unroll
+          for (int off = G << SH; off < LPP; off <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+          const float mn = fmaxf(m_l, bm);
+          const float corr = exp2f(m_l - mn);
+          const float pv = valid ? exp2f(sc - mn) : 0.f;
+          float ps = pv;
+#pragma unroll
+          for (int off = G << SH; off < LPP; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+          l_l = l_l * corr + ps;
+          m_l = mn;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float c = __shfl_sync(0xffffffffu, corr, gbase + ((h) << SH));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[h][e] *= c;
+          }
+#pragma unroll
+          for (int tt = 0; tt < TB; ++tt) {
+            float vf[8];
+            if (t0 + tt < np) {
+              unpack8(*reinterpret_cast<const uint4*>(Vb + (size_t)(t0 + tt) * HD + vi * 8), vf);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) vf[e] = 0.f;
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float pr = __shfl_sync(0xffffffffu, pv, gbase + ((tt * G + h) << SH));
+#pragma unroll
+              for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e]);
+            }
+          }
+        };
+        // -- cached positions, streamed K stage then V stage
+        for (int s = 0; s < a.nsub; ++s) {
+          const int np = min(a.P, a.n_cached - s * a.P);
+          const uint16_t* Ks = reinterpret_cast<const uint16_t*>(wait_stage(k));
+          const uint16_t* Vs = reinterpret_cast<const uint16_t*>(wait_stage(k + 1));
+          if (tr && s == 0) tr[5] = globaltimer();
+          for (int tb = warp * PPW * TB; tb < np; tb += kConsumerWarps * PPW * TB) block(Ks, Vs, tb + pl * TB, np);
+          release();  // K slot
+          release();  // V slot
+        }
+        if (tr) tr[6] = globaltimer();
+        // -- the new token (warp 0, first position group)
+        if (a.owns_new && warp == 0) block(ctl->knew, ctl->vnew, pl * TB, 1);
+        // every lane gets (m, l) of every head of its group
+        float m[G], l[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          ctl->aml[(warp * kMaxGroup + h) * 2] = m[h];
-          ctl->aml[(warp * kMaxGroup + h) * 2 + 1] = l[h];
+          m[h] = __shfl_sync(0xffffffffu, m_l, gbase + (h << SH));
+          l[h] = __shfl_sync(0xffffffffu, l_l, gbase + (h << SH));
         }
-      }
+        // -- merge the position groups of each warp
 #pragma unroll
-      for (int h0 = 0; h0 < G; h0 += HR) {
-        if (pl == 0) {
+        for (int off = LPP; off < 32; off <<= 1) {
 #pragma unroll
-          for (int hh = 0; hh < HR; ++hh) {
+          for (int h = 0; h < G; ++h) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m[h], off);
+            const float l2 = __shfl_xor_sync(0xffffffffu, l[h], off);
+            const float mn = fmaxf(m[h], m2);
+            const float c1 = exp2f(m[h] - mn), c2 = exp2f(m2 - mn);
+            l[h] = l[h] * c1 + l2 * c2;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) red[(warp * HR + hh) * HD + vi * 8 + e] = o[h0 + hh][e];
+            for (int e = 0; e < 8; ++e) {
+              const float o2 = __shfl_xor_sync(0xffffffffu, o[h][e], off);
+              o[h][e] = o[h][e] * c1 + o2 * c2;
+            }
+            m[h] = mn;
           }
         }
-        consumer_bar();
-        for (int id = t; id < HR * HD; id += kConsumerThreads) {
-          const int hh = id / HD, d = id % HD, h = h0 + hh;
-          float M = -1e30f;
+        // -- merge the warps through shared memory, HR heads per round
+        constexpr int HR = kRedFloats / (kConsumerWarps * HD) < G ? kRedFloats / (kConsumerWarps * HD) : G;
+        const size_t pbase = ((size_t)a.b * p.nq + q0) * p.n_chunks + a.c;
+        if (pl == 0 && vi == 0) {
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ctl->aml[(w * kMaxGroup + h) * 2]);
-          float den = 0.f, num = 0.f;
-#pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) {
-            const float c = exp2f(ctl->aml[(w * kMaxGroup + h) * 2] - M);
-            den = fmaf(c, ctl->aml[(w * kMaxGroup + h) * 2 + 1], den);
-            num = fmaf(c, red[(w * HR + hh) * HD + d], num);
-          }
-          const size_t pi = pbase + (size_t)h * p.n_chunks;
-          p.part_o[pi * HD + d] = num;
-          if (d == 0) {
-            p.part_ml[pi * 2] = M;
-            p.part_ml[pi * 2 + 1] = den;
+          for (int h = 0; h < G; ++h) {
+            ctl->aml[(warp * kMaxGroup + h) * 2] = m[h];
+            ctl->aml[(warp * kMaxGroup + h) * 2 + 1] = l[h];
           }
         }
-        consumer_bar();
+#pragma unroll
+        for (int h0 = 0; h0 < G; h0 += HR) {
+          if (pl == 0) {
+#pragma unroll
+            for (int hh = 0; hh < HR; ++hh) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) red[(warp * HR + hh) * HD + vi * 8 + e] = o[h0 + hh][e];
+            }
+          }
+          consumer_bar();
+          for (int id = t; id < HR * HD; id += kConsumerThreads) {
+            const int hh = id / HD, d = id % HD, h = h0 + hh;
+            float M = -1e30f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ctl->aml[(w * kMaxGroup + h) * 2]);
+            float den = 0.f, num = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+              const float c = exp2f(ctl->aml[(w * kMaxGroup + h) * 2] - M);
+              den = fmaf(c, ctl->aml[(w * kMaxGroup + h) * 2 + 1], den);
+              num = fmaf(c, red[(w * HR + hh) * HD + d], num);
+            }
+            if (a.npieces == 1) {  // the whole row: the output itself
+              p.attn[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = num / den;
+            } else {
+              const size_t pi = pbase + (size_t)h * p.n_chunks;
+              p.part_o[pi * HD + d] = num;
+              if (d == 0) {
+                p.part_ml[pi * 2] = M;
+                p.part_ml[pi * 2 + 1] = den;
+              }
+            }
+          }
+          consumer_bar();
+        }
+      } else {
+        attn_tc<HD, G>(a, q0);
       }
     }
-    // -- ticket: the last chunk of (sequence, KV head) to arrive merges
+    if (a.npieces == 1) {  // written above: no partials to merge
+      signal(sig_idx);
+      return;
+    }
+    // -- ticket: the last piece of the row to arrive merges.  The barrier
+    // orders every thread's partial stores before thread 0's acq_rel add at
+    // gpu scope (cumulative), so the merging CTA's acquire sees them.
     consumer_bar();
     if (t == 0) {
-      __threadfence();
-      const uint32_t old =
-          atom_acq_rel_add(p.tickets + (((size_t)layer * p.B + a.b) * p.nkv + a.kvh) * nhg + a.hg, 1u);
-      ctl->last = (old + 1u == p.epoch * (uint32_t)p.n_chunks);
+      uint32_t* ticket = p.tickets + (((size_t)layer * p.B + a.b) * p.nkv + a.kvh) * nhg + a.hg;
+      const uint32_t old = atom_acq_rel_add(ticket, 1u);
+      const bool last = old + 1u == (uint32_t)a.npieces;
+      // the row's pieces have all counted: ready for the next step
+      if (last) *ticket = 0u;
+      ctl->last = last;
     }
     consumer_bar();
     if (ctl->last) {
-      // (m, l) of every (head, chunk) into shared memory with one parallel
-      // pass, then each output element reads its chunks' o with independent loads
-      const int nvalid = a.S / p.chunk + 1;  // chunks holding a position <= S
+      // (m, l) of every (head, piece) into shared memory with one parallel
+      // pass, then each output element reads its pieces' o with independent loads
+      const int nvalid = a.npieces;
       const size_t pg = ((size_t)a.b * p.nq + q0) * p.n_chunks;
       for (int idx = t; idx < G * nvalid; idx += kConsumerThreads) {
         const int h = idx / nvalid, c = idx % nvalid;
@@ -1451,7 +1703,6 @@ struct Consumer {
       }
       signal(sig_idx);
     }
-    return true;
   }
 
   __device__ __forceinline__ bool attn(const mk_instr& in, int layer, int sig_idx) {
@@ -1533,7 +1784,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
     }
     ctl->dead = 0;
     ctl->last = 0;
-    ctl->waiting = 0;
     // a sticky error from an earlier step, or out-of-range inputs: do nothing
     int bad = ld_relaxed_i32(p.status) != 0;
     for (int b = 0; b < p.B && !bad; ++b) {

@@ -7,7 +7,8 @@
 // that must not block on the allocator; or a process whose memory budget is
 // fully reserved up front.  For them this entry point runs the same
 // persistent kernel as mk_decode_step, but every byte of library state
-// (instruction lists, dependency counters, activation scratch, RoPE table)
+// (instruction lists, dependency counters, activation scratch, RoPE table,
+// the batch > 1 kernel's TMA tensor maps)
 // lives in one file-scope static device array of kStaticScratchBytes (8 MiB).
 // Every GPU that loads this library holds that array until the process exits.
 //
@@ -139,7 +140,14 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   const size_t o_off = take(sizeof(int32_t) * offsets.size());
   const size_t o_lay = take(sizeof(mk::LayerPtrs) * (size_t)L);
   const size_t o_rope = take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
+  const size_t n_tmaps = B > 1 ? (size_t)mk::kTmapsPerLayer * L + 3 : 0;  // batch > 1: TMA tensor maps
+  const size_t o_tmap = n_tmaps ? take(128 * n_tmaps) : 0;
   if (off > kStaticScratchBytes) return MK_ERR_UNSUPPORTED;  // model needs more than the 8 MiB array
+  std::vector<uint8_t> tmaps(128 * n_tmaps);
+  if (n_tmaps) {
+    const cudaError_t te = mk::encode_tmaps(d, *w, *kv, tmaps.data());
+    if (te != cudaSuccess) return te == cudaErrorInvalidValue ? MK_ERR_UNSUPPORTED : MK_ERR_CUDA;
+  }
 
   std::vector<mk::LayerPtrs> lp(L);
   for (int l = 0; l < L; ++l) {
@@ -166,7 +174,8 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
           cudaSuccess ||
       cudaMemcpyAsync(base + o_lay, lp.data(), sizeof(mk::LayerPtrs) * L, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(base + o_rope, rope.data(), sizeof(float2) * rope.size(), cudaMemcpyHostToDevice, s) !=
-          cudaSuccess)
+          cudaSuccess ||
+      (n_tmaps && cudaMemcpyAsync(base + o_tmap, tmaps.data(), tmaps.size(), cudaMemcpyHostToDevice, s) != cudaSuccess))
     return MK_ERR_CUDA;
 
   mk::Params p;
@@ -191,6 +200,7 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   p.kc = (uint16_t*)kv->k;
   p.vc = (uint16_t*)kv->v;
   p.rope = (const float2*)(base + o_rope);
+  p.tmaps = n_tmaps ? base + o_tmap : nullptr;
   p.xres = (float*)(base + o_xres);
   p.qkv = (float*)(base + o_qkv);
   p.attn = (float*)(base + o_attn);
@@ -208,7 +218,6 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   p.seq_lens = seq_lens;
   p.logits = out_logits;
   p.epoch = 1;  // counters were just cleared
-  p.l2_ahead = mk::kDefaultL2AheadBytes;
   p.copy_piece = mk::kDefaultCopyPiece;
   if (mk::launch_step(p, n_sm, s) != cudaSuccess) {
     cudaGetLastError();

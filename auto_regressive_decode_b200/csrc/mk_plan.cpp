@@ -6,9 +6,10 @@
 // and "dependency counters replacing the global synchronization".  The
 // lowering below is this library's own: every GEMV is cut into one contiguous
 // row range per SM (so each SM streams the same number of weight bytes per
-// op), attention is cut into (sequence, KV head, chunk) pieces dealt
-// round-robin over the SMs, and every instruction waits on exactly one
-// counter: the one bumped by the op it reads.
+// op), attention gets one slot per SM whose share of the step's cached
+// positions the kernel computes from the sequence lengths (equal for every
+// SM), and every instruction waits on exactly one counter: the one bumped by
+// the op it reads.
 #include <stdlib.h>
 #include <string.h>
 
@@ -111,15 +112,13 @@ struct Builder {
   }
 };
 
-int default_chunk(const mk_model_desc* d, int n_sm) {
-  const char* env = getenv("MK_ATTN_CHUNK");
-  if (env && atoi(env) > 0) return atoi(env);
+// Positions per attention unit: one ring stage of K (and one of V).
+// MK_ATTN_UNIT (1 .. that) sets a smaller unit, for tests of ragged pieces.
+int attn_unit(const mk_model_desc* d) {
   const int P = attn_stage_positions(d->head_dim);
-  int64_t total = (int64_t)d->batch * d->n_kv_heads * d->max_ctx;
-  int64_t c = (total + n_sm - 1) / n_sm;
-  c = (c + P - 1) / P * P;
-  c = std::max<int64_t>(P, std::min<int64_t>(c, 1024));
-  return (int)c;
+  const char* env = getenv("MK_ATTN_UNIT");
+  if (env && atoi(env) > 0) return std::min(atoi(env), P);
+  return P;
 }
 
 }  // namespace
@@ -131,9 +130,10 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
   const int L = d->n_layers, H = d->hidden, hd = d->head_dim;
   const int qd = d->n_q_heads * hd, kvd = d->n_kv_heads * hd;
   p->targets.assign(n_counters(L), 0);
-  p->chunk = default_chunk(d, n_sm);
-  p->n_chunks = (d->max_ctx + p->chunk - 1) / p->chunk;
-  // the merging CTA stages (m, l) of every (query head of the group, chunk) in
+  // attention: one slot per SM per layer; a row's pieces are at most n_sm
+  p->chunk = attn_unit(d);
+  p->n_chunks = n_sm;
+  // the merging CTA stages (m, l) of every (query head of the group, piece) in
   // its kRedFloats-float reduction buffer
   if (2 * attn_heads_per_instr(d->n_q_heads / d->n_kv_heads) * p->n_chunks > kRedFloats) return MK_ERR_UNSUPPORTED;
   Builder b{p};
@@ -148,21 +148,15 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
   p->targets[c_embed] = n_embed;
 
   int prev_idx = c_embed, prev_count = n_embed;
-  int64_t attn_rr = 0;
   for (int l = 0; l < L; ++l) {
     const int cq = counter_index(l, C_QKV), ca = counter_index(l, C_ATTN), co = counter_index(l, C_OPROJ);
     const int cg = counter_index(l, C_GATEUP), cd = counter_index(l, C_DOWN);
     // rows of wq | wk | wv concatenated; an instruction may span matrices
     int n_qkv = b.rows_op(OP_QKV, l, qd + 2 * kvd, {}, prev_idx, prev_count, cq);
     p->targets[cq] = n_qkv;
+    // attention: slot j = SM j; the kernel deals the step's units to the slots
     const int group = d->n_q_heads / d->n_kv_heads, nhg = group / attn_heads_per_instr(group);
-    for (int s = 0; s < d->batch; ++s)
-      for (int h = 0; h < d->n_kv_heads; ++h)
-        for (int hg = 0; hg < nhg; ++hg)
-          for (int c = 0; c < p->n_chunks; ++c) {
-            b.emit((int)(attn_rr % n_sm), OP_ATTN, l, cq, n_qkv, ca, s, h, c, hg);
-            ++attn_rr;
-          }
+    for (int s = 0; s < n_sm; ++s) b.emit(s, OP_ATTN, l, cq, n_qkv, ca, s, n_sm, 0, 0);
     p->targets[ca] = d->batch * d->n_kv_heads * nhg;  // one bump per merged (sequence, KV head, head group)
     int n_o = b.rows_op(OP_OPROJ, l, H, {}, ca, p->targets[ca], co);
     p->targets[co] = n_o;
@@ -240,6 +234,37 @@ extern "C" int mk_plan_attn_chunk(const mk_plan* p, int32_t* chunk, int32_t* n_c
   *chunk = p->chunk;
   *n_chunks = p->n_chunks;
   return MK_OK;
+}
+
+extern "C" int mk_plan_attn_pieces(const mk_plan* p, const int32_t* seq_lens, int32_t* out, int32_t max_pieces,
+                                   int32_t* n_out) {
+  if (!p || !seq_lens || !n_out || max_pieces < 0 || (max_pieces > 0 && !out)) return MK_ERR_INVALID_ARG;
+  for (int b = 0; b < p->d.batch; ++b)
+    if (seq_lens[b] < 0 || seq_lens[b] >= p->d.max_ctx) return MK_ERR_RANGE;
+  const int group = p->d.n_q_heads / p->d.n_kv_heads;
+  mk::AttnSched sc;
+  mk::attn_sched_init(sc, seq_lens, p->d.batch, p->d.n_kv_heads * (group / mk::attn_heads_per_instr(group)), p->chunk,
+                  p->n_chunks);
+  int n = 0;
+  for (int j = 0; j < sc.n_slots; ++j) {
+    for (int64_t g = mk::attn_slot_begin(sc, j), g1 = mk::attn_slot_begin(sc, j + 1); g < g1;) {
+      const mk::AttnPiece pc = mk::attn_piece_at(sc, g, j);
+      if (n < max_pieces) {
+        int32_t* o = out + (size_t)n * 7;
+        o[0] = j;
+        o[1] = pc.b;
+        o[2] = pc.row;
+        o[3] = pc.ua;
+        o[4] = pc.ub;
+        o[5] = pc.slot_in_row;
+        o[6] = pc.n_pieces;
+      }
+      ++n;
+      g += pc.ub - pc.ua;
+    }
+  }
+  *n_out = n;
+  return n <= max_pieces ? MK_OK : MK_ERR_INVALID_ARG;
 }
 
 extern "C" int mk_plan_destroy(mk_plan* p) {

@@ -1,4 +1,4 @@
-// TMA tensor maps of the weight matrices, for the batch > 1 tensor-core GEMV.
+// TMA tensor maps of the weight matrices and KV caches, for the batch > 1 kernel.
 //
 // A row-major bf16 matrix W[N][K] (K a multiple of 64) is described as the
 // 3-D tensor (64, N, K/64) with strides (2 B, 2K B, 128 B): element
@@ -6,7 +6,9 @@
 // brings kBBoxRows rows of one kBChunk-column chunk into shared memory as
 // [column block][row][64 columns], with the 128-byte swizzle (16-byte chunk
 // c of 128-byte line L at position c ^ (L & 7)).  Coordinates past K/64 read
-// as zeros (the tail chunk of a K that is not a multiple of kBChunk).
+// as zeros (the tail chunk of a K that is not a multiple of kBChunk).  The KV
+// caches get the same view with head_dim columns and one attention stage of
+// positions per box.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <string.h>
@@ -34,13 +36,14 @@ EncodeTiledFn encoder() {
   return fn;
 }
 
-bool encode_one(EncodeTiledFn enc, const void* w, int rows, int K, uint8_t* out) {
+bool encode_one(EncodeTiledFn enc, const void* w, int64_t rows, int K, uint8_t* out, int box_rows = kBBoxRows,
+                int box_blocks = kBChunk / 64) {
   static_assert(sizeof(CUtensorMap) == 128, "tensor map size");
-  if (!w || rows <= 0 || K % 64) return false;
+  if (!w || rows <= 0 || rows >= (1ll << 31) || K % 64) return false;  // rows are int coordinates
   CUtensorMap m;
   const cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(K / 64)};
   const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
-  const cuuint32_t box[3] = {64, (cuuint32_t)kBBoxRows, (cuuint32_t)(kBChunk / 64)};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_blocks};
   const cuuint32_t elem[3] = {1, 1, 1};
   const CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims, strides, box, elem,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -52,7 +55,7 @@ bool encode_one(EncodeTiledFn enc, const void* w, int rows, int K, uint8_t* out)
 
 }  // namespace
 
-cudaError_t encode_weight_tmaps(const mk_model_desc& d, const mk_weights& w, uint8_t* out) {
+cudaError_t encode_tmaps(const mk_model_desc& d, const mk_weights& w, const mk_kv& kv, uint8_t* out) {
   EncodeTiledFn enc = encoder();
   if (!enc) return cudaErrorNotSupported;
   const int H = d.hidden, qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim, I = d.ffn_dim;
@@ -66,7 +69,14 @@ cudaError_t encode_weight_tmaps(const mk_model_desc& d, const mk_weights& w, uin
     if (!ok) return cudaErrorInvalidValue;
   }
   const void* lm = d.tied_embeddings ? w.embed : w.lm_head;
-  if (!encode_one(enc, lm, d.vocab, H, out + (size_t)d.n_layers * kTmapsPerLayer * 128))
+  uint8_t* g = out + (size_t)d.n_layers * kTmapsPerLayer * 128;
+  if (!encode_one(enc, lm, d.vocab, H, g)) return cudaErrorInvalidValue;
+  // KV caches: rows are (layer, sequence, KV head, position), head_dim columns;
+  // a box is one attention stage of positions
+  const int64_t kv_rows = (int64_t)d.n_layers * d.batch * d.n_kv_heads * d.max_ctx;
+  const int P = attn_stage_positions(d.head_dim);
+  if (!encode_one(enc, kv.k, kv_rows, d.head_dim, g + 128, P, d.head_dim / 64) ||
+      !encode_one(enc, kv.v, kv_rows, d.head_dim, g + 256, P, d.head_dim / 64))
     return cudaErrorInvalidValue;
   return cudaSuccess;
 }

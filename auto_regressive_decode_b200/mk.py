@@ -79,6 +79,7 @@ def _load():
         "mk_plan_copy": (_i32, [H, _P, _P]),
         "mk_plan_counter_targets": (_i32, [H, _P]),
         "mk_plan_attn_chunk": (_i32, [H, ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
+        "mk_plan_attn_pieces": (_i32, [H, _P, _P, _i32, ctypes.POINTER(_i32)]),
         "mk_plan_destroy": (_i32, [H]),
     }
     for name, (res, args) in sig.items():
@@ -105,6 +106,7 @@ mk_plan_n_instrs = lib.mk_plan_n_instrs
 mk_plan_copy = lib.mk_plan_copy
 mk_plan_counter_targets = lib.mk_plan_counter_targets
 mk_plan_attn_chunk = lib.mk_plan_attn_chunk
+mk_plan_attn_pieces = lib.mk_plan_attn_pieces
 mk_plan_destroy = lib.mk_plan_destroy
 
 
@@ -156,6 +158,23 @@ class Plan:
             check(mk_plan_attn_chunk(h, ctypes.byref(c), ctypes.byref(nch)), "mk_plan_attn_chunk")
             self.chunk, self.n_chunks = c.value, nch.value
             self.n_sm = n_sm
+        finally:
+            mk_plan_destroy(h)
+        self._desc = desc
+
+    def attn_pieces(self, seq_lens):
+        """int32[n][7] (slot, b, row, first unit, end unit, piece index in row, pieces of row) for one step."""
+        import numpy as np
+        sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        h = _P()
+        check(mk_plan_create(ctypes.byref(self._desc), self.n_sm, ctypes.byref(h)), "mk_plan_create")
+        try:
+            n = _i32()
+            mk_plan_attn_pieces(h, sl.ctypes.data, None, 0, ctypes.byref(n))
+            out = np.zeros((max(n.value, 1), 7), dtype=np.int32)
+            check(mk_plan_attn_pieces(h, sl.ctypes.data, out.ctypes.data, n.value, ctypes.byref(n)),
+                  "mk_plan_attn_pieces")
+            return out[:n.value]
         finally:
             mk_plan_destroy(h)
 

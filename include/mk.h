@@ -194,8 +194,20 @@ int mk_plan_n_instrs(const mk_plan* p);
 int mk_plan_copy(const mk_plan* p, mk_instr* instrs, int32_t* offsets);
 /* Per-step producers of each counter: int32[n_counters]. */
 int mk_plan_counter_targets(const mk_plan* p, int32_t* targets);
-/* Attention split: positions per chunk and chunks per sequence. */
+/* Attention schedule: `chunk` = positions per unit (one ring stage of K and
+ * one of V), `n_chunks` = slots (one per SM per layer; also the most pieces a
+ * (sequence, KV head, head group) row is cut into). */
 int mk_plan_attn_chunk(const mk_plan* p, int32_t* chunk, int32_t* n_chunks);
+/* The attention pieces the kernel derives for one step from `seq_lens`
+ * (host int32[batch]): every row (sequence b, KV head, head group) covers
+ * positions 0..seq_lens[b] in units of `chunk` positions, and the units of
+ * all rows, in row order, are dealt to the slots as equal contiguous runs.
+ * Writes up to max_pieces records of 7 int32 (slot, b, row, first unit,
+ * end unit, index of the piece within its row, pieces of the row) to `out`
+ * and the total count to *n_out; MK_ERR_INVALID_ARG when it exceeds
+ * max_pieces, MK_ERR_RANGE for a length outside [0, max_ctx). */
+int mk_plan_attn_pieces(const mk_plan* p, const int32_t* seq_lens, int32_t* out, int32_t max_pieces,
+                        int32_t* n_out);
 int mk_plan_destroy(mk_plan* p);
 
 #ifdef __cplusplus

@@ -27,8 +27,8 @@ def test_tiny_variants(kw, gains):
     assert_parity(res)
 
 
-def test_tiny_head_dim_128_small_chunks(monkeypatch):
-    monkeypatch.setenv("MK_ATTN_CHUNK", "40")            # many chunks, ragged last sub-chunk
+def test_tiny_head_dim_128_small_units(monkeypatch):
+    monkeypatch.setenv("MK_ATTN_UNIT", "40")             # 40-position units: rows cut into many pieces
     cfg = fx.CONFIGS["tiny"].replace(n_q_heads=4, n_kv_heads=2, head_dim=128, ctx=200, steps=3)
     assert_parity(run_teacher_forced(cfg, gains="random"))
 
@@ -54,6 +54,14 @@ def test_dense_0_6b_first_steps():
 def test_tiny_batched(kw, gains):
     cfg = fx.CONFIGS["tiny"].replace(ffn_dim=704, **kw)
     assert_parity(run_teacher_forced(cfg, steps=kw.get("steps", 3), gains=gains))
+
+
+def test_batched_small_units(monkeypatch):
+    # tensor-core attention with 24-position units: every stage box carries
+    # positions past the piece (masked keys, zeroed values) and rows span many slots
+    monkeypatch.setenv("MK_ATTN_UNIT", "24")
+    cfg = fx.CONFIGS["tiny"].replace(ffn_dim=704, batch=5, ctx=0, ctx_lo=1, ctx_hi=140, steps=3)
+    assert_parity(run_teacher_forced(cfg, gains="random"))
 
 
 def test_batched_multi_chunk():

@@ -39,7 +39,8 @@ def test_rows_and_chunks_covered_once(name, n_sm):
     for row in p.instrs:
         op, layer = p.op(row), p.layer(row)
         if op == OP_ATTN:
-            attn[(layer, int(row[4]), int(row[5]), int(row[6]), int(row[7]))] += 1
+            attn[(layer, int(row[4]))] += 1
+            assert int(row[5]) == n_sm
         else:
             cover[(layer, op)].append((int(row[4]), int(row[5])))
             assert 0 < row[5] - row[4] <= 256
@@ -47,11 +48,12 @@ def test_rows_and_chunks_covered_once(name, n_sm):
         segs.sort()
         assert segs[0][0] == 0 and segs[-1][1] == rows_of(cfg, op)
         assert all(a[1] == b[0] for a, b in zip(segs, segs[1:])), (layer, op)
-    group = cfg.n_q_heads // cfg.n_kv_heads
-    nhg = group // min(group, 4)
-    assert len(attn) == cfg.n_layers * cfg.batch * cfg.n_kv_heads * nhg * p.n_chunks
+    # attention: one slot per SM per layer, on that SM; units of one ring stage
+    assert set(attn) == {(l, s) for l in range(cfg.n_layers) for s in range(n_sm)}
     assert set(attn.values()) == {1}
-    assert p.chunk * p.n_chunks >= cfg.max_ctx > p.chunk * (p.n_chunks - 1)
+    for s in range(n_sm):
+        assert all(int(r[4]) == s for r in p.sm_list(s) if p.op(r) == OP_ATTN)
+    assert p.chunk == 32768 // (2 * cfg.head_dim) and p.n_chunks == n_sm
 
 
 @pytest.mark.parametrize("name,n_sm", CASES)
@@ -86,11 +88,18 @@ def test_counter_targets_and_wait_order(name, n_sm):
         assert keys == sorted(keys)
 
 
-def simulate(p, cfg, order_seed=0):
-    """Counter protocol on the host: SMs progress in a random order; returns instructions executed."""
+def simulate(p, cfg, order_seed=0, seq_lens=None):
+    """Counter protocol on the host: SMs progress in a random order; returns instructions executed.
+
+    An attention slot runs its pieces for this step's lengths; the last piece
+    of a (sequence, KV head, head group) row to count bumps the layer's counter."""
     rng = np.random.default_rng(order_seed)
     counters = np.zeros(len(p.targets), dtype=np.int64)
     tickets = collections.Counter()
+    pieces = p.attn_pieces(fx.context_lengths(cfg) if seq_lens is None else seq_lens)
+    by_slot = collections.defaultdict(list)
+    for pc in pieces:
+        by_slot[int(pc[0])].append(pc)
     pos = [0] * p.n_sm
     done = 0
     total = len(p.instrs)
@@ -104,10 +113,11 @@ def simulate(p, cfg, order_seed=0):
                 if w >= 0 and counters[w] < int(r[2]):
                     break
                 if p.op(r) == OP_ATTN:
-                    key = (p.layer(r), int(r[4]), int(r[5]), int(r[7]))
-                    tickets[key] += 1
-                    if tickets[key] == p.n_chunks:
-                        counters[int(r[3])] += 1
+                    for pc in by_slot[int(r[4])]:
+                        key = (p.layer(r), int(pc[1]), int(pc[2]))
+                        tickets[key] += 1
+                        if tickets[key] == int(pc[6]):
+                            counters[int(r[3])] += 1
                 elif int(r[3]) >= 0:
                     counters[int(r[3])] += 1
                 pos[s] += 1
@@ -119,7 +129,8 @@ def simulate(p, cfg, order_seed=0):
     return done
 
 
-@pytest.mark.parametrize("name,n_sm", [("tiny", 148), ("tiny", 3), ("dense-0.6b", 148), ("dense-8b", 148)])
+@pytest.mark.parametrize("name,n_sm", [("tiny", 148), ("tiny", 3), ("dense-0.6b", 148), ("dense-8b", 148),
+                                       ("dense-13b-b8", 148)])
 def test_counter_protocol_completes(name, n_sm):
     cfg, p = plan_of(name, n_sm)
     for seed in range(2):
@@ -187,3 +198,63 @@ def test_batched_row_ranges_on_box_boundaries(name, kw, n_sm):
                 if p.op(r) == op and p.layer(r) == 0:
                     per[s] += int(r[5]) - int(r[4])
         assert max(per.values()) <= rows_of(cfg, op) / n_sm + 8
+
+
+def _pieces_reference(seq_lens, rows_per_seq, unit, n_slots):
+    """The schedule restated directly: units of every row in row order, dealt in equal runs."""
+    owner = []                                   # (b, row, unit) of every global unit
+    for b, S in enumerate(seq_lens):
+        for r in range(rows_per_seq):
+            owner += [(b, r, u) for u in range(S // unit + 1)]
+    U = len(owner)
+    n = min(n_slots, U)                          # a slot in use holds at least one unit
+    out = []
+    for j in range(n):
+        run = owner[U * j // n:U * (j + 1) // n]
+        k = 0
+        while k < len(run):
+            b, r, ua = run[k]
+            e = k
+            while e < len(run) and run[e][:2] == (b, r):
+                e += 1
+            out.append((j, b, r, ua, run[e - 1][2] + 1))
+            k = e
+    return out
+
+
+@pytest.mark.parametrize("name,kw,n_sm,lens", [
+    ("dense-13b-b8", {}, 148, None),
+    ("dense-13b-b8", {}, 148, [0, 0, 0, 0, 0, 0, 0, 4159]),
+    ("dense-8b", {}, 148, [4096]),
+    ("tiny", {"batch": 5, "ffn_dim": 704}, 7, [0, 1, 127, 128, 140]),
+    ("tiny", {"batch": 3, "n_q_heads": 8, "n_kv_heads": 1, "ffn_dim": 704}, 148, [3, 0, 9]),
+])
+def test_attention_schedule_partition(name, kw, n_sm, lens):
+    cfg, p = plan_of(name, n_sm, **kw)
+    lens = fx.context_lengths(cfg) if lens is None else np.asarray(lens, dtype=np.int32)
+    group = cfg.n_q_heads // cfg.n_kv_heads
+    rows_per_seq = cfg.n_kv_heads * (group // min(group, 4))
+    pieces = p.attn_pieces(lens)
+    # the library's pieces are the restated schedule's
+    assert [tuple(int(x) for x in pc[:5]) for pc in pieces] == _pieces_reference(lens, rows_per_seq, p.chunk, n_sm)
+    # every unit of every row exactly once; slots' unit counts differ by at most one
+    per_slot = collections.Counter()
+    covered = collections.defaultdict(list)
+    for j, b, r, ua, ub, k, npc in (tuple(int(x) for x in pc) for pc in pieces):
+        per_slot[j] += ub - ua
+        covered[(b, r)].append((ua, ub, k, npc))
+    assert max(per_slot.values(), default=0) - min([per_slot[j] for j in range(n_sm)]) <= 1
+    assert set(covered) == {(b, r) for b in range(cfg.batch) for r in range(rows_per_seq)}
+    for (b, r), segs in covered.items():
+        segs.sort()
+        assert segs[0][0] == 0 and segs[-1][1] == int(lens[b]) // p.chunk + 1
+        assert all(x[1] == y[0] for x, y in zip(segs, segs[1:]))
+        assert [s[2] for s in segs] == list(range(len(segs))) and {s[3] for s in segs} == {len(segs)}
+    # the counter protocol completes under these lengths too
+    assert simulate(p, cfg, 0, lens) == len(p.instrs)
+
+
+def test_attention_schedule_rejects_out_of_range_lengths():
+    cfg, p = plan_of("tiny", 148)
+    with pytest.raises(mk.MkError):
+        p.attn_pieces([cfg.max_ctx])

@@ -21,10 +21,11 @@ from tests.helpers import bf16_f64, rel_l2
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name", ["tiny", "dense-0.6b"])
-def test_noalloc_matches_allocating_path_two_calls(name):
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("dense-0.6b", {}),
+                                     ("tiny", {"batch": 4, "ffn_dim": 704, "ctx": 0, "ctx_lo": 5, "ctx_hi": 130})])
+def test_noalloc_matches_allocating_path_two_calls(name, kw):
     import auto_regressive_decode_b200.mk as mk
-    cfg = fx.CONFIGS[name]
+    cfg = fx.CONFIGS[name].replace(**kw)
     S0 = fx.context_lengths(cfg)
     toks = fx.tokens(cfg)
     w = device_model(cfg)
@@ -49,9 +50,10 @@ def test_noalloc_matches_allocating_path_two_calls(name):
         assert np.isfinite(b).all()
         assert float(np.max(np.abs(a - b))) <= TOL_LOGITS_ABS
         for cache_a, cache_b in ((kc_a, kc_b), (vc_a, vc_b)):
-            ra = bf16_f64(bits(cache_a[:, 0, :, S[0]].contiguous()))
-            rb = bf16_f64(bits(cache_b[:, 0, :, S[0]].contiguous()))
-            assert rel_l2(rb, ra) <= TOL_KV
+            for b in range(cfg.batch):
+                ra = bf16_f64(bits(cache_a[:, b, :, S[b]].contiguous()))
+                rb = bf16_f64(bits(cache_b[:, b, :, S[b]].contiguous()))
+                assert rel_l2(rb, ra) <= TOL_KV
         lb.fill_(float("nan"))
     dec.close()
     del keep
