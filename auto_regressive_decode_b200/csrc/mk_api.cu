@@ -87,6 +87,7 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
     for (const void* q : need)
       if (!aligned16(q)) return q ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
     if (d.qk_norm && (!aligned16(lw.q_norm) || !aligned16(lw.k_norm))) return MK_ERR_INVALID_ARG;
+    if (d.n_experts && !aligned16(lw.router)) return lw.router ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
   }
 
   int dev = 0, n_sm = 0, coop = 0, smem_optin = 0;
@@ -95,10 +96,10 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) return MK_ERR_CUDA;
   if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return MK_ERR_CUDA;
-  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes(d.batch > 1)) return MK_ERR_UNSUPPORTED;
+  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes(mk::batched(d))) return MK_ERR_UNSUPPORTED;
   if (mk::kernel_prepare() != cudaSuccess) return MK_ERR_CUDA;
   int per_sm = 0;
-  if (mk::kernel_occupancy(&per_sm, d.batch > 1) != cudaSuccess) return MK_ERR_CUDA;
+  if (mk::kernel_occupancy(&per_sm, mk::batched(d)) != cudaSuccess) return MK_ERR_CUDA;
   if (per_sm < 1) return MK_ERR_UNSUPPORTED;
 
   mk_plan* plan = nullptr;
@@ -129,7 +130,13 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const size_t o_xres = cv.take(sizeof(float) * (size_t)(2 * L + 1) * B * H);
   const size_t o_qkv = cv.take(sizeof(float) * (size_t)B * (qd + 2 * kvd));
   const size_t o_attn = cv.take(sizeof(float) * (size_t)B * qd);
-  const size_t o_act = cv.take(sizeof(float) * (size_t)B * d.ffn_dim);
+  const size_t o_act = cv.take(sizeof(float) * (size_t)B * (d.n_experts ? 1 : d.ffn_dim));
+  const int E = d.n_experts, K = d.top_k;
+  const size_t o_mr = E ? cv.take(sizeof(float) * (size_t)L * B * E) : 0;
+  const size_t o_ms = E ? cv.take(sizeof(int32_t) * (size_t)L * B * K) : 0;
+  const size_t o_mw = E ? cv.take(sizeof(float) * (size_t)L * B * K) : 0;
+  const size_t o_mc = E ? cv.take(sizeof(int32_t) * (size_t)L) : 0;
+  const size_t o_ma = E ? cv.take(sizeof(float) * (size_t)mk::moe_slots(E, B, K) * B * d.expert_ffn_dim) : 0;
   const size_t o_po = cv.take(sizeof(float) * (size_t)B * nq * n_chunks * hd);
   const size_t o_pml = cv.take(sizeof(float) * (size_t)B * nq * n_chunks * 2);
   const size_t o_cnt = cv.take(sizeof(uint32_t) * (size_t)n_cnt);
@@ -139,7 +146,7 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const size_t o_off = cv.take(sizeof(int32_t) * offsets.size());
   const size_t o_lay = cv.take(sizeof(mk::LayerPtrs) * (size_t)L);
   const size_t o_rope = cv.take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
-  const size_t n_tmaps = B > 1 ? (size_t)mk::kTmapsPerLayer * L + 3 : 0;
+  const size_t n_tmaps = mk::batched(d) ? (size_t)mk::kTmapsPerLayer * L + 3 : 0;
   const size_t o_tmap = n_tmaps ? cv.take(128 * n_tmaps) : 0;
   const char* trace_env = getenv("MK_TRACE");
   const bool tracing = trace_env && atoi(trace_env) > 0;
@@ -211,6 +218,7 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   p.I = d.ffn_dim;
   p.V = d.vocab;
   p.B = B;
+  p.tc = mk::batched(d);
   p.T = d.max_ctx;
   p.qk_norm = d.qk_norm;
   p.eps = d.rms_eps;
@@ -230,6 +238,16 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   p.act = (float*)(base + o_act);
   p.part_o = (float*)(base + o_po);
   p.part_ml = (float*)(base + o_pml);
+  if (E) {
+    p.E = E;
+    p.topk = K;
+    p.Ie = d.expert_ffn_dim;
+    p.moe_router = (float*)(base + o_mr);
+    p.moe_sel = (int32_t*)(base + o_ms);
+    p.moe_selw = (float*)(base + o_mw);
+    p.moe_count = (int32_t*)(base + o_mc);
+    p.moe_act = (float*)(base + o_ma);
+  }
   p.counters = (uint32_t*)(base + o_cnt);
   p.tickets = (uint32_t*)(base + o_tk);
   p.status = (int*)(base + o_st);
@@ -291,6 +309,10 @@ extern "C" size_t mk_state_bytes(const mk_handle* h, int which) {
   const mk_model_desc& d = h->d;
   switch (which) {
     case MK_STATE_HIDDEN: return sizeof(float) * (size_t)(2 * d.n_layers + 1) * d.batch * d.hidden;
+    case MK_STATE_ROUTER: return sizeof(float) * (size_t)d.n_layers * d.batch * d.n_experts;
+    case MK_STATE_SELECTION: return d.n_experts ? sizeof(int32_t) * (size_t)d.n_layers * d.batch * d.top_k : 0;
+    case MK_STATE_SEL_WEIGHT: return d.n_experts ? sizeof(float) * (size_t)d.n_layers * d.batch * d.top_k : 0;
+    case MK_STATE_EXPERT_COUNT: return d.n_experts ? sizeof(int32_t) * (size_t)d.n_layers : 0;
     case MK_STATE_TRACE: return sizeof(uint64_t) * mk::kTraceStamps * h->n_instr;
     default: return 0;
   }
@@ -304,6 +326,10 @@ extern "C" int mk_read_state(mk_handle* h, int which, void* dst, size_t bytes, v
   const void* src = nullptr;
   if (which == MK_STATE_HIDDEN) src = h->p.xres;
   if (which == MK_STATE_TRACE) src = h->p.trace;
+  if (which == MK_STATE_ROUTER) src = h->p.moe_router;
+  if (which == MK_STATE_SELECTION) src = h->p.moe_sel;
+  if (which == MK_STATE_SEL_WEIGHT) src = h->p.moe_selw;
+  if (which == MK_STATE_EXPERT_COUNT) src = h->p.moe_count;
   if (cudaMemcpyAsync(dst, src, need, cudaMemcpyDefault, (cudaStream_t)stream) != cudaSuccess) return MK_ERR_CUDA;
   return MK_OK;
 }

@@ -16,6 +16,7 @@ struct LayerPtrs {
 struct Params {
   // shape
   int L, H, nq, nkv, hd, I, V, B, T, qk_norm;
+  int tc;  // the tensor-core kernel (batch > 1 or MoE)
   float eps;
   int chunk, n_chunks;
   // weights (device)
@@ -37,6 +38,14 @@ struct Params {
   float* act;               // [B][I]
   float* part_o;            // [B][nq][n_chunks][hd]
   float* part_ml;           // [B][nq][n_chunks][2]
+  // MoE: E experts, top-k, expert SwiGLU width Ie; router logits and routing
+  // of every layer of the step (kept for mk_read_state)
+  int E, topk, Ie;
+  float* moe_router;        // [L][B][E]
+  int32_t* moe_sel;         // [L][B][topk] picked experts, best first
+  float* moe_selw;          // [L][B][topk] their weights
+  int32_t* moe_count;       // [L] distinct picked experts
+  float* moe_act;           // [slots][B][Ie] SwiGLU outputs of the picked experts
   uint32_t* counters;       // [n_counters]
   uint32_t* tickets;        // [L][B][nkv]
   const mk_instr* instrs;

@@ -122,8 +122,29 @@ constexpr int kBBoxRows = 8;                         // weight rows per TMA box
 constexpr int kBBoxBytes = kBBoxRows * kBChunk * 2;  // 16 KB
 constexpr int kBatchedMaxRows = 128;                 // rows per instruction: 8 tiles of 16
 constexpr int kBatchedMaxRowsGated = 96;             // gate/up: 12 tiles of 8 neurons
-constexpr int kTmapsPerLayer = 7;                    // wq wk wv wo w_gate w_up w_down (+ one LM head map)
+constexpr int kTmapsPerLayer = 8;  // wq wk wv wo w_gate w_up w_down router (then LM head, K cache, V cache)
 MK_HD int btile_rows(bool gated) { return gated ? 8 : 16; }
+// The tensor-core kernel runs every batch > 1 model and every MoE model.
+MK_HD bool batched(const mk_model_desc& d) { return d.batch > 1 || d.n_experts > 0; }
+
+// ---- mixture of experts ------------------------------------------------------------
+// Router GEMV over the experts, top-k per sequence, then the distinct picked
+// experts ("slots", ascending expert index).  Gate/up work is (slot, 8-neuron
+// tile) units dealt evenly to one instruction per SM; down is split by output
+// rows and runs over all slots, the routing weights folded into its inputs.
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 8;
+constexpr int kMaxSel = 64;  // distinct experts of one step: at most batch * top_k
+MK_HD int moe_slots(int n_experts, int batch, int top_k) {
+  return n_experts < batch * top_k ? n_experts : batch * top_k;
+}
+
+// Even deal of U units to n slots (n cut to U when U < n, so that every slot
+// in use holds a unit): the first unit of slot j.
+MK_HD int64_t even_begin(int64_t U, int n, int j) {
+  const int m = U < n ? (int)U : n;
+  return j >= m ? U : U * j / m;
+}
 
 // ---- attention split -------------------------------------------------------------
 // Query heads one attention instruction handles: a KV head with more query

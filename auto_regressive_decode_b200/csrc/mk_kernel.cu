@@ -48,6 +48,14 @@ struct Ctl {
   alignas(16) uint16_t knew[kMaxHeadDim];     // the new token's K/V rows (bf16, as appended)
   alignas(16) uint16_t vnew[kMaxHeadDim];
   AttnSched psched;  // the producer's attention schedule of its current slot
+  // MoE: the current layer's routing.  The consumers compute it; the
+  // producer, which cannot stream expert weights before it exists, waits for
+  // moe_pub == layer + 1.
+  int moe_pub;
+  int moe_count;                       // distinct picked experts (slots)
+  int16_t moe_uniq[kMaxSel];           // expert of each slot, ascending
+  uint32_t moe_mask[kMaxExperts / 32];
+  float moe_tw[kMaxSel][kMaxBatch];    // routing weight of (slot, sequence); 0 if not picked
 };
 
 // Shared memory: the ring of weight / KV stages (slots 1024-byte aligned, as
@@ -406,6 +414,14 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
         g.sw0 = lp.w_gate + (size_t)g.r0 * g.K;
         g.wup = lp.w_up + (size_t)g.r0 * g.K;
         break;
+      case OP_ROUTER:
+        g.K = p.H;
+        g.sw0 = lp.router + (size_t)g.r0 * g.K;
+        break;
+      case OP_EXP_DOWN:  // rows of every picked expert's down matrix (tensor maps)
+        g.K = p.Ie;
+        g.sw0 = lp.w_down;
+        break;
       default:  // OP_DOWN
         g.K = p.I;
         g.sw0 = lp.w_down + (size_t)g.r0 * g.K;
@@ -415,12 +431,45 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
   g.ks = gemv_ksplit(g.K, g.wup ? 2 : 1);
   g.Kc = g.K / g.ks;
   g.tile = gemv_tile(g.Kc, g.wup ? 2 : 1);
-  if (p.B > 1) {
+  if (p.tc) {
     const int tr = btile_rows(g.wup != nullptr);
     g.bnch = (g.K + kBChunk - 1) / kBChunk;
     g.bnt = (g.r1 - g.r0 + tr - 1) / tr;
   }
   return g;
+}
+
+// MoE down: its K runs over the picked experts one after another, each in
+// chunks of kBChunk of its Ie columns.
+__device__ __forceinline__ int moe_down_chunks(const Params& p) { return (p.Ie + kBChunk - 1) / kBChunk; }
+
+// MoE gate/up: the piece of an expert slot instruction that starts at unit g
+// (units are (slot, 8-neuron tile), slot-major) and ends by g1, at most
+// kBatchedMaxRowsGated rows.  Geometry in the stacked [E * Ie] row space.
+__device__ __forceinline__ Gemv moe_gate_piece(const Params& p, const Ctl* ctl, int layer, int64_t g, int64_t g1,
+                                               int* slot) {
+  const int nte = p.Ie / 8;
+  const int s = (int)(g / nte), t0 = (int)(g % nte);
+  const int64_t left = g1 - g < (int64_t)(kBatchedMaxRowsGated / 8) ? g1 - g : (int64_t)(kBatchedMaxRowsGated / 8);
+  const int t1 = (int)(nte - t0 < left ? nte : t0 + left);
+  const int e = ctl->moe_uniq[s];
+  const LayerPtrs& lp = p.layers[layer];
+  Gemv gm;
+  gm.K = p.H;
+  gm.r0 = e * p.Ie + t0 * 8;
+  gm.r1 = e * p.Ie + t1 * 8;
+  gm.nseg = 1;
+  gm.sn0 = gm.r1 - gm.r0;
+  gm.sn1 = gm.sn2 = 0;
+  gm.sw0 = lp.w_gate;
+  gm.sw1 = gm.sw2 = nullptr;
+  gm.wup = lp.w_up;
+  gm.ks = 1;
+  gm.Kc = gm.K;
+  gm.bnch = (p.H + kBChunk - 1) / kBChunk;
+  gm.bnt = t1 - t0;
+  *slot = s;
+  return gm;
 }
 
 // One attention piece: units [ua, ub) of row (b, kvh, hg), i.e. positions
@@ -478,9 +527,12 @@ struct Cursor {
   AttnSched* sc;   // attention: this step's schedule (shared memory), slot aslot's units [ag, ag1)
   int64_t ag, ag1;
   int aslot, pieceu;  // slot, units of the current piece
+  const Ctl* ctl;     // MoE: the layer's routing
+  bool pending;       // an expert instruction waits for its layer's routing
+  int eslot;          // MoE gate/up: expert slot of the current piece (units [ag, ag1) as above)
 
-  __device__ Cursor(const Params& prm, const mk_instr* l, int nn, AttnSched* sched)
-      : pp(&prm), list(l), n(nn), i(0), sc(sched) {}
+  __device__ Cursor(const Params& prm, const mk_instr* l, int nn, AttnSched* sched, const Ctl* c)
+      : pp(&prm), list(l), n(nn), i(0), sc(sched), ctl(c), pending(false) {}
 
   // Position on the first stage of instruction j or of the next one that has stages.
   __device__ __forceinline__ void seek(int j) {
@@ -495,12 +547,37 @@ struct Cursor {
         ag1 = attn_slot_begin(*sc, aslot + 1);
         sub = kv = 0;
         if (next_piece()) return;
-      } else if (op >= OP_QKV && op <= OP_LMHEAD) {
+      } else if (op == OP_EXP_GATEUP || op == OP_EXP_DOWN) {
+        if (*(const volatile int*)&ctl->moe_pub != layer + 1) {
+          pending = true;  // the producer waits, then seeks here again
+          return;
+        }
+        __threadfence_block();
+        kc = sg = rr = 0;
+        if (op == OP_EXP_DOWN) {
+          g = gemv_geo(*pp, in, op, layer);
+          g.bnch = ctl->moe_count * moe_down_chunks(*pp);
+          if (g.bnch > 0) return;
+        } else {
+          const int64_t U = (int64_t)ctl->moe_count * (pp->Ie / 8);
+          ag = even_begin(U, in.b, in.a);
+          ag1 = even_begin(U, in.b, in.a + 1);
+          if (next_moe_piece()) return;
+        }
+      } else if ((op >= OP_QKV && op <= OP_LMHEAD) || op == OP_ROUTER) {
         g = gemv_geo(*pp, in, op, layer);
         kc = sg = rr = 0;
         return;
       }
     }
+  }
+
+  // MoE gate/up: the piece of the slot that starts at unit ag, if any.
+  __device__ __forceinline__ bool next_moe_piece() {
+    if (ag >= ag1) return false;
+    g = moe_gate_piece(*pp, ctl, layer, ag, ag1, &eslot);
+    kc = sg = rr = 0;
+    return true;
   }
 
   // From unit ag on: the first piece of the slot that has cached positions.
@@ -525,10 +602,16 @@ struct Cursor {
       }
       return;
     }
-    if (pp->B > 1) {  // batched GEMV: chunk kc, tile sg within it
+    if (pp->tc) {  // batched GEMV: chunk kc, tile sg within it
       if (++sg >= g.bnt) {
         sg = 0;
-        if (++kc >= g.bnch) seek(i + 1);
+        if (++kc >= g.bnch) {
+          if (op == OP_EXP_GATEUP) {
+            ag += g.bnt;
+            if (next_moe_piece()) return;
+          }
+          seek(i + 1);
+        }
       }
       return;
     }
@@ -588,6 +671,12 @@ struct Cursor {
       return 2u * kBBoxBytes;
     }
     const int nh = g.r1 - g.r0 - sg * 16 > 8 ? 2 : 1;
+    int kbx = kb, rowx = 0;
+    if (op == OP_EXP_DOWN) {  // chunk kc = (slot, column chunk of that expert's down rows)
+      const int nd = moe_down_chunks(p);
+      kbx = (kc % nd) * (kBChunk / 64);
+      rowx = ctl->moe_uniq[kc / nd] * p.H;
+    }
     for (int h = 0; h < nh; ++h) {
       int row = g.r0 + sg * 16 + h * 8, m;
       if (op == OP_QKV) {
@@ -595,11 +684,11 @@ struct Cursor {
         m = row < qd ? 0 : (row < qd + kvd ? 1 : 2);
         row -= m == 0 ? 0 : (m == 1 ? qd : qd + kvd);
       } else {
-        m = op == OP_OPROJ ? 3 : 6;
+        m = op == OP_OPROJ ? 3 : (op == OP_ROUTER ? 7 : 6);
       }
       const uint8_t* map = op == OP_LMHEAD ? p.tmaps + (size_t)p.L * kTmapsPerLayer * 128
                                            : p.tmaps + ((size_t)layer * kTmapsPerLayer + m) * 128;
-      f(map, row, kb, (uint32_t)(h * kBBoxBytes));
+      f(map, row + rowx, kbx, (uint32_t)(h * kBBoxBytes));
     }
     return (uint32_t)nh * kBBoxBytes;
   }
@@ -615,8 +704,8 @@ struct Cursor {
 
   __device__ __forceinline__ uint32_t stage_bytes() const {
     if (op == OP_ATTN)
-      return pp->B > 1 ? (uint32_t)kStageBytes : (uint32_t)min(a.P, a.n_cached - sub * a.P) * pp->hd * 2u;
-    if (pp->B > 1) return (g.wup || g.r1 - g.r0 - sg * 16 > 8) ? 2u * kBBoxBytes : (uint32_t)kBBoxBytes;
+      return pp->tc ? (uint32_t)kStageBytes : (uint32_t)min(a.P, a.n_cached - sub * a.P) * pp->hd * 2u;
+    if (pp->tc) return (g.wup || g.r1 - g.r0 - sg * 16 > 8) ? 2u * kBBoxBytes : (uint32_t)kBBoxBytes;
     const uint32_t b = (uint32_t)min(g.tile.rows_per_stage, g.seg_rows(sg) - rr) * (uint32_t)g.Kc * 2u;
     return g.wup ? 2 * b : b;
   }
@@ -632,6 +721,24 @@ struct Producer {
   uint32_t k = 0;  // stages issued
 
   __device__ Producer(const Params& pp, Ctl* c, uint8_t* r) : p(pp), ctl(c), ring(r) { pol = evict_first_policy(); }
+
+  // MoE: wait (bounded) until the consumers have put layer `layer`'s routing in place.
+  __device__ __forceinline__ bool wait_routing(int layer) {
+    const uint64_t t0 = globaltimer();
+    uint32_t spins = 0;
+    while (*(const volatile int*)&ctl->moe_pub != layer + 1) {
+      if (*(volatile int*)&ctl->dead) return false;
+      if ((++spins & 63) == 0) {
+        if (ld_relaxed_i32(p.status) != 0) return false;
+        if (globaltimer() - t0 > p.timeout_ns) {
+          set_status(p, MK_ERR_DEVICE_TIMEOUT, -4);
+          return false;
+        }
+      }
+    }
+    __threadfence_block();
+    return true;
+  }
 
   // Claim the next slot (waiting until the consumers released it).
   __device__ __forceinline__ bool claim(uint8_t** dst, unsigned long long** bar) {
@@ -675,11 +782,17 @@ template <bool BATCHED>
 __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
   Producer<BATCHED> pr(p, ctl, ring);
   uint64_t* trace = p.trace ? p.trace + (size_t)p.offsets[blockIdx.x] * kTraceStamps : nullptr;
-  Cursor cur(p, list, n, &ctl->psched);
+  Cursor cur(p, list, n, &ctl->psched, ctl);
   cur.seek(0);
   bool ok = true;
   int last = -1;
   while (cur.i < n) {
+    if (cur.pending) {  // an expert instruction: its weights follow from the routing
+      if (!(ok = pr.wait_routing(cur.layer))) break;
+      cur.pending = false;
+      cur.seek(cur.i);
+      continue;
+    }
     if (trace && cur.i != last) {
       const uint64_t now = globaltimer();
       if (last >= 0) trace[last * kTraceStamps + 7] = now;
@@ -1019,13 +1132,19 @@ struct Consumer {
   // one chunk ahead.  RMSNorm: the gain is applied to the inputs, and the
   // per-sequence 1/rms factor, whose sum of squares accumulates from the same
   // loads, scales the outputs in the epilogue (it is constant along K).
+  //
+  // MoE: the router and the expert gate/up read the MLP input like gate/up;
+  // expert down runs K over the picked experts (slot after slot), its inputs
+  // being each slot's SwiGLU output times the sequence's routing weight.
+  // `slot` is the expert slot of a gate/up piece; wait_idx < 0: no wait.
   template <bool NORM, bool GATED>
-  __device__ __forceinline__ bool gemv_tc(const mk_instr& in, int op, int layer) {
+  __device__ __forceinline__ bool gemv_tc(const Gemv& g, int op, int layer, int wait_idx, int wait_count, int slot) {
     constexpr int TR = GATED ? 8 : 16;  // output rows per tile
     constexpr int MAXT = (GATED ? kBatchedMaxRowsGated : kBatchedMaxRows) / TR;
     constexpr int KPW = kBChunk / 16 / kConsumerWarps;  // k-steps per warp per chunk
-    const Gemv g = gemv_geo(p, in, op, layer);
     const int B = p.B, BH = B * p.H, nrows = g.r1 - g.r0, ntiles = g.bnt;
+    const bool moe_down = op == OP_EXP_DOWN;
+    const int nd = moe_down ? moe_down_chunks(p) : 1;
     const float* src;
     const uint16_t* gain = nullptr;
     int ld;  // elements per sequence in src
@@ -1033,18 +1152,27 @@ struct Consumer {
       src = p.xres + (size_t)(2 * layer) * BH, gain = p.layers[layer].attn_norm, ld = p.H;
     } else if (op == OP_OPROJ) {
       src = p.attn, ld = p.nq * p.hd;
-    } else if (op == OP_GATEUP) {
+    } else if (op == OP_GATEUP || op == OP_ROUTER || op == OP_EXP_GATEUP) {
       src = p.xres + (size_t)(2 * layer + 1) * BH, gain = p.layers[layer].mlp_norm, ld = p.H;
     } else if (op == OP_DOWN) {
       src = p.act, ld = p.I;
+    } else if (moe_down) {
+      src = p.moe_act, ld = p.Ie;  // slot s, sequence b at (s * B + b) * Ie
     } else {
       src = p.xres + (size_t)(2 * p.L) * BH, gain = p.final_norm, ld = p.H;
     }
-    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
-    if (tr) tr[1] = globaltimer();
+    if (wait_idx >= 0) {
+      if (!wait_counter(wait_idx, wait_count)) return false;
+      if (tr) tr[1] = globaltimer();
+    }
     const int gq = lane >> 2, cq = lane & 3;
     const bool bval = gq < B;  // this lane's B-fragment column (sequence gq) exists
     const float* xrow = src + (size_t)(bval ? gq : 0) * ld;
+    // columns of chunk j, and where its inputs start
+    auto cols = [&](int j) { return moe_down ? min(kBChunk, p.Ie - (j % nd) * kBChunk) : min(kBChunk, g.K - j * kBChunk); };
+    auto xbase = [&](int j) {
+      return moe_down ? xrow + (size_t)(j / nd) * B * p.Ie + (j % nd) * kBChunk : xrow + (size_t)j * kBChunk;
+    };
     float acc[MAXT][4];
 #pragma unroll
     for (int t2 = 0; t2 < MAXT; ++t2) acc[t2][0] = acc[t2][1] = acc[t2][2] = acc[t2][3] = 0.f;
@@ -1054,14 +1182,15 @@ struct Consumer {
     uint32_t xf[KPW][2];
     // raw inputs (and gains) of chunk j: k = 16 ks + 2 cq (+1) and + 8 (+1)
     auto load = [&](int j) {
-      const int nks = min(kBChunk, g.K - j * kBChunk) / 16;
+      const int nks = cols(j) / 16;
+      const float* xb = xbase(j);
 #pragma unroll
       for (int kk = 0; kk < KPW; ++kk) {
         const int ks = warp + kk * kConsumerWarps;
-        const int k = j * kBChunk + ks * 16 + 2 * cq;
+        const int kl = ks * 16 + 2 * cq, k = j * kBChunk + kl;
         if (bval && ks < nks) {
-          xr[kk][0] = __ldcg(reinterpret_cast<const float2*>(xrow + k));
-          xr[kk][1] = __ldcg(reinterpret_cast<const float2*>(xrow + k + 8));
+          xr[kk][0] = __ldcg(reinterpret_cast<const float2*>(xb + kl));
+          xr[kk][1] = __ldcg(reinterpret_cast<const float2*>(xb + kl + 8));
           if (NORM) {
             gr[kk][0] = __ldg(reinterpret_cast<const unsigned int*>(gain + k));
             gr[kk][1] = __ldg(reinterpret_cast<const unsigned int*>(gain + k + 8));
@@ -1081,7 +1210,9 @@ struct Consumer {
     const uint32_t lrow = (uint32_t)((lane >> 3) & 1) * kBBoxBytes + (uint32_t)(warp >> 2) * 1024u + rr7 * 128u +
                           ((ch ^ rr7) << 4);
     for (int j = 0; j < g.bnch; ++j) {
-      const int nks = min(kBChunk, g.K - j * kBChunk) / 16;
+      const int nks = cols(j) / 16;
+      // expert down: the sequence's routing weight of this chunk's slot (0 if not picked)
+      const float rw = moe_down && bval ? ctl->moe_tw[j / nd][gq] : 1.f;
 #pragma unroll
       for (int kk = 0; kk < KPW; ++kk) {
 #pragma unroll
@@ -1091,7 +1222,7 @@ struct Consumer {
             ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
             xf[kk][h] = pack_bf16x2(x.x * bf16_lo(gr[kk][h]), x.y * bf16_hi(gr[kk][h]));
           } else {
-            xf[kk][h] = pack_bf16x2(x.x, x.y);
+            xf[kk][h] = pack_bf16x2(x.x * rw, x.y * rw);
           }
         }
       }
@@ -1156,7 +1287,13 @@ struct Consumer {
           v1 *= sc;
           if (GATED) {
             const int row = tile * TR + lgq;  // v0 = gate, v1 = up of neuron row
-            if (row < nrows) p.act[(size_t)b * p.I + g.r0 + row] = v0 / (1.f + expf(-v0)) * v1;
+            if (row < nrows) {
+              const float a = v0 / (1.f + expf(-v0)) * v1;
+              if (op == OP_EXP_GATEUP)
+                p.moe_act[((size_t)slot * B + b) * p.Ie + (g.r0 - ctl->moe_uniq[slot] * p.Ie) + row] = a;
+              else
+                p.act[(size_t)b * p.I + g.r0 + row] = a;
+            }
           } else {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -1169,9 +1306,11 @@ struct Consumer {
                 } else if (op == OP_OPROJ) {
                   const size_t o = (size_t)b * p.H + row;
                   p.xres[(size_t)(2 * layer + 1) * BH + o] = __ldcg(p.xres + (size_t)(2 * layer) * BH + o) + y;
-                } else if (op == OP_DOWN) {
+                } else if (op == OP_DOWN || moe_down) {
                   const size_t o = (size_t)b * p.H + row;
                   p.xres[(size_t)(2 * layer + 2) * BH + o] = __ldcg(p.xres + (size_t)(2 * layer + 1) * BH + o) + y;
+                } else if (op == OP_ROUTER) {
+                  p.moe_router[((size_t)layer * B + b) * p.E + row] = y;
                 } else {
                   p.logits[(size_t)b * p.V + row] = y;
                 }
@@ -1186,9 +1325,12 @@ struct Consumer {
 
   __device__ __forceinline__ bool gemv(const mk_instr& in, int op, int layer) {
     if constexpr (BATCHED) {
-      if (op == OP_GATEUP) return gemv_tc<true, true>(in, op, layer);
-      if (op == OP_QKV || op == OP_LMHEAD) return gemv_tc<true, false>(in, op, layer);
-      return gemv_tc<false, false>(in, op, layer);
+      Gemv g = gemv_geo(p, in, op, layer);
+      if (op == OP_EXP_DOWN) g.bnch = ctl->moe_count * moe_down_chunks(p);  // routing of this layer, in place
+      if (op == OP_GATEUP) return gemv_tc<true, true>(g, op, layer, in.wait_idx, in.wait_count, -1);
+      if (op == OP_QKV || op == OP_LMHEAD || op == OP_ROUTER)
+        return gemv_tc<true, false>(g, op, layer, in.wait_idx, in.wait_count, -1);
+      return gemv_tc<false, false>(g, op, layer, in.wait_idx, in.wait_count, -1);
     }
     const bool norm = op == OP_QKV || op == OP_GATEUP || op == OP_LMHEAD;
     const int K = op == OP_OPROJ ? p.nq * p.hd : (op == OP_DOWN ? p.I : p.H);
@@ -1198,6 +1340,112 @@ struct Consumer {
     if (op == OP_GATEUP) return gemv_nvsel<true, true>(in, op, layer, tl.nv, rpt);
     if (norm) return gemv_nvsel<true, false>(in, op, layer, tl.nv, rpt);
     return gemv_nvsel<false, false>(in, op, layer, tl.nv, rpt);
+  }
+
+  // ---- MoE routing ---------------------------------------------------------------
+  // Top-k of each sequence's router logits (the larger logit first, a tie to
+  // the lower expert index; Shazeer et al. 2017, sparsely-gated mixture of
+  // experts), weights = softmax over the k picked logits, and the distinct
+  // picked experts in ascending order as slots.  Every SM computes the same
+  // routing from the same logits; the SM of slot instruction 0 writes it out.
+  __device__ __forceinline__ void moe_select(int layer, bool dump) {
+    const int E = p.E, K = p.topk, B = p.B;
+    if (t < kMaxExperts / 32) ctl->moe_mask[t] = 0u;
+    for (int i = t; i < kMaxSel * kMaxBatch; i += kConsumerThreads) (&ctl->moe_tw[0][0])[i] = 0.f;
+    consumer_bar();
+    int pick = 0;    // lane j < K of warp b < B: the j-th pick of sequence b
+    float pw = 0.f;  // and its weight
+    if (warp < B) {
+      const float* r = p.moe_router + ((size_t)layer * B + warp) * E;
+      float v[kMaxExperts / 32];
+#pragma unroll
+      for (int q = 0; q < kMaxExperts / 32; ++q) {
+        const int e = lane + 32 * q;
+        const float x = e < E ? __ldcg(r + e) : -INFINITY;
+        v[q] = x != x ? -INFINITY : x;  // NaN ranks below every number
+      }
+      uint32_t taken = 0u;
+      float top0 = 0.f, den = 0.f, mine = 0.f;
+      for (int j = 0; j < K; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < kMaxExperts / 32; ++q) {
+          const int e = lane + 32 * q;
+          if (e < E && !((taken >> q) & 1u) && (v[q] > bv || (v[q] == bv && e < bi))) {
+            bv = v[q];
+            bi = e;
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (j == 0) top0 = bv;
+        const float ex = expf(bv - top0);
+        den += ex;
+        if (lane == j) {
+          pick = bi;
+          mine = ex;
+        }
+      }
+      if (lane < K) {
+        pw = mine / den;
+        atomicOr(&ctl->moe_mask[pick >> 5], 1u << (pick & 31));
+        if (dump) {
+          p.moe_sel[((size_t)layer * B + warp) * K + lane] = pick;
+          p.moe_selw[((size_t)layer * B + warp) * K + lane] = pw;
+        }
+      }
+    }
+    consumer_bar();
+    // slot of a picked expert: the picked experts below it
+    auto slot_of = [&](int e) {
+      int sl = 0;
+      for (int w = 0; w < (e >> 5); ++w) sl += __popc(ctl->moe_mask[w]);
+      return sl + __popc(ctl->moe_mask[e >> 5] & ((1u << (e & 31)) - 1u));
+    };
+    if (t < E && ((ctl->moe_mask[t >> 5] >> (t & 31)) & 1u)) ctl->moe_uniq[slot_of(t)] = (int16_t)t;
+    if (t == 0) {
+      int c = 0;
+      for (int w = 0; w < kMaxExperts / 32; ++w) c += __popc(ctl->moe_mask[w]);
+      ctl->moe_count = c;
+      if (dump) p.moe_count[layer] = c;
+    }
+    if (warp < B && lane < K) ctl->moe_tw[slot_of(pick)][warp] = pw;
+    consumer_bar();
+    if (t == 0) {  // hand the routing to the producer
+      __threadfence_block();
+      *(volatile int*)&ctl->moe_pub = layer + 1;
+    }
+  }
+
+  // One expert gate/up slot: wait for the router, route, then this slot's
+  // even share of the (picked expert, 8-neuron tile) units, piece by piece.
+  __device__ __forceinline__ bool moe_gateup(const mk_instr& in, int layer) {
+    if constexpr (BATCHED) {
+      if (!wait_counter(in.wait_idx, in.wait_count)) return false;
+      if (tr) tr[1] = globaltimer();
+      moe_select(layer, in.a == 0);
+      const int64_t U = (int64_t)ctl->moe_count * (p.Ie / 8);
+      const int64_t g1 = even_begin(U, in.b, in.a + 1);
+      for (int64_t g = even_begin(U, in.b, in.a); g < g1;) {
+        int sl;
+        const Gemv gm = moe_gate_piece(p, ctl, layer, g, g1, &sl);
+        if (!gemv_tc<true, true>(gm, OP_EXP_GATEUP, layer, -1, 0, sl)) return false;
+        g += gm.bnt;
+        consumer_bar();  // the reduction buffer is free for the next piece
+      }
+      return true;
+    } else {
+      return false;  // MoE runs on the tensor-core kernel only
+    }
   }
 
   // ---- attention ---------------------------------------------------------------
@@ -1748,7 +1996,16 @@ __device__ __forceinline__ void run_consumers(const Params& p, const mk_instr* l
       case OP_GATEUP:
       case OP_DOWN:
       case OP_LMHEAD:
+      case OP_ROUTER:
+      case OP_EXP_DOWN:
         ok = cs.gemv(in, op, layer);  // waits on the instruction's counter inside
+        if (ok) {
+          if (trace) trace[i * kTraceStamps + 2] = globaltimer();
+          cs.signal(in.sig_idx);
+        }
+        break;
+      case OP_EXP_GATEUP:
+        ok = cs.moe_gateup(in, layer);
         if (ok) {
           if (trace) trace[i * kTraceStamps + 2] = globaltimer();
           cs.signal(in.sig_idx);
@@ -1784,6 +2041,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
     }
     ctl->dead = 0;
     ctl->last = 0;
+    ctl->moe_pub = 0;
     // a sticky error from an earlier step, or out-of-range inputs: do nothing
     int bad = ld_relaxed_i32(p.status) != 0;
     for (int b = 0; b < p.B && !bad; ++b) {
@@ -1835,7 +2093,7 @@ cudaError_t kernel_occupancy(int* blocks_per_sm, bool batched) {
 
 cudaError_t launch_step(const Params& p, int n_blocks, cudaStream_t stream) {
   void* args[] = {const_cast<Params*>(&p)};
-  if (p.B > 1)
+  if (p.tc)
     return cudaLaunchCooperativeKernel((const void*)mk_persistent<true>, dim3(n_blocks), dim3(kThreads), args,
                                        Smem<true>::kTotal, stream);
   return cudaLaunchCooperativeKernel((const void*)mk_persistent<false>, dim3(n_blocks), dim3(kThreads), args,

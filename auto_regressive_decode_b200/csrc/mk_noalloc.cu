@@ -89,6 +89,7 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
     for (const void* q : need)
       if (!aligned16(q)) return q ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
     if (d.qk_norm && (!aligned16(lw.q_norm) || !aligned16(lw.k_norm))) return MK_ERR_INVALID_ARG;
+    if (d.n_experts && !aligned16(lw.router)) return lw.router ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
   }
 
   int dev = 0, n_sm = 0, coop = 0, smem_optin = 0, per_sm = 0;
@@ -99,9 +100,9 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-      mk::kernel_occupancy(&per_sm, d.batch > 1) != cudaSuccess)
+      mk::kernel_occupancy(&per_sm, mk::batched(d)) != cudaSuccess)
     return MK_ERR_CUDA;
-  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes(d.batch > 1) || per_sm < 1) return MK_ERR_UNSUPPORTED;
+  if (!coop || (size_t)smem_optin < mk::kernel_smem_bytes(mk::batched(d)) || per_sm < 1) return MK_ERR_UNSUPPORTED;
 
   mk_plan* plan = nullptr;
   rc = mk_plan_create(desc, n_sm, &plan);
@@ -133,14 +134,20 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   const size_t o_xres = take(sizeof(float) * (size_t)(2 * L + 1) * B * H);
   const size_t o_qkv = take(sizeof(float) * (size_t)B * (qd + 2 * kvd));
   const size_t o_attn = take(sizeof(float) * (size_t)B * qd);
-  const size_t o_act = take(sizeof(float) * (size_t)B * d.ffn_dim);
+  const size_t o_act = take(sizeof(float) * (size_t)B * (d.n_experts ? 1 : d.ffn_dim));
+  const int E = d.n_experts, K = d.top_k;
+  const size_t o_mr = E ? take(sizeof(float) * (size_t)L * B * E) : 0;
+  const size_t o_ms = E ? take(sizeof(int32_t) * (size_t)L * B * K) : 0;
+  const size_t o_mw = E ? take(sizeof(float) * (size_t)L * B * K) : 0;
+  const size_t o_mc = E ? take(sizeof(int32_t) * (size_t)L) : 0;
+  const size_t o_ma = E ? take(sizeof(float) * (size_t)mk::moe_slots(E, B, K) * B * d.expert_ffn_dim) : 0;
   const size_t o_po = take(sizeof(float) * (size_t)B * nq * n_chunks * hd);
   const size_t o_pml = take(sizeof(float) * (size_t)B * nq * n_chunks * 2);
   const size_t o_ins = take(sizeof(mk_instr) * instrs.size());
   const size_t o_off = take(sizeof(int32_t) * offsets.size());
   const size_t o_lay = take(sizeof(mk::LayerPtrs) * (size_t)L);
   const size_t o_rope = take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
-  const size_t n_tmaps = B > 1 ? (size_t)mk::kTmapsPerLayer * L + 3 : 0;  // batch > 1: TMA tensor maps
+  const size_t n_tmaps = mk::batched(d) ? (size_t)mk::kTmapsPerLayer * L + 3 : 0;  // batch > 1: TMA tensor maps
   const size_t o_tmap = n_tmaps ? take(128 * n_tmaps) : 0;
   if (off > kStaticScratchBytes) return MK_ERR_UNSUPPORTED;  // model needs more than the 8 MiB array
   std::vector<uint8_t> tmaps(128 * n_tmaps);
@@ -188,6 +195,7 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   p.I = d.ffn_dim;
   p.V = d.vocab;
   p.B = B;
+  p.tc = mk::batched(d);
   p.T = d.max_ctx;
   p.qk_norm = d.qk_norm;
   p.eps = d.rms_eps;
@@ -207,6 +215,16 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   p.act = (float*)(base + o_act);
   p.part_o = (float*)(base + o_po);
   p.part_ml = (float*)(base + o_pml);
+  if (E) {
+    p.E = E;
+    p.topk = K;
+    p.Ie = d.expert_ffn_dim;
+    p.moe_router = (float*)(base + o_mr);
+    p.moe_sel = (int32_t*)(base + o_ms);
+    p.moe_selw = (float*)(base + o_mw);
+    p.moe_count = (int32_t*)(base + o_mc);
+    p.moe_act = (float*)(base + o_ma);
+  }
   p.counters = (uint32_t*)(base + o_cnt);
   p.tickets = (uint32_t*)(base + o_tk);
   p.status = (int*)(base + o_st);

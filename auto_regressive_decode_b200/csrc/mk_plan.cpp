@@ -48,15 +48,23 @@ int validate_desc(const mk_model_desc* d) {
   if (g != 1 && g != 2 && g != 4 && g != 8) return MK_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128) return MK_ERR_UNSUPPORTED;
   if (d->batch > kMaxBatch) return MK_ERR_UNSUPPORTED;
-  if (d->n_experts) return MK_ERR_UNSUPPORTED;   // MoE lowering not built yet
-  if (d->ffn_dim <= 0) return MK_ERR_INVALID_ARG;
   const int qd = d->n_q_heads * d->head_dim;
-  if (!aligned_ok(d->hidden, 1) || !aligned_ok(d->hidden, 2) || !aligned_ok(qd, 1) || !aligned_ok(d->ffn_dim, 1))
-    return MK_ERR_UNSUPPORTED;
+  if (d->n_experts) {
+    // MoE runs on the tensor-core kernel at any batch size
+    if (d->top_k <= 0 || d->top_k > d->n_experts || d->expert_ffn_dim <= 0) return MK_ERR_INVALID_ARG;
+    if (d->n_experts > kMaxExperts || d->top_k > kMaxTopK || d->batch * d->top_k > kMaxSel) return MK_ERR_UNSUPPORTED;
+    const int ks[3] = {d->hidden, qd, d->expert_ffn_dim};
+    for (int K : ks)
+      if (K % 64) return MK_ERR_UNSUPPORTED;
+  } else {
+    if (d->ffn_dim <= 0) return MK_ERR_INVALID_ARG;
+    if (!aligned_ok(d->ffn_dim, 1)) return MK_ERR_UNSUPPORTED;
+  }
+  if (!aligned_ok(d->hidden, 1) || !aligned_ok(d->hidden, 2) || !aligned_ok(qd, 1)) return MK_ERR_UNSUPPORTED;
   // GEMVs with an RMSNorm prologue (K = hidden) read whole rows in one pass
   if (gemv_ksplit(d->hidden, 1) != 1 || gemv_ksplit(d->hidden, 2) != 1) return MK_ERR_UNSUPPORTED;
   if ((int64_t)d->max_ctx * d->head_dim > (1ll << 31)) return MK_ERR_UNSUPPORTED;
-  if (d->batch > 1) {
+  if (d->batch > 1 && !d->n_experts) {
     // tensor-core GEMVs: the weight tensor maps view K as blocks of 64 columns
     const int ks[3] = {d->hidden, qd, d->ffn_dim};
     for (int K : ks)
@@ -89,10 +97,10 @@ struct Builder {
     int n = 0;
     const int n_sm = p->n_sm;
     const int max_rows =
-        p->d.batch > 1 ? (op == OP_GATEUP ? kBatchedMaxRowsGated : kBatchedMaxRows) : kMaxRows;
+        batched(p->d) ? (op == OP_GATEUP ? kBatchedMaxRowsGated : kBatchedMaxRows) : kMaxRows;
     // batch > 1: row ranges start at multiples of kBBoxRows (a TMA box
     // never reaches into another SM's rows or across wq | wk | wv)
-    const int unit = p->d.batch > 1 ? kBBoxRows : 1;
+    const int unit = batched(p->d) ? kBBoxRows : 1;
     const int64_t NU = (N + unit - 1) / unit;
     for (int s = 0; s < n_sm; ++s) {
       int r0 = (int)std::min<int64_t>(N, NU * s / n_sm * unit);
@@ -160,6 +168,20 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
     p->targets[ca] = d->batch * d->n_kv_heads * nhg;  // one bump per merged (sequence, KV head, head group)
     int n_o = b.rows_op(OP_OPROJ, l, H, {}, ca, p->targets[ca], co);
     p->targets[co] = n_o;
+    if (d->n_experts) {
+      // router rows; one expert gate/up slot per SM; down by output rows
+      const int cr = counter_index(l, C_ROUTER), ceg = counter_index(l, C_EXP_GATEUP);
+      const int ced = counter_index(l, C_EXP_DOWN);
+      int n_r = b.rows_op(OP_ROUTER, l, d->n_experts, {}, co, n_o, cr);
+      p->targets[cr] = n_r;
+      for (int s = 0; s < n_sm; ++s) b.emit(s, OP_EXP_GATEUP, l, cr, n_r, ceg, s, n_sm, 0, 0);
+      p->targets[ceg] = n_sm;
+      int n_ed = b.rows_op(OP_EXP_DOWN, l, H, {}, ceg, n_sm, ced);
+      p->targets[ced] = n_ed;
+      prev_idx = ced;
+      prev_count = n_ed;
+      continue;
+    }
     int n_gu = b.rows_op(OP_GATEUP, l, d->ffn_dim, {}, co, n_o, cg);
     p->targets[cg] = n_gu;
     int n_dn = b.rows_op(OP_DOWN, l, H, {}, cg, n_gu, cd);

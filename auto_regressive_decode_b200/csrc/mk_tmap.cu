@@ -58,14 +58,19 @@ bool encode_one(EncodeTiledFn enc, const void* w, int64_t rows, int K, uint8_t* 
 cudaError_t encode_tmaps(const mk_model_desc& d, const mk_weights& w, const mk_kv& kv, uint8_t* out) {
   EncodeTiledFn enc = encoder();
   if (!enc) return cudaErrorNotSupported;
-  const int H = d.hidden, qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim, I = d.ffn_dim;
+  const int H = d.hidden, qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim;
+  // MoE: the experts' matrices are stacked, [E][Ie][H] for gate and up and
+  // [E][H][Ie] for down, and read as one tall matrix each
+  const int E = d.n_experts, I = E ? d.expert_ffn_dim : d.ffn_dim;
+  const int64_t gu_rows = E ? (int64_t)E * I : I, dn_rows = E ? (int64_t)E * H : H;
+  memset(out, 0, (size_t)(kTmapsPerLayer * d.n_layers + 3) * 128);
   for (int l = 0; l < d.n_layers; ++l) {
     const mk_layer_weights& lw = w.layers[l];
     uint8_t* o = out + (size_t)l * kTmapsPerLayer * 128;
     const bool ok = encode_one(enc, lw.wq, qd, H, o) && encode_one(enc, lw.wk, kvd, H, o + 128) &&
                     encode_one(enc, lw.wv, kvd, H, o + 256) && encode_one(enc, lw.wo, H, qd, o + 384) &&
-                    encode_one(enc, lw.w_gate, I, H, o + 512) && encode_one(enc, lw.w_up, I, H, o + 640) &&
-                    encode_one(enc, lw.w_down, H, I, o + 768);
+                    encode_one(enc, lw.w_gate, gu_rows, H, o + 512) && encode_one(enc, lw.w_up, gu_rows, H, o + 640) &&
+                    encode_one(enc, lw.w_down, dn_rows, I, o + 768) && (!E || encode_one(enc, lw.router, E, H, o + 896));
     if (!ok) return cudaErrorInvalidValue;
   }
   const void* lm = d.tied_embeddings ? w.embed : w.lm_head;

@@ -239,6 +239,18 @@ class Decoder:
         out = self.torch.empty((2 * c.n_layers + 1, c.batch, c.hidden), dtype=self.torch.float32, device="cuda")
         return self.read_state(MK_STATE_HIDDEN, out)
 
+    def routing(self):
+        """MoE routing of the last step (host numpy): router logits float32 [L][B][E], picks int32
+        [L][B][k] (best first), their weights float32 [L][B][k], distinct experts int32 [L]."""
+        c, torch = self.cfg, self.torch
+        L, B, E, K = c.n_layers, c.batch, c.n_experts, c.top_k
+        r = self.read_state(MK_STATE_ROUTER, torch.empty((L, B, E), dtype=torch.float32, device="cuda"))
+        sel = self.read_state(MK_STATE_SELECTION, torch.empty((L, B, K), dtype=torch.int32, device="cuda"))
+        w = self.read_state(MK_STATE_SEL_WEIGHT, torch.empty((L, B, K), dtype=torch.float32, device="cuda"))
+        n = self.read_state(MK_STATE_EXPERT_COUNT, torch.empty((L,), dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        return r.cpu().numpy(), sel.cpu().numpy(), w.cpu().numpy(), n.cpu().numpy()
+
     def close(self):
         if getattr(self, "h", None):
             mk_destroy(self.h)

@@ -10,6 +10,13 @@ closer than the bf16 rounding of the activations moves a logit.  A step agrees
 when the GPU's pick is a top-1 token of the oracle up to TOP1_TIE: its oracle
 logit is within TOP1_TIE of the oracle's maximum.  The exact-argmax rate is
 recorded beside it ("top1_exact").
+
+MoE selection reading ("bit-exact" selection): (i) the GPU's picks and their
+order equal the oracle's top-k applied to the GPU's own router logits, for
+every (layer, sequence); (ii) the GPU's router logits match the oracle's
+within the hidden-state tolerance; (iii) the end-to-end pick sets agree
+except where the oracle's k-th and (k+1)-th logits are closer than twice the
+measured router-logit error (a near-tie either side may resolve).
 """
 from __future__ import annotations
 
@@ -50,7 +57,8 @@ def run_teacher_forced(cfg, steps=None, gains="ones", seed=fx.DEFAULT_SEED, seq_
                       expert_loader(cfg, seed) if cfg.n_experts else None)
     B, L = cfg.batch, cfg.n_layers
     logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
-    res = {"hidden": [], "logits_abs": [], "kv": [], "top1": [], "top1_exact": [], "status": []}
+    res = {"hidden": [], "logits_abs": [], "kv": [], "top1": [], "top1_exact": [], "status": [],
+           "router": [], "sel_own": [], "sel_w": [], "sel_e2e": [], "sel_e2e_unexplained": 0, "count_ok": []}
     for t in range(steps):
         S = (S0 + t).astype(np.int32)
         tok = toks[t % toks.shape[0]]
@@ -74,6 +82,8 @@ def run_teacher_forced(cfg, steps=None, gains="ones", seed=fx.DEFAULT_SEED, seq_
             gv = bf16_f64(bits(vc[:, b, :, S[b]].contiguous()))
             kv_err = max(kv_err, rel_l2(gk, bf16_f64(okc[:, b, :, S[b]])), rel_l2(gv, bf16_f64(ovc[:, b, :, S[b]])))
         res["kv"].append(kv_err)
+        if cfg.n_experts:
+            check_routing(res, dec.routing(), ref, cfg)
         res["top1"].extend(top1_agree(lg, ref["logits"]))
         res["top1_exact"].extend(list(np.argmax(lg, axis=1) == np.argmax(ref["logits"], axis=1)))
     # cache bytes other than the appended rows are untouched
@@ -94,6 +104,26 @@ def top1_agree(gpu_logits: np.ndarray, ref_logits: np.ndarray) -> list:
     return list(got >= ref_logits.max(axis=1) - TOP1_TIE)
 
 
+def check_routing(res, gpu, ref, cfg):
+    """Record the MoE selection checks (i)-(iii) of one step."""
+    r, sel, w, n = gpu
+    K = cfg.top_k
+    for l in range(cfg.n_layers):
+        res["router"].append(rel_l2(r[l].astype(np.float64), ref["router_logits"][l]))
+        res["count_ok"].append(int(n[l]) == len(np.unique(sel[l])))
+        for b in range(cfg.batch):
+            own, own_w = ora.topk(r[l, b].astype(np.float64), K)
+            res["sel_own"].append(bool(np.array_equal(sel[l, b], own)))
+            res["sel_w"].append(float(np.max(np.abs(w[l, b] - own_w))))
+            same = set(sel[l, b].tolist()) == set(ref["sel"][l, b].tolist())
+            res["sel_e2e"].append(same)
+            if not same:
+                srt = np.sort(ref["router_logits"][l, b])[::-1]
+                err = float(np.max(np.abs(r[l, b] - ref["router_logits"][l, b])))
+                if K < srt.size and srt[K - 1] - srt[K] >= 2 * err:
+                    res["sel_e2e_unexplained"] += 1
+
+
 def assert_parity(res):
     assert all(s == 0 for s in res["status"]), res["status"]
     assert max(res["hidden"]) <= TOL_HIDDEN, res["hidden"]
@@ -101,3 +131,9 @@ def assert_parity(res):
     assert max(res["kv"]) <= TOL_KV, res["kv"]
     assert np.mean(res["top1"]) >= MIN_TOP1, np.mean(res["top1"])
     assert res["untouched_ok"]
+    if res["router"]:
+        assert max(res["router"]) <= TOL_HIDDEN, max(res["router"])
+        assert all(res["sel_own"]), res["sel_own"].count(False)
+        assert max(res["sel_w"]) <= 1e-5, max(res["sel_w"])
+        assert all(res["count_ok"])
+        assert res["sel_e2e_unexplained"] == 0, res["sel_e2e_unexplained"]

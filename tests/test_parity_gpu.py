@@ -71,3 +71,18 @@ def test_batched_multi_chunk():
     cfg = fx.ModelConfig("mid-b8", n_layers=3, hidden=640, n_q_heads=5, n_kv_heads=5, head_dim=128, ffn_dim=4608,
                          vocab=2000, batch=8, ctx_lo=10, ctx_hi=300, steps=3)
     assert_parity(run_teacher_forced(cfg, gains="random"))
+
+
+# ---- mixture of experts (tensor-core kernel at any batch size) -------------------------------------
+
+@pytest.mark.parametrize("kw,gains", [
+    ({"n_experts": 8, "top_k": 2, "expert_ffn_dim": 128, "batch": 4, "ctx": 0, "ctx_lo": 3, "ctx_hi": 120}, "random"),
+    ({"n_experts": 16, "top_k": 4, "expert_ffn_dim": 64, "batch": 1}, "ones"),                      # MoE at batch 1
+    ({"n_experts": 32, "top_k": 8, "expert_ffn_dim": 64, "batch": 8, "ctx": 0, "ctx_lo": 0, "ctx_hi": 60}, "random"),
+    ({"n_experts": 256, "top_k": 8, "expert_ffn_dim": 1088, "batch": 3, "n_layers": 1}, "random"),   # ragged Ie chunk
+])
+def test_tiny_moe(kw, gains):
+    cfg = fx.CONFIGS["tiny"].replace(ffn_dim=0, **kw)
+    res = run_teacher_forced(cfg, steps=3, gains=gains)
+    assert_parity(res)
+    assert len(res["sel_own"]) == 3 * cfg.n_layers * cfg.batch

@@ -16,9 +16,12 @@ import fixtures as fx
 mk = pytest.importorskip("auto_regressive_decode_b200.mk")
 
 OP_EMBED, OP_QKV, OP_ATTN, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LMHEAD = 1, 2, 3, 4, 5, 6, 7
-ORDER = {OP_EMBED: 0, OP_QKV: 1, OP_ATTN: 2, OP_OPROJ: 3, OP_GATEUP: 4, OP_DOWN: 5, OP_LMHEAD: 6}
+OP_ROUTER, OP_EXP_GATEUP, OP_EXP_DOWN = 8, 9, 10
+ORDER = {OP_EMBED: 0, OP_QKV: 1, OP_ATTN: 2, OP_OPROJ: 3, OP_GATEUP: 4, OP_DOWN: 5, OP_LMHEAD: 6,
+         OP_ROUTER: 4, OP_EXP_GATEUP: 4.5, OP_EXP_DOWN: 5}
 
-CASES = [("tiny", 148), ("tiny", 7), ("tiny", 1), ("dense-0.6b", 148), ("dense-8b", 148), ("dense-8b", 132)]
+CASES = [("tiny", 148), ("tiny", 7), ("tiny", 1), ("dense-0.6b", 148), ("dense-8b", 148), ("dense-8b", 132),
+         ("moe-128x8", 148), ("moe-128x8", 5)]
 
 
 def plan_of(name, n_sm, **kw):
@@ -28,7 +31,7 @@ def plan_of(name, n_sm, **kw):
 
 def rows_of(cfg, op):
     return {OP_QKV: cfg.q_dim + 2 * cfg.kv_dim, OP_OPROJ: cfg.hidden, OP_GATEUP: cfg.ffn_dim, OP_DOWN: cfg.hidden,
-            OP_LMHEAD: cfg.vocab, OP_EMBED: cfg.hidden}[op]
+            OP_LMHEAD: cfg.vocab, OP_EMBED: cfg.hidden, OP_ROUTER: cfg.n_experts, OP_EXP_DOWN: cfg.hidden}[op]
 
 
 @pytest.mark.parametrize("name,n_sm", CASES)
@@ -36,14 +39,18 @@ def test_rows_and_chunks_covered_once(name, n_sm):
     cfg, p = plan_of(name, n_sm)
     cover = collections.defaultdict(list)
     attn = collections.Counter()
+    slots = collections.Counter()
     for row in p.instrs:
         op, layer = p.op(row), p.layer(row)
         if op == OP_ATTN:
             attn[(layer, int(row[4]))] += 1
             assert int(row[5]) == n_sm
+        elif op == OP_EXP_GATEUP:
+            slots[(layer, int(row[4]))] += 1
+            assert int(row[5]) == n_sm
         else:
             cover[(layer, op)].append((int(row[4]), int(row[5])))
-            assert 0 < row[5] - row[4] <= 256
+            assert 0 < row[5] - row[4] and (op == OP_EMBED or row[5] - row[4] <= 256)
     for (layer, op), segs in cover.items():
         segs.sort()
         assert segs[0][0] == 0 and segs[-1][1] == rows_of(cfg, op)
@@ -54,6 +61,9 @@ def test_rows_and_chunks_covered_once(name, n_sm):
     for s in range(n_sm):
         assert all(int(r[4]) == s for r in p.sm_list(s) if p.op(r) == OP_ATTN)
     assert p.chunk == 32768 // (2 * cfg.head_dim) and p.n_chunks == n_sm
+    # MoE: one expert gate/up slot per SM per layer
+    assert set(slots) == ({(l, s) for l in range(cfg.n_layers) for s in range(n_sm)} if cfg.n_experts else set())
+    assert set(slots.values()) <= {1}
 
 
 @pytest.mark.parametrize("name,n_sm", CASES)
@@ -130,7 +140,7 @@ def simulate(p, cfg, order_seed=0, seq_lens=None):
 
 
 @pytest.mark.parametrize("name,n_sm", [("tiny", 148), ("tiny", 3), ("dense-0.6b", 148), ("dense-8b", 148),
-                                       ("dense-13b-b8", 148)])
+                                       ("dense-13b-b8", 148), ("moe-128x8", 148), ("moe-128x8", 3)])
 def test_counter_protocol_completes(name, n_sm):
     cfg, p = plan_of(name, n_sm)
     for seed in range(2):
@@ -258,3 +268,36 @@ def test_attention_schedule_rejects_out_of_range_lengths():
     cfg, p = plan_of("tiny", 148)
     with pytest.raises(mk.MkError):
         p.attn_pieces([cfg.max_ctx])
+
+
+def test_moe_lowering_edges_and_targets():
+    # per layer: ... o_proj -> router rows -> one expert gate/up slot per SM -> expert down rows -> next qkv
+    cfg, p = plan_of("moe-128x8", 148)
+    kinds = collections.defaultdict(list)
+    for r in p.instrs:
+        kinds[(p.layer(r), p.op(r))].append(r)
+    assert not any(op in (OP_GATEUP, OP_DOWN) for (_, op) in kinds)
+    sig = {}
+    for (l, op), rows in kinds.items():
+        assert len({int(r[3]) for r in rows}) == 1
+        sig[(l, op)] = int(rows[0][3])
+    for l in range(cfg.n_layers):
+        router, slots, down = kinds[(l, OP_ROUTER)], kinds[(l, OP_EXP_GATEUP)], kinds[(l, OP_EXP_DOWN)]
+        assert sum(int(r[5]) - int(r[4]) for r in router) == cfg.n_experts
+        assert sum(int(r[5]) - int(r[4]) for r in down) == cfg.hidden
+        assert len(slots) == 148 and p.targets[sig[(l, OP_EXP_GATEUP)]] == 148
+        assert all(int(r[1]) == sig[(l, OP_OPROJ)] for r in router)
+        assert all(int(r[1]) == sig[(l, OP_ROUTER)] and int(r[2]) == len(router) for r in slots)
+        assert all(int(r[1]) == sig[(l, OP_EXP_GATEUP)] and int(r[2]) == 148 for r in down)
+        if l + 1 < cfg.n_layers:
+            assert all(int(r[1]) == sig[(l, OP_EXP_DOWN)] and int(r[2]) == len(down) for r in kinds[(l + 1, OP_QKV)])
+
+
+def test_moe_shape_limits():
+    base = fx.CONFIGS["tiny"].replace(ffn_dim=0, n_experts=8, top_k=2, expert_ffn_dim=128, batch=4)
+    mk.Plan(mk.model_desc(base), 148)
+    mk.Plan(mk.model_desc(base.replace(batch=1)), 148)       # MoE at batch 1 runs on the tensor-core kernel
+    for bad in (base.replace(top_k=9, n_experts=16), base.replace(top_k=0), base.replace(top_k=9),
+                base.replace(expert_ffn_dim=100), base.replace(n_experts=512), base.replace(batch=8, top_k=9, n_experts=16)):
+        with pytest.raises(mk.MkError):
+            mk.Plan(mk.model_desc(bad), 148)
