@@ -136,7 +136,9 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const size_t o_ms = E ? cv.take(sizeof(int32_t) * (size_t)L * B * K) : 0;
   const size_t o_mw = E ? cv.take(sizeof(float) * (size_t)L * B * K) : 0;
   const size_t o_mc = E ? cv.take(sizeof(int32_t) * (size_t)L) : 0;
-  const size_t o_ma = E ? cv.take(sizeof(float) * (size_t)mk::moe_slots(E, B, K) * B * d.expert_ffn_dim) : 0;
+  const size_t o_ma = E ? cv.take(sizeof(uint16_t) * (size_t)mk::moe_slots(E, B, K) * B * d.expert_ffn_dim) : 0;
+  const size_t o_abf = mk::batched(d) ? cv.take(sizeof(uint16_t) * (size_t)B * qd) : 0;
+  const size_t o_xbf = mk::batched(d) && !E ? cv.take(sizeof(uint16_t) * (size_t)B * d.ffn_dim) : 0;
   const size_t o_po = cv.take(sizeof(float) * (size_t)B * nq * n_chunks * hd);
   const size_t o_pml = cv.take(sizeof(float) * (size_t)B * nq * n_chunks * 2);
   const size_t o_cnt = cv.take(sizeof(uint32_t) * (size_t)n_cnt);
@@ -246,8 +248,10 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
     p.moe_sel = (int32_t*)(base + o_ms);
     p.moe_selw = (float*)(base + o_mw);
     p.moe_count = (int32_t*)(base + o_mc);
-    p.moe_act = (float*)(base + o_ma);
+    p.moe_act = (uint16_t*)(base + o_ma);
   }
+  p.attn_bf = o_abf ? (uint16_t*)(base + o_abf) : nullptr;
+  p.act_bf = o_xbf ? (uint16_t*)(base + o_xbf) : nullptr;
   p.counters = (uint32_t*)(base + o_cnt);
   p.tickets = (uint32_t*)(base + o_tk);
   p.status = (int*)(base + o_st);

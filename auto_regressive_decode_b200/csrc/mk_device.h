@@ -36,6 +36,9 @@ struct Params {
   float* qkv;               // [B][nq*hd + 2*nkv*hd]
   float* attn;              // [B][nq*hd]
   float* act;               // [B][I]
+  // tensor-core kernel: the inputs of o_proj and down, bf16 (the mma operand type)
+  uint16_t* attn_bf;        // [B][nq*hd]
+  uint16_t* act_bf;         // [B][I]
   float* part_o;            // [B][nq][n_chunks][hd]
   float* part_ml;           // [B][nq][n_chunks][2]
   // MoE: E experts, top-k, expert SwiGLU width Ie; router logits and routing
@@ -45,7 +48,8 @@ struct Params {
   int32_t* moe_sel;         // [L][B][topk] picked experts, best first
   float* moe_selw;          // [L][B][topk] their weights
   int32_t* moe_count;       // [L] distinct picked experts
-  float* moe_act;           // [slots][B][Ie] SwiGLU outputs of the picked experts
+  uint16_t* moe_act;        // [slots][B][Ie] SwiGLU outputs of the picked experts times the
+                            // sequence's routing weight (0 if it did not pick the slot), bf16
   uint32_t* counters;       // [n_counters]
   uint32_t* tickets;        // [L][B][nkv]
   const mk_instr* instrs;

@@ -38,7 +38,11 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;  // 256
 constexpr int kThreads = kConsumerThreads + 32;        // + one producer warp
 constexpr int kStageBytes = 32 * 1024;                 // one ring slot
 constexpr int kStages = 6;                             // ring depth (192 KB), batch-1 kernel
-constexpr int kStagesBatched = 6;                      // ring depth of the batch > 1 kernel
+constexpr int kStagesBatched = 5;                      // ring depth of the tensor-core kernel
+// tensor-core kernel: bf16 inputs of o_proj / down / expert down staged in
+// shared memory, kXsSlots chunks of [kMaxBatch][kBChunk] at a padded pitch
+constexpr int kXsPitchBytes = 1024 * 2 + 16;
+constexpr int kXsSlots = 3;
 constexpr int kMaxRows = 256;                          // rows per GEMV instruction
 constexpr int kRedFloats = 4096;                       // cross-warp reduction buffer
 constexpr int kMaxBatch = 8;
@@ -122,6 +126,11 @@ constexpr int kBBoxRows = 8;                         // weight rows per TMA box
 constexpr int kBBoxBytes = kBBoxRows * kBChunk * 2;  // 16 KB
 constexpr int kBatchedMaxRows = 128;                 // rows per instruction: 8 tiles of 16
 constexpr int kBatchedMaxRowsGated = 96;             // gate/up: 12 tiles of 8 neurons
+constexpr int kBatchedMaxRowsLongK = 64;             // o_proj, down, expert down: 4 tiles of 16
+MK_HD int batched_max_rows(int op) {
+  return op == OP_GATEUP ? kBatchedMaxRowsGated
+                         : (op == OP_OPROJ || op == OP_DOWN || op == OP_EXP_DOWN ? kBatchedMaxRowsLongK : kBatchedMaxRows);
+}
 constexpr int kTmapsPerLayer = 8;  // wq wk wv wo w_gate w_up w_down router (then LM head, K cache, V cache)
 MK_HD int btile_rows(bool gated) { return gated ? 8 : 16; }
 // The tensor-core kernel runs every batch > 1 model and every MoE model.

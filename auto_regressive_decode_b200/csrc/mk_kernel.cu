@@ -66,7 +66,9 @@ struct Smem {
   static constexpr size_t kSlot = (size_t)kStageBytes;
   static_assert(2 * kBBoxBytes == kStageBytes, "a batched GEMV stage is two boxes");
   static constexpr size_t kRing = (size_t)kNst * kSlot;
-  static constexpr size_t kRed = (size_t)kRedFloats * sizeof(float);
+  // the reduction buffer doubles as the tensor-core kernel's input ring (never both at once)
+  static constexpr size_t kXs = BATCHED ? (size_t)kXsSlots * kMaxBatch * kXsPitchBytes : 0;
+  static constexpr size_t kRed = (size_t)kRedFloats * sizeof(float) > kXs ? (size_t)kRedFloats * sizeof(float) : kXs;
   static constexpr size_t kTotal = kRing + kRed + sizeof(Ctl);
   static_assert(kNst <= kStages, "Ctl holds kStages barrier pairs");
   static_assert(kTotal <= 227 * 1024, "dynamic shared memory of one CTA");
@@ -111,6 +113,18 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
 }
 
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// 16 bytes global -> shared, asynchronous, cached in L2 only (the source may
+// have been written by another SM during this kernel).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// all but the newest N committed groups of this thread have landed
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // One box of a 3-D tensor map (coordinates c0, c1, c2) into shared memory,
 // completing on `bar`.
 __device__ __forceinline__ void tma_box3(void* dst, const void* map, int c0, int c1, int c2, unsigned long long* bar,
@@ -1140,7 +1154,7 @@ struct Consumer {
   template <bool NORM, bool GATED>
   __device__ __forceinline__ bool gemv_tc(const Gemv& g, int op, int layer, int wait_idx, int wait_count, int slot) {
     constexpr int TR = GATED ? 8 : 16;  // output rows per tile
-    constexpr int MAXT = (GATED ? kBatchedMaxRowsGated : kBatchedMaxRows) / TR;
+    constexpr int MAXT = (GATED ? kBatchedMaxRowsGated : (NORM ? kBatchedMaxRows : kBatchedMaxRowsLongK)) / TR;
     constexpr int KPW = kBChunk / 16 / kConsumerWarps;  // k-steps per warp per chunk
     const int B = p.B, BH = B * p.H, nrows = g.r1 - g.r0, ntiles = g.bnt;
     const bool moe_down = op == OP_EXP_DOWN;
@@ -1150,14 +1164,10 @@ struct Consumer {
     int ld;  // elements per sequence in src
     if (op == OP_QKV) {
       src = p.xres + (size_t)(2 * layer) * BH, gain = p.layers[layer].attn_norm, ld = p.H;
-    } else if (op == OP_OPROJ) {
-      src = p.attn, ld = p.nq * p.hd;
     } else if (op == OP_GATEUP || op == OP_ROUTER || op == OP_EXP_GATEUP) {
       src = p.xres + (size_t)(2 * layer + 1) * BH, gain = p.layers[layer].mlp_norm, ld = p.H;
-    } else if (op == OP_DOWN) {
-      src = p.act, ld = p.I;
-    } else if (moe_down) {
-      src = p.moe_act, ld = p.Ie;  // slot s, sequence b at (s * B + b) * Ie
+    } else if (!NORM) {
+      src = nullptr, ld = 0;  // o_proj, down, expert down: bf16 inputs, staged below
     } else {
       src = p.xres + (size_t)(2 * p.L) * BH, gain = p.final_norm, ld = p.H;
     }
@@ -1167,41 +1177,12 @@ struct Consumer {
     }
     const int gq = lane >> 2, cq = lane & 3;
     const bool bval = gq < B;  // this lane's B-fragment column (sequence gq) exists
-    const float* xrow = src + (size_t)(bval ? gq : 0) * ld;
-    // columns of chunk j, and where its inputs start
+    const float* xrow = NORM ? src + (size_t)(bval ? gq : 0) * ld : nullptr;
+    // columns of chunk j
     auto cols = [&](int j) { return moe_down ? min(kBChunk, p.Ie - (j % nd) * kBChunk) : min(kBChunk, g.K - j * kBChunk); };
-    auto xbase = [&](int j) {
-      return moe_down ? xrow + (size_t)(j / nd) * B * p.Ie + (j % nd) * kBChunk : xrow + (size_t)j * kBChunk;
-    };
     float acc[MAXT][4];
 #pragma unroll
     for (int t2 = 0; t2 < MAXT; ++t2) acc[t2][0] = acc[t2][1] = acc[t2][2] = acc[t2][3] = 0.f;
-    float ss = 0.f;
-    float2 xr[KPW][2];
-    uint32_t gr[KPW][2];
-    uint32_t xf[KPW][2];
-    // raw inputs (and gains) of chunk j: k = 16 ks + 2 cq (+1) and + 8 (+1)
-    auto load = [&](int j) {
-      const int nks = cols(j) / 16;
-      const float* xb = xbase(j);
-#pragma unroll
-      for (int kk = 0; kk < KPW; ++kk) {
-        const int ks = warp + kk * kConsumerWarps;
-        const int kl = ks * 16 + 2 * cq, k = j * kBChunk + kl;
-        if (bval && ks < nks) {
-          xr[kk][0] = __ldcg(reinterpret_cast<const float2*>(xb + kl));
-          xr[kk][1] = __ldcg(reinterpret_cast<const float2*>(xb + kl + 8));
-          if (NORM) {
-            gr[kk][0] = __ldg(reinterpret_cast<const unsigned int*>(gain + k));
-            gr[kk][1] = __ldg(reinterpret_cast<const unsigned int*>(gain + k + 8));
-          }
-        } else {
-          xr[kk][0] = xr[kk][1] = make_float2(0.f, 0.f);
-          if (NORM) gr[kk][0] = gr[kk][1] = 0u;
-        }
-      }
-    };
-    load(0);
     // ldmatrix row address of this lane within a stage: A-row R = lane & 15
     // lives in box R >> 3 as row r = R & 7; k-step ks = warp + 8 kk reads
     // column block (warp >> 2) + 2 kk, 16-byte chunk ((warp & 3) << 1) | (lane >> 4),
@@ -1209,42 +1190,115 @@ struct Consumer {
     const uint32_t rr7 = (uint32_t)(lane & 7), ch = ((uint32_t)(warp & 3) << 1) | (uint32_t)(lane >> 4);
     const uint32_t lrow = (uint32_t)((lane >> 3) & 1) * kBBoxBytes + (uint32_t)(warp >> 2) * 1024u + rr7 * 128u +
                           ((ch ^ rr7) << 4);
-    for (int j = 0; j < g.bnch; ++j) {
-      const int nks = cols(j) / 16;
-      // expert down: the sequence's routing weight of this chunk's slot (0 if not picked)
-      const float rw = moe_down && bval ? ctl->moe_tw[j / nd][gq] : 1.f;
+    float ss = 0.f;
+    if constexpr (NORM) {
+      // K = hidden: few chunks of many tiles.  fp32 inputs (and gains) of the
+      // next chunk load into registers while this one streams.
+      float2 xr[KPW][2];
+      uint32_t gr[KPW][2];
+      uint32_t xf[KPW][2];
+      auto load = [&](int j) {
+        const int nks = cols(j) / 16;
 #pragma unroll
-      for (int kk = 0; kk < KPW; ++kk) {
+        for (int kk = 0; kk < KPW; ++kk) {
+          const int ks = warp + kk * kConsumerWarps;
+          const int k = j * kBChunk + ks * 16 + 2 * cq;
+          if (bval && ks < nks) {
+            xr[kk][0] = __ldcg(reinterpret_cast<const float2*>(xrow + k));
+            xr[kk][1] = __ldcg(reinterpret_cast<const float2*>(xrow + k + 8));
+            gr[kk][0] = __ldg(reinterpret_cast<const unsigned int*>(gain + k));
+            gr[kk][1] = __ldg(reinterpret_cast<const unsigned int*>(gain + k + 8));
+          } else {
+            xr[kk][0] = xr[kk][1] = make_float2(0.f, 0.f);
+            gr[kk][0] = gr[kk][1] = 0u;
+          }
+        }
+      };
+      load(0);
+      for (int j = 0; j < g.bnch; ++j) {
+        const int nks = cols(j) / 16;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float2 x = xr[kk][h];
-          if (NORM) {
+        for (int kk = 0; kk < KPW; ++kk) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float2 x = xr[kk][h];
             ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
             xf[kk][h] = pack_bf16x2(x.x * bf16_lo(gr[kk][h]), x.y * bf16_hi(gr[kk][h]));
-          } else {
-            xf[kk][h] = pack_bf16x2(x.x * rw, x.y * rw);
           }
         }
-      }
-      if (tr && j == 0) tr[4] = globaltimer();
-      if (j + 1 < g.bnch) load(j + 1);
+        if (tr && j == 0) tr[4] = globaltimer();
+        if (j + 1 < g.bnch) load(j + 1);
 #pragma unroll
-      for (int t2 = 0; t2 < MAXT; ++t2) {
-        if (t2 < ntiles) {
-          const uint32_t st = smem_addr(wait_full()) + lrow;
-          if (tr && j == 0 && t2 == 0) tr[5] = globaltimer();
+        for (int t2 = 0; t2 < MAXT; ++t2) {
+          if (t2 < ntiles) {
+            const uint32_t st = smem_addr(wait_full()) + lrow;
+            if (tr && j == 0 && t2 == 0) tr[5] = globaltimer();
 #pragma unroll
-          for (int kk = 0; kk < KPW; ++kk) {
-            const int ks = warp + kk * kConsumerWarps;
-            if (ks < nks) {
-              uint32_t a[4];
-              ldmatrix_x4(a, st + (uint32_t)kk * 2048u);
-              mma16816(acc[t2], a[0], a[1], a[2], a[3], xf[kk][0], xf[kk][1]);
+            for (int kk = 0; kk < KPW; ++kk) {
+              const int ks = warp + kk * kConsumerWarps;
+              if (ks < nks) {
+                uint32_t a[4];
+                ldmatrix_x4(a, st + (uint32_t)kk * 2048u);
+                mma16816(acc[t2], a[0], a[1], a[2], a[3], xf[kk][0], xf[kk][1]);
+              }
             }
+            release();
           }
-          release();
         }
       }
+    } else {
+      // Long K over few rows (o_proj, down, expert down): a chunk may be one
+      // tile, shorter than an L2 round trip.  The chunks' bf16 inputs stream
+      // into a shared-memory ring with cp.async, two chunks ahead; the ring
+      // is [slot][sequence][column] at a padded pitch (conflict-free
+      // fragment reads), in the reduction buffer.
+      const uint16_t* xsrc = op == OP_OPROJ ? p.attn_bf : (moe_down ? p.moe_act : p.act_bf);
+      const int xld = op == OP_OPROJ ? p.nq * p.hd : (moe_down ? p.Ie : p.I);
+      uint8_t* xs = reinterpret_cast<uint8_t*>(red);
+      auto stage_x = [&](int j) {  // chunk j into ring slot j % kXsSlots (this thread's pieces)
+        const int c16 = cols(j) / 8;  // 16-byte pieces per sequence
+        const uint16_t* s0 = moe_down ? xsrc + (size_t)(j / nd) * B * p.Ie + (j % nd) * kBChunk
+                                      : xsrc + (size_t)j * kBChunk;
+        uint8_t* d0 = xs + (size_t)(j % kXsSlots) * kMaxBatch * kXsPitchBytes;
+        for (int idx = t; idx < B * c16; idx += kConsumerThreads) {
+          const int b = idx / c16, c = idx % c16;
+          cp_async16(d0 + (size_t)b * kXsPitchBytes + c * 16, s0 + (size_t)b * xld + c * 8);
+        }
+      };
+      stage_x(0);
+      cp_async_commit();
+      if (g.bnch > 1) stage_x(1);
+      cp_async_commit();
+      if (tr) tr[4] = globaltimer();
+      const uint32_t xrd = (uint32_t)gq * kXsPitchBytes + (uint32_t)cq * 4u;  // this lane's fragment row
+      for (int j = 0; j < g.bnch; ++j) {
+        const int nks = cols(j) / 16;
+        cp_async_wait<1>();  // chunk j landed (only chunk j + 1 may be pending)
+        consumer_bar();      // ... for every thread's pieces; every warp is done with chunk j - 1
+        if (j + 2 < g.bnch) stage_x(j + 2);  // into chunk j - 1's slot
+        cp_async_commit();
+        const uint32_t xb = smem_addr(xs + (size_t)(j % kXsSlots) * kMaxBatch * kXsPitchBytes) + xrd;
+#pragma unroll
+        for (int t2 = 0; t2 < MAXT; ++t2) {
+          if (t2 < ntiles) {
+            const uint32_t st = smem_addr(wait_full()) + lrow;
+            if (tr && j == 0 && t2 == 0) tr[5] = globaltimer();
+#pragma unroll
+            for (int kk = 0; kk < KPW; ++kk) {
+              const int ks = warp + kk * kConsumerWarps;
+              if (ks < nks) {
+                uint32_t a[4], b0, b1;
+                ldmatrix_x4(a, st + (uint32_t)kk * 2048u);
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0) : "r"(xb + (uint32_t)ks * 32u));
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1) : "r"(xb + (uint32_t)ks * 32u + 16u));
+                mma16816(acc[t2], a[0], a[1], a[2], a[3], b0, b1);
+              }
+            }
+            release();
+          }
+        }
+      }
+      consumer_bar();  // the ring (the reduction buffer) is free for the reduction below
     }
     if (tr) tr[6] = globaltimer();
     if (NORM) {
@@ -1289,10 +1343,11 @@ struct Consumer {
             const int row = tile * TR + lgq;  // v0 = gate, v1 = up of neuron row
             if (row < nrows) {
               const float a = v0 / (1.f + expf(-v0)) * v1;
-              if (op == OP_EXP_GATEUP)
-                p.moe_act[((size_t)slot * B + b) * p.Ie + (g.r0 - ctl->moe_uniq[slot] * p.Ie) + row] = a;
+              if (op == OP_EXP_GATEUP)  // weighted by the sequence's routing weight of the slot
+                p.moe_act[((size_t)slot * B + b) * p.Ie + (g.r0 - ctl->moe_uniq[slot] * p.Ie) + row] =
+                    f32_to_bf16_bits(a * ctl->moe_tw[slot][b]);
               else
-                p.act[(size_t)b * p.I + g.r0 + row] = a;
+                p.act_bf[(size_t)b * p.I + g.r0 + row] = f32_to_bf16_bits(a);
             }
           } else {
 #pragma unroll
@@ -1625,7 +1680,7 @@ struct Consumer {
           num = fmaf(c, red[(w * HR + hh) * HD + d], num);
         }
         if (a.npieces == 1) {  // the whole row: the output itself
-          p.attn[(size_t)a.b * p.nq * HD + (size_t)(q0 + h) * HD + d] = num / den;
+          p.attn_bf[(size_t)a.b * p.nq * HD + (size_t)(q0 + h) * HD + d] = f32_to_bf16_bits(num / den);
         } else {
           const size_t pi = pbase + (size_t)h * p.n_chunks;
           p.part_o[pi * HD + d] = num;
@@ -1947,7 +2002,10 @@ struct Consumer {
           den = fmaf(w, ml[2 * c + 1], den);
           num = fmaf(w, __ldcg(po + (size_t)c * HD), num);
         }
-        p.attn[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = num / den;
+        if constexpr (BATCHED)
+          p.attn_bf[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = f32_to_bf16_bits(num / den);
+        else
+          p.attn[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = num / den;
       }
       signal(sig_idx);
     }

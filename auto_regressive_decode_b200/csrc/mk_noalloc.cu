@@ -140,7 +140,9 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   const size_t o_ms = E ? take(sizeof(int32_t) * (size_t)L * B * K) : 0;
   const size_t o_mw = E ? take(sizeof(float) * (size_t)L * B * K) : 0;
   const size_t o_mc = E ? take(sizeof(int32_t) * (size_t)L) : 0;
-  const size_t o_ma = E ? take(sizeof(float) * (size_t)mk::moe_slots(E, B, K) * B * d.expert_ffn_dim) : 0;
+  const size_t o_ma = E ? take(sizeof(uint16_t) * (size_t)mk::moe_slots(E, B, K) * B * d.expert_ffn_dim) : 0;
+  const size_t o_abf = mk::batched(d) ? take(sizeof(uint16_t) * (size_t)B * qd) : 0;
+  const size_t o_xbf = mk::batched(d) && !E ? take(sizeof(uint16_t) * (size_t)B * d.ffn_dim) : 0;
   const size_t o_po = take(sizeof(float) * (size_t)B * nq * n_chunks * hd);
   const size_t o_pml = take(sizeof(float) * (size_t)B * nq * n_chunks * 2);
   const size_t o_ins = take(sizeof(mk_instr) * instrs.size());
@@ -223,8 +225,10 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
     p.moe_sel = (int32_t*)(base + o_ms);
     p.moe_selw = (float*)(base + o_mw);
     p.moe_count = (int32_t*)(base + o_mc);
-    p.moe_act = (float*)(base + o_ma);
+    p.moe_act = (uint16_t*)(base + o_ma);
   }
+  p.attn_bf = o_abf ? (uint16_t*)(base + o_abf) : nullptr;
+  p.act_bf = o_xbf ? (uint16_t*)(base + o_xbf) : nullptr;
   p.counters = (uint32_t*)(base + o_cnt);
   p.tickets = (uint32_t*)(base + o_tk);
   p.status = (int*)(base + o_st);

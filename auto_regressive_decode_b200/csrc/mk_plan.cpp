@@ -96,8 +96,7 @@ struct Builder {
   int rows_op(int op, int layer, int N, const std::vector<int>& cuts, int wait_idx, int wait_count, int sig_idx) {
     int n = 0;
     const int n_sm = p->n_sm;
-    const int max_rows =
-        batched(p->d) ? (op == OP_GATEUP ? kBatchedMaxRowsGated : kBatchedMaxRows) : kMaxRows;
+    const int max_rows = batched(p->d) ? batched_max_rows(op) : kMaxRows;
     // batch > 1: row ranges start at multiples of kBBoxRows (a TMA box
     // never reaches into another SM's rows or across wq | wk | wv)
     const int unit = batched(p->d) ? kBBoxRows : 1;

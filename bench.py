@@ -45,12 +45,19 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 def weight_bytes_read(cfg) -> int:
-    """bf16 weight bytes a dense step reads: every layer matrix and norm, the LM head, B embedding rows."""
+    """bf16 weight bytes a step reads apart from MoE experts: every layer matrix and norm (MoE: the
+    router instead of the MLP), the LM head, B embedding rows."""
     H, L = cfg.hidden, cfg.n_layers
-    per = 2 * H + cfg.q_dim * H * 2 + cfg.kv_dim * H * 2 + 3 * cfg.ffn_dim * H
+    per = 2 * H + cfg.q_dim * H * 2 + cfg.kv_dim * H * 2
+    per += cfg.n_experts * H if cfg.n_experts else 3 * cfg.ffn_dim * H
     if cfg.qk_norm:
         per += 2 * cfg.head_dim
     return 2 * (L * per + H + cfg.vocab * H + cfg.batch * H)
+
+
+def expert_bytes_read(cfg, distinct_per_step) -> float:
+    """MoE: bf16 bytes of the distinct picked experts' gate, up and down matrices (each read once)."""
+    return 2.0 * 3 * cfg.expert_ffn_dim * cfg.hidden * float(np.mean(distinct_per_step))
 
 
 def kv_bytes(cfg, seq_lens) -> int:
@@ -142,13 +149,14 @@ class ClockSampler:
 
 def cpu_baseline(cfg, seed=fx.DEFAULT_SEED, max_layers=2):
     import oracle as ora
-    from tests.helpers import host_model
+    from tests.helpers import expert_loader, host_model
     n = min(max_layers, cfg.n_layers)
     g, ls = host_model(cfg, seed, layers=range(n))
     S = fx.context_lengths(cfg, seed)
     kc = [fx.kv_prefill(cfg, l, 0, S, seed) for l in range(n)]
     vc = [fx.kv_prefill(cfg, l, 1, S, seed) for l in range(n)]
-    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls)
+    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls,
+                      expert_loader(cfg, seed) if cfg.n_experts else None)
     tok = fx.tokens(cfg, seed)[0]
     x = fx.bf16_to_f32(g["embed"][tok]).astype(np.float64)
     t0 = time.perf_counter()
@@ -172,13 +180,14 @@ def run_reference(args, cfg, rank):
     if rank != 0:
         return
     import oracle as ora
-    from tests.helpers import host_model
+    from tests.helpers import expert_loader, host_model
     n_lay = min(2, cfg.n_layers)
     g, ls = host_model(cfg, layers=range(n_lay))
     S = fx.context_lengths(cfg)
     kc = [fx.kv_prefill(cfg, l, 0, S) for l in range(n_lay)]
     vc = [fx.kv_prefill(cfg, l, 1, S) for l in range(n_lay)]
-    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls)
+    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls,
+                      expert_loader(cfg) if cfg.n_experts else None)
     tok = fx.tokens(cfg)[0]
     x = fx.bf16_to_f32(g["embed"][tok]).astype(np.float64)
     times = []
@@ -300,6 +309,14 @@ def run_mk(args, cfg, rank, world):
     if st != 0:
         raise RuntimeError(f"device status {mk.mk_status_string(st)}")
 
+    # ---- MoE: the distinct experts each timed step read (its routing, replayed untimed)
+    distinct = []
+    if cfg.n_experts:
+        for j in range(args.steps):
+            i = args.warmup + j
+            dec.step(all_tok[i], all_len[i], all_len[i], logits)
+            distinct.append(int(dec.routing()[3].sum()))
+
     # ---- max over ranks
     t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -315,6 +332,8 @@ def run_mk(args, cfg, rank, world):
     e2e_tok_s = world * B * args.steps / (e2e_ms / 1e3)
     lens = [S0 + (k % cfg.steps) for k in range(args.warmup, n_total)]
     bytes_step = weight_bytes_read(cfg) + float(np.mean([kv_bytes(cfg, s) for s in lens]))
+    if cfg.n_experts:
+        bytes_step += expert_bytes_read(cfg, distinct)
     peak, peak_kind = measured_peaks()
     achieved = bytes_step / (ms / 1e3) / 1e9
     traffic = ncu_traffic(cfg.name)
@@ -327,6 +346,7 @@ def run_mk(args, cfg, rank, world):
         "step_latency_ms": {"median": statistics.median(per_step_ms), "p10": float(np.percentile(per_step_ms, 10)),
                             "p90": float(np.percentile(per_step_ms, 90))},
         "bytes_per_step": bytes_step,
+        **({"moe_distinct_experts_per_layer": float(np.mean(distinct)) / cfg.n_layers} if cfg.n_experts else {}),
         "mbu": {"vs_spec_8tbs": achieved / SPEC_HBM_GBS, f"vs_{peak_kind}_{peak:.0f}gbs": achieved / peak},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
