@@ -370,10 +370,14 @@ def main():
     ap.add_argument("--config", default="dense-8b", choices=sorted(fx.CONFIGS))
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: the config with this many layers (same shapes); not a bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = fx.CONFIGS[args.config]
+    if args.layers:
+        cfg = cfg.replace(name=f"{cfg.name}-{args.layers}l", n_layers=args.layers)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
