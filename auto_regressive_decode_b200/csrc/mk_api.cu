@@ -148,7 +148,7 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const size_t o_off = cv.take(sizeof(int32_t) * offsets.size());
   const size_t o_lay = cv.take(sizeof(mk::LayerPtrs) * (size_t)L);
   const size_t o_rope = cv.take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
-  const size_t n_tmaps = mk::batched(d) ? (size_t)mk::kTmapsPerLayer * L + 3 : 0;
+  const size_t n_tmaps = (size_t)mk::kTmapsPerLayer * L + 3;  // KV caches always; weights on the tensor-core kernel
   const size_t o_tmap = n_tmaps ? cv.take(128 * n_tmaps) : 0;
   const char* trace_env = getenv("MK_TRACE");
   const bool tracing = trace_env && atoi(trace_env) > 0;

@@ -642,13 +642,6 @@ struct Cursor {
   // f(src, bytes, smem offset) for every copy of the current stage; returns the stage's bytes.
   template <typename F>
   __device__ __forceinline__ uint32_t copies(F&& f) const {
-    if (op == OP_ATTN) {
-      const int np = min(a.P, a.n_cached - sub * a.P);
-      const uint32_t bytes = (uint32_t)np * pp->hd * 2u;
-      const uint16_t* src = (kv ? pp->vc : pp->kc) + a.cache_base + (size_t)sub * a.P * pp->hd;
-      for (uint32_t o = 0; o < bytes; o += pp->copy_piece) f(src + o / 2, min(pp->copy_piece, bytes - o), o);
-      return bytes;
-    }
     const int R = g.tile.rows_per_stage;
     const int nr = min(R, g.seg_rows(sg) - rr);
     const uint32_t seg = (uint32_t)g.Kc * 2u;
@@ -718,7 +711,7 @@ struct Cursor {
 
   __device__ __forceinline__ uint32_t stage_bytes() const {
     if (op == OP_ATTN)
-      return pp->tc ? (uint32_t)kStageBytes : (uint32_t)min(a.P, a.n_cached - sub * a.P) * pp->hd * 2u;
+      return (uint32_t)kStageBytes;  // a TMA box: always a whole stage of positions
     if (pp->tc) return (g.wup || g.r1 - g.r0 - sg * 16 > 8) ? 2u * kBBoxBytes : (uint32_t)kBBoxBytes;
     const uint32_t b = (uint32_t)min(g.tile.rows_per_stage, g.seg_rows(sg) - rr) * (uint32_t)g.Kc * 2u;
     return g.wup ? 2 * b : b;
@@ -818,7 +811,7 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
     if (!(ok = pr.claim(&dst, &bar))) break;
     const uint32_t bytes = cur.stage_bytes();
     mbar_arrive_expect_tx(bar, bytes);
-    if (BATCHED && cur.op == OP_ATTN) {
+    if (cur.op == OP_ATTN) {
       const uint8_t* map;
       int row;
       cur.attn_box(&map, &row);
@@ -1522,15 +1515,25 @@ struct Consumer {
     constexpr int DT = HD / 16;                  // dimension tiles of the P.V mma
     constexpr uint32_t CBB = (uint32_t)P * 128u;  // bytes of one 64-column block of a stage
     const int gq = lane >> 2, cq = lane & 3;
-    uint32_t qf[KS][2];
+    // The batch-1 kernel (fp32 activations elsewhere) takes q and the
+    // probabilities as sums of two bf16 parts (hi + lo), whose two mma keep
+    // scores and outputs at about fp32 accuracy (keys and values are bf16
+    // already); the tensor-core kernel rounds them to one bf16, like its GEMV inputs.
+    constexpr bool SPLIT = !BATCHED;
+    uint32_t qf[KS][2], ql[KS][2];
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       if (gq < G) {
         const float* qh = ctl->qs + gq * HD + ks * 16 + 2 * cq;
-        qf[ks][0] = pack_bf16x2(qh[0], qh[1]);
-        qf[ks][1] = pack_bf16x2(qh[8], qh[9]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float x0 = qh[8 * h], x1 = qh[8 * h + 1];
+          const uint32_t hi = pack_bf16x2(x0, x1);
+          qf[ks][h] = hi;
+          ql[ks][h] = SPLIT ? pack_bf16x2(x0 - bf16_lo(hi), x1 - bf16_hi(hi)) : 0u;
+        }
       } else {
-        qf[ks][0] = qf[ks][1] = 0u;
+        qf[ks][0] = qf[ks][1] = ql[ks][0] = ql[ks][1] = 0u;
       }
     }
     float o[DT][4];
@@ -1558,6 +1561,7 @@ struct Consumer {
             uint32_t af[4];
             ldmatrix_x4(af, Ks + (uint32_t)(ks >> 2) * CBB + (uint32_t)key0 * 128u + krow + ((ch ^ r7) << 4));
             mma16816(sc, af[0], af[1], af[2], af[3], qf[ks][0], qf[ks][1]);
+            if (SPLIT) mma16816(sc, af[0], af[1], af[2], af[3], ql[ks][0], ql[ks][1]);
           }
           // this lane: keys key0 + gq (sc[0..1]) and key0 + gq + 8 (sc[2..3]), heads 2cq, 2cq + 1
           const bool v0 = key0 + gq < np, v1 = key0 + gq + 8 < np;
@@ -1590,8 +1594,11 @@ struct Consumer {
             o[dt][2] *= c0;
             o[dt][3] *= c1;
           }
-          const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p00, p01));  // P[keys 2cq, 2cq+1][head gq]
-          const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p10, p11));  // P[keys 8+2cq, 9+2cq][head gq]
+          // P[keys 2cq, 2cq+1][head gq] and P[keys 8+2cq, 9+2cq][head gq], each as hi + lo bf16
+          const uint32_t ph0 = pack_bf16x2(p00, p01), ph1 = pack_bf16x2(p10, p11);
+          const uint32_t pb0 = movmatrix_trans(ph0), pb1 = movmatrix_trans(ph1);
+          const uint32_t pl0 = SPLIT ? movmatrix_trans(pack_bf16x2(p00 - bf16_lo(ph0), p01 - bf16_hi(ph0))) : 0u;
+          const uint32_t pl1 = SPLIT ? movmatrix_trans(pack_bf16x2(p10 - bf16_lo(ph1), p11 - bf16_hi(ph1))) : 0u;
           if (key0 + 16 > np) {
             // V rows past the cached positions may hold anything (0 * NaN is
             // NaN): zero this tile's absent rows, in every 64-column block
@@ -1611,6 +1618,7 @@ struct Consumer {
             uint32_t af[4];
             ldmatrix_x4_trans(af, Vs + (uint32_t)(dt >> 2) * CBB + (uint32_t)key0 * 128u + vrow + ((ch ^ r7) << 4));
             mma16816(o[dt], af[0], af[1], af[2], af[3], pb0, pb1);
+            if (SPLIT) mma16816(o[dt], af[0], af[1], af[2], af[3], pl0, pl1);
           }
         }
       }
@@ -1680,7 +1688,10 @@ struct Consumer {
           num = fmaf(c, red[(w * HR + hh) * HD + d], num);
         }
         if (a.npieces == 1) {  // the whole row: the output itself
-          p.attn_bf[(size_t)a.b * p.nq * HD + (size_t)(q0 + h) * HD + d] = f32_to_bf16_bits(num / den);
+          if constexpr (BATCHED)
+            p.attn_bf[(size_t)a.b * p.nq * HD + (size_t)(q0 + h) * HD + d] = f32_to_bf16_bits(num / den);
+          else
+            p.attn[(size_t)a.b * p.nq * HD + (size_t)(q0 + h) * HD + d] = num / den;
         } else {
           const size_t pi = pbase + (size_t)h * p.n_chunks;
           p.part_o[pi * HD + d] = num;
@@ -1718,8 +1729,6 @@ struct Consumer {
   // row to finish merges all partials.
   template <int HD, int G>
   __device__ __forceinline__ void attn_piece(const Attn& a, int layer, int sig_idx) {
-    constexpr int LPP = HD / 8;    // lanes per position (16-byte vectors)
-    constexpr int PPW = 32 / LPP;  // positions per warp pass
     constexpr int NP = HD / 64;    // rotation pairs per lane
     const int qd = p.nq * HD, kvd = p.nkv * HD;
     const float* qkv = p.qkv + (size_t)a.b * (qd + 2 * kvd);
@@ -1727,7 +1736,6 @@ struct Consumer {
     const int group = p.nq / p.nkv, nhg = group / G;
     const int q0 = a.kvh * group + a.hg * G;  // first query head
     const float qscale = 1.4426950408889634f * rsqrtf((float)HD);  // log2(e) / sqrt(hd)
-    const int pl = lane / LPP, vi = lane % LPP;
     float2 csr[NP];
     if (a.active) {
       const float2* cs = p.rope + (size_t)p.positions[a.b] * (HD / 2);
@@ -1793,172 +1801,7 @@ struct Consumer {
       }
       consumer_bar();
       if (tr) tr[4] = globaltimer();
-      if constexpr (!BATCHED) {
-        // Each group of LPP lanes owns 8 dimensions per lane and walks blocks
-        // of TB consecutive positions.  One transposed reduction leaves every
-        // (position, head) score of the block on its own lane (R = TB * G
-        // values), so each exponential is computed once; p and the rescale
-        // factors are then broadcast for the P.V update.
-        constexpr int TB = LPP / G < 4 ? LPP / G : 4;
-        constexpr int R = TB * G;
-        constexpr int SH = ilog2c(LPP) - ilog2c(R);  // lane -> value index shift
-        const int gbase = lane & ~(LPP - 1);
-        const int my_t = (vi >> SH) / G;  // this lane's position in a block (its head is (vi >> SH) % G)
-        float q[G][8], o[G][8];
-        float m_l = -1e30f, l_l = 0.f;  // running max / sum of this lane's head
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            q[h][e] = ctl->qs[h * HD + vi * 8 + e];
-            o[h][e] = 0.f;
-          }
-        }
-        // one block of TB positions starting at row t0 of Kb/Vb (rows >= np are absent)
-        auto block = [&](const uint16_t* Kb, const uint16_t* Vb, int t0, int np) {
-          float acc[R];
-#pragma unroll
-          for (int tt = 0; tt < TB; ++tt) {
-            float kf[8];
-            if (t0 + tt < np) {
-              unpack8(*reinterpret_cast<const uint4*>(Kb + (size_t)(t0 + tt) * HD + vi * 8), kf);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) kf[e] = 0.f;
-            }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              float d = 0.f;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) d = fmaf(q[h][e], kf[e], d);
-              acc[tt * G + h] = d;
-            }
-          }
-          // every lane takes part in the reduction (full-mask shuffles), then
-          // lanes whose position is absent drop their score
-          const float red_sc = group_reduce_multi<R, LPP>(acc, lane);
-          const bool valid = t0 + my_t < np;
-          const float sc = valid ? red_sc : -1e30f;
-          float bm = sc;
-#pragma unroll
-          for (int off = G << SH; off < LPP; off <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-          const float mn = fmaxf(m_l, bm);
-          const float corr = exp2f(m_l - mn);
-          const float pv = valid ? exp2f(sc - mn) : 0.f;
-          float ps = pv;
-#pragma unroll
-          for (int off = G << SH; off < LPP; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-          l_l = l_l * corr + ps;
-          m_l = mn;
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float c = __shfl_sync(0xffffffffu, corr, gbase + ((h) << SH));
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[h][e] *= c;
-          }
-#pragma unroll
-          for (int tt = 0; tt < TB; ++tt) {
-            float vf[8];
-            if (t0 + tt < np) {
-              unpack8(*reinterpret_cast<const uint4*>(Vb + (size_t)(t0 + tt) * HD + vi * 8), vf);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) vf[e] = 0.f;
-            }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const float pr = __shfl_sync(0xffffffffu, pv, gbase + ((tt * G + h) << SH));
-#pragma unroll
-              for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e]);
-            }
-          }
-        };
-        // -- cached positions, streamed K stage then V stage
-        for (int s = 0; s < a.nsub; ++s) {
-          const int np = min(a.P, a.n_cached - s * a.P);
-          const uint16_t* Ks = reinterpret_cast<const uint16_t*>(wait_stage(k));
-          const uint16_t* Vs = reinterpret_cast<const uint16_t*>(wait_stage(k + 1));
-          if (tr && s == 0) tr[5] = globaltimer();
-          for (int tb = warp * PPW * TB; tb < np; tb += kConsumerWarps * PPW * TB) block(Ks, Vs, tb + pl * TB, np);
-          release();  // K slot
-          release();  // V slot
-        }
-        if (tr) tr[6] = globaltimer();
-        // -- the new token (warp 0, first position group)
-        if (a.owns_new && warp == 0) block(ctl->knew, ctl->vnew, pl * TB, 1);
-        // every lane gets (m, l) of every head of its group
-        float m[G], l[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          m[h] = __shfl_sync(0xffffffffu, m_l, gbase + (h << SH));
-          l[h] = __shfl_sync(0xffffffffu, l_l, gbase + (h << SH));
-        }
-        // -- merge the position groups of each warp
-#pragma unroll
-        for (int off = LPP; off < 32; off <<= 1) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, m[h], off);
-            const float l2 = __shfl_xor_sync(0xffffffffu, l[h], off);
-            const float mn = fmaxf(m[h], m2);
-            const float c1 = exp2f(m[h] - mn), c2 = exp2f(m2 - mn);
-            l[h] = l[h] * c1 + l2 * c2;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float o2 = __shfl_xor_sync(0xffffffffu, o[h][e], off);
-              o[h][e] = o[h][e] * c1 + o2 * c2;
-            }
-            m[h] = mn;
-          }
-        }
-        // -- merge the warps through shared memory, HR heads per round
-        constexpr int HR = kRedFloats / (kConsumerWarps * HD) < G ? kRedFloats / (kConsumerWarps * HD) : G;
-        const size_t pbase = ((size_t)a.b * p.nq + q0) * p.n_chunks + a.c;
-        if (pl == 0 && vi == 0) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            ctl->aml[(warp * kMaxGroup + h) * 2] = m[h];
-            ctl->aml[(warp * kMaxGroup + h) * 2 + 1] = l[h];
-          }
-        }
-#pragma unroll
-        for (int h0 = 0; h0 < G; h0 += HR) {
-          if (pl == 0) {
-#pragma unroll
-            for (int hh = 0; hh < HR; ++hh) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) red[(warp * HR + hh) * HD + vi * 8 + e] = o[h0 + hh][e];
-            }
-          }
-          consumer_bar();
-          for (int id = t; id < HR * HD; id += kConsumerThreads) {
-            const int hh = id / HD, d = id % HD, h = h0 + hh;
-            float M = -1e30f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ctl->aml[(w * kMaxGroup + h) * 2]);
-            float den = 0.f, num = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-              const float c = exp2f(ctl->aml[(w * kMaxGroup + h) * 2] - M);
-              den = fmaf(c, ctl->aml[(w * kMaxGroup + h) * 2 + 1], den);
-              num = fmaf(c, red[(w * HR + hh) * HD + d], num);
-            }
-            if (a.npieces == 1) {  // the whole row: the output itself
-              p.attn[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = num / den;
-            } else {
-              const size_t pi = pbase + (size_t)h * p.n_chunks;
-              p.part_o[pi * HD + d] = num;
-              if (d == 0) {
-                p.part_ml[pi * 2] = M;
-                p.part_ml[pi * 2 + 1] = den;
-              }
-            }
-          }
-          consumer_bar();
-        }
-      } else {
-        attn_tc<HD, G>(a, q0);
-      }
+      attn_tc<HD, G>(a, q0);
     }
     if (a.npieces == 1) {  // written above: no partials to merge
       signal(sig_idx);
@@ -2110,7 +1953,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
       }
     }
     // the swizzled TMA boxes of the batched GEMV need 1024-byte aligned slots
-    if (!bad && BATCHED && (smem_addr(ring) & 1023u) != 0) {
+    if (!bad && (smem_addr(ring) & 1023u) != 0) {
       set_status(p, MK_ERR_UNSUPPORTED, -3);
       bad = 1;
     }

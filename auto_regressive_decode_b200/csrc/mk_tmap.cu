@@ -58,6 +58,16 @@ bool encode_one(EncodeTiledFn enc, const void* w, int64_t rows, int K, uint8_t* 
 cudaError_t encode_tmaps(const mk_model_desc& d, const mk_weights& w, const mk_kv& kv, uint8_t* out) {
   EncodeTiledFn enc = encoder();
   if (!enc) return cudaErrorNotSupported;
+  if (!batched(d)) {  // CUDA-core GEMVs read weights with 1-D copies: only the KV caches' maps
+    memset(out, 0, (size_t)(kTmapsPerLayer * d.n_layers + 3) * 128);
+    uint8_t* g = out + (size_t)d.n_layers * kTmapsPerLayer * 128;
+    const int64_t kv_rows = (int64_t)d.n_layers * d.batch * d.n_kv_heads * d.max_ctx;
+    const int P = attn_stage_positions(d.head_dim);
+    return encode_one(enc, kv.k, kv_rows, d.head_dim, g + 128, P, d.head_dim / 64) &&
+                   encode_one(enc, kv.v, kv_rows, d.head_dim, g + 256, P, d.head_dim / 64)
+               ? cudaSuccess
+               : cudaErrorInvalidValue;
+  }
   const int H = d.hidden, qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim;
   // MoE: the experts' matrices are stacked, [E][Ie][H] for gate and up and
   // [E][H][Ie] for down, and read as one tall matrix each
