@@ -50,6 +50,7 @@ constexpr int kMaxGroup = 8;                           // query heads per KV hea
 constexpr int kMaxHeadDim = 128;
 constexpr int kTraceStamps = 8;                        // per-instruction trace words
 constexpr uint32_t kDefaultCopyPiece = 32 * 1024;  // bytes per bulk copy
+constexpr uint32_t kL2AheadBytes = 256 * 1024;     // batch-1 kernel: L2 prefetch beyond the ring per instruction
 
 // ---- dependency counters -----------------------------------------------------
 // Each counter is bumped once per producing instruction per step; a waiter

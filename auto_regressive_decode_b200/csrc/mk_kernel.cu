@@ -40,6 +40,7 @@ struct Ctl {
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
   int dead;       // this CTA gives up: every wait returns at once
+  int waiting;    // the consumers are blocked on a dependency counter
   int last;       // attention: this CTA merges (broadcast)
   int flag;       // generic broadcast
   float sred[kConsumerWarps * 2];
@@ -123,6 +124,11 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Bring a global range into L2 (no destination, no completion to wait for).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // One box of a 3-D tensor map (coordinates c0, c1, c2) into shared memory,
@@ -662,6 +668,25 @@ struct Cursor {
     return g.wup ? 2 * bytes : bytes;
   }
 
+  // Batch-1 GEMV: bring into L2 up to `budget` bytes of the rows the ring
+  // has not reached yet (whole rows from the current one to the end of the
+  // instruction; the gate/up pair's up rows alongside).  Row blocks are
+  // contiguous, so this is one prefetch per matrix segment.
+  __device__ __forceinline__ void prefetch_rest(uint32_t budget) const {
+    if (op == OP_ATTN || pp->tc || i >= n) return;
+    const size_t rowb = (size_t)g.K * 2;
+    for (int s2 = sg; s2 < g.nseg && budget >= 16; ++s2) {
+      const int from = s2 == sg ? rr : 0;
+      const size_t left = (size_t)(g.seg_rows(s2) - from) * rowb * (g.wup ? 2 : 1);
+      if (left == 0) continue;
+      const uint32_t take = (uint32_t)(left < budget ? left : budget) / (g.wup ? 2u : 1u) & ~15u;
+      if (take == 0) break;
+      prefetch_l2(g.seg_ptr(s2) + (size_t)from * g.K, take);
+      if (g.wup) prefetch_l2(g.wup + (size_t)from * g.K, take);
+      budget -= take * (g.wup ? 2u : 1u);
+    }
+  }
+
   // Batched GEMV stage: f(tensor map, row, column block, shared-memory
   // offset) per TMA box: the two 8-row halves of 16-row tile sg (the second
   // only if the tile has more than 8 rows), or gate over up rows of 8-row tile
@@ -748,7 +773,9 @@ struct Producer {
   }
 
   // Claim the next slot (waiting until the consumers released it).
-  __device__ __forceinline__ bool claim(uint8_t** dst, unsigned long long** bar) {
+  // on_wait() runs while the ring is full and the consumers wait on a dependency.
+  template <typename F>
+  __device__ __forceinline__ bool claim(uint8_t** dst, unsigned long long** bar, F&& on_wait) {
     const int slot = k % NST;
     if (k >= (uint32_t)NST) {
       const uint32_t parity = ((k / NST) - 1) & 1;
@@ -756,6 +783,7 @@ struct Producer {
         const uint64_t t0 = globaltimer();
         uint32_t spins = 0;
         while (!mbar_try_wait(&ctl->empty[slot], parity)) {
+          if (*(volatile int*)&ctl->waiting) on_wait();
           if (*(volatile int*)&ctl->dead) return false;
           if ((++spins & 63) == 0) {
             if (ld_relaxed_i32(p.status) != 0) return false;
@@ -792,7 +820,7 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
   Cursor cur(p, list, n, &ctl->psched, ctl);
   cur.seek(0);
   bool ok = true;
-  int last = -1;
+  int last = -1, pf_instr = -1;
   while (cur.i < n) {
     if (cur.pending) {  // an expert instruction: its weights follow from the routing
       if (!(ok = pr.wait_routing(cur.layer))) break;
@@ -808,7 +836,16 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
     }
     uint8_t* dst;
     unsigned long long* bar;
-    if (!(ok = pr.claim(&dst, &bar))) break;
+    // While the consumers wait on another SM with the ring full, HBM would
+    // idle: bring the rest of this instruction's weights into L2 (once per
+    // instruction), so the ring refills from L2 when the wait ends.
+    if (!(ok = pr.claim(&dst, &bar, [&]() {
+          if (!BATCHED && cur.i != pf_instr) {
+            pf_instr = cur.i;
+            cur.prefetch_rest(kL2AheadBytes);
+          }
+        })))
+      break;
     const uint32_t bytes = cur.stage_bytes();
     mbar_arrive_expect_tx(bar, bytes);
     if (cur.op == OP_ATTN) {
@@ -887,6 +924,7 @@ struct Consumer {
       const uint32_t target = p.epoch * (uint32_t)count;
       const uint32_t* c = p.counters + idx;
       if ((int32_t)(ld_acquire(c) - target) < 0) {
+        *(volatile int*)&ctl->waiting = 1;
         const uint64_t t0 = globaltimer();
         while (true) {
           if ((int32_t)(ld_acquire(c) - target) >= 0) break;
@@ -900,6 +938,7 @@ struct Consumer {
             break;
           }
         }
+        *(volatile int*)&ctl->waiting = 0;
       }
     }
     if (t == 0 && *(volatile int*)&ctl->dead) fail = true;
@@ -1941,6 +1980,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
       mbar_init(&ctl->empty[s], kConsumerWarps);
     }
     ctl->dead = 0;
+    ctl->waiting = 0;
     ctl->last = 0;
     ctl->moe_pub = 0;
     // a sticky error from an earlier step, or out-of-range inputs: do nothing
