@@ -1748,15 +1748,34 @@ struct Consumer {
   // (equal for every slot), cut into pieces at row boundaries.
   template <int HD, int G>
   __device__ __forceinline__ bool attn_run(const mk_instr& in, int layer, int sig_idx) {
-    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
-    if (tr) tr[1] = globaltimer();
+    constexpr int NP = HD / 64;  // rotation pairs per lane
+    // The schedule and the RoPE factors depend only on this step's lengths
+    // and positions, not on its activations: fetch the first piece's before
+    // the dependency wait.
     AttnSched sc;
     attn_sched(p, in, sc);
     const int j = in.a;
-    for (int64_t g = attn_slot_begin(sc, j), g1 = attn_slot_begin(sc, j + 1); g < g1;) {
+    const int64_t g0 = attn_slot_begin(sc, j), g1 = attn_slot_begin(sc, j + 1);
+    int rb = -1;  // sequence whose RoPE factors csr holds
+    float2 csr[NP];
+    if (g0 < g1) {
+      rb = attn_piece_at(sc, g0, j).b;
+      const float2* cs = p.rope + (size_t)p.positions[rb] * (HD / 2);
+#pragma unroll
+      for (int q = 0; q < NP; ++q) csr[q] = __ldg(cs + lane + 32 * q);
+    }
+    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
+    if (tr) tr[1] = globaltimer();
+    for (int64_t g = g0; g < g1;) {
       const AttnPiece pc = attn_piece_at(sc, g, j);
       g += pc.ub - pc.ua;
-      attn_piece<HD, G>(attn_geo(p, pc, layer, HD), layer, sig_idx);
+      if (pc.b != rb) {
+        rb = pc.b;
+        const float2* cs = p.rope + (size_t)p.positions[rb] * (HD / 2);
+#pragma unroll
+        for (int q = 0; q < NP; ++q) csr[q] = __ldg(cs + lane + 32 * q);
+      }
+      attn_piece<HD, G>(attn_geo(p, pc, layer, HD), layer, sig_idx, csr);
     }
     return true;
   }
@@ -1766,8 +1785,10 @@ struct Consumer {
   // and, in the piece that holds it, the new token's own K/V row.  The result
   // is an unnormalised partial (o, m, l) in log2 units; the last piece of the
   // row to finish merges all partials.
+  // csr: the RoPE factors (cos, sin) of this lane's rotation pairs at the
+  // sequence's position.
   template <int HD, int G>
-  __device__ __forceinline__ void attn_piece(const Attn& a, int layer, int sig_idx) {
+  __device__ __forceinline__ void attn_piece(const Attn& a, int layer, int sig_idx, const float2 (&csr)[HD / 64]) {
     constexpr int NP = HD / 64;    // rotation pairs per lane
     const int qd = p.nq * HD, kvd = p.nkv * HD;
     const float* qkv = p.qkv + (size_t)a.b * (qd + 2 * kvd);
@@ -1775,12 +1796,6 @@ struct Consumer {
     const int group = p.nq / p.nkv, nhg = group / G;
     const int q0 = a.kvh * group + a.hg * G;  // first query head
     const float qscale = 1.4426950408889634f * rsqrtf((float)HD);  // log2(e) / sqrt(hd)
-    float2 csr[NP];
-    if (a.active) {
-      const float2* cs = p.rope + (size_t)p.positions[a.b] * (HD / 2);
-#pragma unroll
-      for (int j = 0; j < NP; ++j) csr[j] = __ldg(cs + lane + 32 * j);
-    }
     if (a.active) {
       // -- prologue: q heads (qk-norm, RoPE, scale) and the new K/V row
       const int tasks = G + (a.owns_new ? 2 : 0);
