@@ -39,6 +39,11 @@ struct mk_handle {
   size_t region_bytes;
   size_t n_instr;
   uint32_t epoch;
+  // greedy decoding loop: the steps' tokens and lengths, per-sequence arg-max, logits
+  int32_t* loop_tok;
+  int32_t* loop_len;
+  unsigned long long* amax;
+  float* loop_logits;
 };
 
 namespace {
@@ -153,6 +158,9 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const char* trace_env = getenv("MK_TRACE");
   const bool tracing = trace_env && atoi(trace_env) > 0;
   const size_t o_trace = tracing ? cv.take(sizeof(uint64_t) * mk::kTraceStamps * instrs.size()) : 0;
+  const size_t o_ltok = cv.take(sizeof(int32_t) * B), o_llen = cv.take(sizeof(int32_t) * B);
+  const size_t o_amax = cv.take(sizeof(unsigned long long) * B);
+  const size_t o_llog = cv.take(sizeof(float) * (size_t)B * d.vocab);
   h->n_instr = tracing ? (size_t)n_instr : 0;
   h->region_bytes = cv.off;
   if (cudaMalloc(&h->region, h->region_bytes) != cudaSuccess) {
@@ -259,6 +267,10 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   p.offsets = (const int32_t*)(base + o_off);
   p.timeout_ns = d.wait_timeout_ns ? d.wait_timeout_ns : kDefaultTimeoutNs;
   p.trace = tracing ? (uint64_t*)(base + o_trace) : nullptr;
+  h->loop_tok = (int32_t*)(base + o_ltok);
+  h->loop_len = (int32_t*)(base + o_llen);
+  h->amax = (unsigned long long*)(base + o_amax);
+  h->loop_logits = (float*)(base + o_llog);
   const char* piece_env = getenv("MK_COPY_PIECE_KB");  // diagnostic knob: bytes per bulk copy
   p.copy_piece = piece_env && atoi(piece_env) > 0 ? (uint32_t)atoi(piece_env) * 1024u : mk::kDefaultCopyPiece;
   *out = h;
@@ -280,6 +292,61 @@ extern "C" int mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t
     return MK_ERR_CUDA;
   }
   h->epoch = p.epoch;
+  return MK_OK;
+}
+
+namespace {
+
+// Greedy loop: copy the first tokens and the lengths, clear the arg-max words.
+__global__ void greedy_init(const int32_t* tok0, const int32_t* len0, int B, int32_t* tok, int32_t* len,
+                            unsigned long long* amax) {
+  const int b = threadIdx.x;
+  if (b < B) {
+    tok[b] = tok0[b];
+    len[b] = len0[b];
+    amax[b] = 0ull;
+  }
+}
+
+// After a step: the arg-max token (the key's low word holds ~token) becomes the
+// next step's input and output, every sequence moves one position on.
+__global__ void greedy_advance(int B, int32_t* tok, int32_t* len, unsigned long long* amax, int32_t* out_tok) {
+  const int b = threadIdx.x;
+  if (b < B) {
+    const int token = (int)(0xFFFFFFFFu - (uint32_t)(amax[b] & 0xFFFFFFFFull));
+    out_tok[b] = token;
+    tok[b] = token;
+    len[b] += 1;
+    amax[b] = 0ull;
+  }
+}
+
+}  // namespace
+
+extern "C" int mk_decode_greedy(mk_handle* h, int n_steps, const int32_t* tokens, const int32_t* seq_lens,
+                                void* stream, int32_t* out_tokens, float* out_logits) {
+  if (!h || n_steps < 0 || !tokens || !seq_lens || (n_steps > 0 && !out_tokens)) return MK_ERR_INVALID_ARG;
+  if (n_steps == 0) return MK_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int B = h->d.batch;
+  greedy_init<<<1, 32, 0, st>>>(tokens, seq_lens, B, h->loop_tok, h->loop_len, h->amax);
+  if (cudaGetLastError() != cudaSuccess) return MK_ERR_CUDA;
+  for (int t = 0; t < n_steps; ++t) {
+    mk::Params p = h->p;
+    p.tokens = h->loop_tok;
+    p.positions = h->loop_len;
+    p.seq_lens = h->loop_len;
+    p.logits = (t == n_steps - 1 && out_logits) ? out_logits : h->loop_logits;
+    p.argmax = h->amax;
+    p.epoch = h->epoch + 1;
+    if (mk::launch_step(p, h->n_sm, st) != cudaSuccess) {
+      cudaGetLastError();
+      return MK_ERR_CUDA;
+    }
+    h->epoch = p.epoch;
+    greedy_advance<<<1, 32, 0, st>>>(B, h->loop_tok, h->loop_len, h->amax, out_tokens + (size_t)t * B);
+    if (cudaGetLastError() != cudaSuccess) return MK_ERR_CUDA;
+  }
   return MK_OK;
 }
 

@@ -60,6 +60,7 @@ struct Params {
   const int32_t* positions;
   const int32_t* seq_lens;
   float* logits;            // [B][V]
+  unsigned long long* argmax;  // greedy decoding: [B] packed (logit, token) maxima, or nullptr
   uint32_t epoch;
   uint64_t timeout_ns;
   uint64_t* trace;          // [n_instr][kTraceStamps] timestamps, or nullptr

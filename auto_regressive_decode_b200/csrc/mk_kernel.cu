@@ -52,6 +52,7 @@ struct Ctl {
   // MoE: the current layer's routing.  The consumers compute it; the
   // producer, which cannot stream expert weights before it exists, waits for
   // moe_pub == layer + 1.
+  unsigned long long amax[kMaxBatch];  // greedy decoding: an LM-head instruction's arg-max per sequence
   int moe_pub;
   int moe_count;                       // distinct picked experts (slots)
   int16_t moe_uniq[kMaxSel];           // expert of each slot, ascending
@@ -315,6 +316,14 @@ __device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, u
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Greedy decoding: a logit and its token packed so that the unsigned maximum
+// is the largest logit and, among equal logits, the lowest token id.
+__device__ __forceinline__ unsigned long long argmax_key(float y, int token) {
+  uint32_t u = __float_as_uint(y);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // order-preserving map of the float
+  return ((unsigned long long)u << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)token);
 }
 
 // Two fp32 values rounded to nearest-even bf16, `lo` in the low half.
@@ -1124,6 +1133,8 @@ struct Consumer {
     }
     // epilogue: fixed-order sum of the per-warp partials, then the op's output
     const int wpr = g.tile.tpr / 32, n = g.r1 - g.r0;
+    const bool amx = op == OP_LMHEAD && p.argmax;
+    unsigned long long best = 0ull;
     for (int i = t; i < n; i += kConsumerThreads) {
       const int row = g.r0 + i;
       if (GATED) {
@@ -1145,6 +1156,17 @@ struct Consumer {
         p.xres[(size_t)(2 * layer + 2) * BH + row] = resid + y;
       } else {
         p.logits[row] = y;
+        if (amx) best = max(best, argmax_key(y, row));
+      }
+    }
+    if (amx) {  // the instruction's arg-max: warps, then shared memory, then one global atomic
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, off));
+      if (lane == 0) atomicMax(&ctl->amax[0], best);
+      consumer_bar();
+      if (t == 0) {
+        atomicMax(p.argmax, ctl->amax[0]);
+        ctl->amax[0] = 0ull;
       }
     }
     return true;
@@ -1344,6 +1366,7 @@ struct Consumer {
     // accumulator elements i and i + 2 of lane l over the warps.
     const int q = t >> 6, l = (t >> 1) & 31, i = t & 1;
     const int lgq = l >> 2, b = 2 * (l & 3) + i;
+    const bool amx = op == OP_LMHEAD && p.argmax;
     float sc = 1.f;
     const int qkvw = p.nq * p.hd + 2 * p.nkv * p.hd;
 #pragma unroll
@@ -1400,11 +1423,19 @@ struct Consumer {
                   p.moe_router[((size_t)layer * B + b) * p.E + row] = y;
                 } else {
                   p.logits[(size_t)b * p.V + row] = y;
+                  if (amx) atomicMax(&ctl->amax[b], argmax_key(y, row));
                 }
               }
             }
           }
         }
+      }
+    }
+    if (amx) {  // the instruction's arg-max per sequence (shared atomics above), one global atomic each
+      consumer_bar();
+      if (t < B) {
+        atomicMax(p.argmax + t, ctl->amax[t]);
+        ctl->amax[t] = 0ull;
       }
     }
     return true;
@@ -1997,6 +2028,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
     ctl->dead = 0;
     ctl->waiting = 0;
     ctl->last = 0;
+    for (int b = 0; b < kMaxBatch; ++b) ctl->amax[b] = 0ull;
     ctl->moe_pub = 0;
     // a sticky error from an earlier step, or out-of-range inputs: do nothing
     int bad = ld_relaxed_i32(p.status) != 0;

@@ -65,6 +65,7 @@ def _load():
         "mk_create": (_i32, [ctypes.POINTER(mk_model_desc), ctypes.POINTER(mk_weights), ctypes.POINTER(mk_kv),
                              ctypes.POINTER(H)]),
         "mk_decode_step": (_i32, [H, _P, _P, _P, _P, _P]),
+        "mk_decode_greedy": (_i32, [H, _i32, _P, _P, _P, _P, _P]),
         "mk_get_status": (_i32, [H, _P]),
         "mk_destroy": (_i32, [H]),
         "mk_status_string": (ctypes.c_char_p, [_i32]),
@@ -94,6 +95,7 @@ lib = _load()
 # Same names as the C ABI -----------------------------------------------------------------------
 mk_create = lib.mk_create
 mk_decode_step = lib.mk_decode_step
+mk_decode_greedy = lib.mk_decode_greedy
 mk_get_status = lib.mk_get_status
 mk_destroy = lib.mk_destroy
 mk_read_state = lib.mk_read_state
@@ -223,6 +225,12 @@ class Decoder:
         s = (stream or self.torch.cuda.current_stream()).cuda_stream
         check(mk_decode_step(self.h, tokens.data_ptr(), positions.data_ptr(), seq_lens.data_ptr(), s,
                              logits.data_ptr()), "mk_decode_step")
+
+    def greedy(self, n_steps, tokens, seq_lens, out_tokens, logits=None, stream=None):
+        """n_steps greedy steps on the device (asynchronous); out_tokens int32 [n_steps][B] device tensor."""
+        s = (stream or self.torch.cuda.current_stream()).cuda_stream
+        check(mk_decode_greedy(self.h, n_steps, tokens.data_ptr(), seq_lens.data_ptr(), s, out_tokens.data_ptr(),
+                               None if logits is None else logits.data_ptr()), "mk_decode_greedy")
 
     def status(self, stream=None):
         s = (stream or self.torch.cuda.current_stream()).cuda_stream

@@ -348,12 +348,30 @@ def run_mk(args, cfg, rank, world):
             dec.step(all_tok[i], all_len[i], all_len[i], logits)
             distinct.append(int(dec.routing()[3].sum()))
 
+    # ---- on-device greedy decoding: K steps in one call, each step's arg-max fed back on the device
+    # (after the MoE replay: the loop rewrites cache rows below S0 to make room)
+    picks = torch.empty((args.steps, B), dtype=torch.int32, device=dev)
+    g_len = torch.from_numpy(np.maximum(S0 - args.steps, 0).astype(np.int32)).to(dev)  # room for K steps
+    g_tok = all_tok[0].clone()
+    dec.greedy(3, g_tok, g_len, picks)  # warm-up
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    dec.greedy(args.steps, g_tok, g_len, picks)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    greedy_ms = e0.elapsed_time(e1)
+    st = dec.status()
+    if st != 0:
+        raise RuntimeError(f"device status {mk.mk_status_string(st)}")
+
     # ---- max over ranks
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    t = torch.tensor([total_ms, e2e_ms, greedy_ms], dtype=torch.float64, device=dev)
     if world > 1:
         import torch.distributed as dist
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms, greedy_ms = float(t[0]), float(t[1]), float(t[2])
     dec.close()
     if rank != 0:
         return
@@ -384,6 +402,8 @@ def run_mk(args, cfg, rank, world):
                      else "fallback", "traffic": traffic, "kernel": "mk_persistent"},
         "e2e": {"value": e2e_tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 3 * 4 * B,
                 "d2h_bytes_per_step": 4 * B * V},
+        "greedy_loop": {"value": world * B * args.steps / (greedy_ms / 1e3), "unit": "tokens/s",
+                        "note": "mk_decode_greedy: K steps in one call, arg-max fed back on the device"},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
     }

@@ -107,6 +107,25 @@ int mk_create(const mk_model_desc* desc, const mk_weights* weights, const mk_kv*
 int mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions, const int32_t* seq_lens,
                    void* stream, float* out_logits);
 
+/*
+ * On-device greedy decoding: n_steps decode steps back to back on `stream`,
+ * with no host round trip between them.  Step t runs every sequence b on
+ * token x_t[b] at position and cache index seq_lens[b] + t (appending its
+ * K/V there), then picks x_{t+1}[b] = argmax of its logits (the largest
+ * logit; among equal logits the lowest token id).
+ *   tokens     device int32[batch]: x_0, the first step's tokens
+ *   seq_lens   device int32[batch]: cached tokens before the first step
+ *              (positions equal lengths throughout; both arrays are only read)
+ *   out_tokens device int32[n_steps][batch]: x_1 .. x_{n_steps}
+ *   out_logits device fp32[batch][vocab] for the last step's logits, or NULL
+ * Asynchronous on `stream`; device-side errors (e.g. a length reaching
+ * max_ctx, MK_ERR_RANGE) are reported by mk_get_status.  Each step is the
+ * same kernel as mk_decode_step; the pick folds the LM head's outputs into
+ * per-sequence maxima on the device and a one-warp kernel advances the state.
+ */
+int mk_decode_greedy(mk_handle* h, int n_steps, const int32_t* tokens, const int32_t* seq_lens, void* stream,
+                     int32_t* out_tokens, float* out_logits);
+
 /* Synchronise `stream` and return the device-side status of the last steps
  * (MK_OK, MK_ERR_DEVICE_TIMEOUT or MK_ERR_RANGE).  A failure is cleared and
  * the dependency counters are reset, so the handle is usable again. */

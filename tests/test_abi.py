@@ -18,7 +18,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("mk_create", "mk_decode_step", "mk_get_status", "mk_destroy", "mk_status_string",
-                     "mk_read_state", "mk_decode_step_noalloc", "mk_plan_create"):
+                     "mk_read_state", "mk_decode_step_noalloc", "mk_decode_greedy", "mk_plan_create"):
         assert required in names
 
 
@@ -38,6 +38,7 @@ def test_status_strings_and_null_handles():
     assert mk.mk_get_status(None, None) == mk.MK_ERR_INVALID_ARG
     assert mk.mk_decode_step(None, None, None, None, None, None) == mk.MK_ERR_INVALID_ARG
     assert mk.mk_create(None, None, None, None) == mk.MK_ERR_INVALID_ARG
+    assert mk.mk_decode_greedy(None, 1, None, None, None, None, None) == mk.MK_ERR_INVALID_ARG
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
