@@ -85,6 +85,12 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   // pointers: present and 16-byte aligned
   if (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(kv->k) || !aligned16(kv->v))
     return w->embed && w->final_norm && kv->k && kv->v ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
+  if (kv->block_table) {  // paged cache: pages hold whole attention stages
+    if (kv->page_size <= 0 || kv->n_pages <= 0) return MK_ERR_INVALID_ARG;
+    if (kv->page_size % mk::attn_stage_positions(d.head_dim) ||
+        (int64_t)d.n_layers * kv->n_pages * d.n_kv_heads * kv->page_size >= (1ll << 31))
+      return MK_ERR_UNSUPPORTED;
+  }
   if (!d.tied_embeddings && !aligned16(w->lm_head)) return w->lm_head ? MK_ERR_UNSUPPORTED : MK_ERR_INVALID_ARG;
   for (int l = 0; l < d.n_layers; ++l) {
     const mk_layer_weights& lw = w->layers[l];
@@ -117,6 +123,10 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const int n_cnt = mk_plan_n_counters(plan);
   int32_t chunk = 0, n_chunks = 0;
   mk_plan_attn_chunk(plan, &chunk, &n_chunks);
+  if (kv->block_table && chunk != mk::attn_stage_positions(d.head_dim)) {  // a stage must not straddle pages
+    mk_plan_destroy(plan);
+    return MK_ERR_UNSUPPORTED;
+  }
   mk_plan_destroy(plan);
 
   mk_handle* h = new (std::nothrow) mk_handle();
@@ -240,6 +250,12 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   p.layers = (const mk::LayerPtrs*)(base + o_lay);
   p.kc = (uint16_t*)kv->k;
   p.vc = (uint16_t*)kv->v;
+  if (kv->block_table) {
+    p.bt = kv->block_table;
+    p.page = kv->page_size;
+    p.n_pages = kv->n_pages;
+    p.bt_stride = (d.max_ctx + kv->page_size - 1) / kv->page_size;
+  }
   p.rope = (const float2*)(base + o_rope);
   p.tmaps = n_tmaps ? base + o_tmap : nullptr;
   p.xres = (float*)(base + o_xres);

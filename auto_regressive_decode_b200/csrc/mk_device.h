@@ -24,8 +24,10 @@ struct Params {
   const uint16_t* final_norm;
   const uint16_t* lm_head;
   const LayerPtrs* layers;  // [L]
-  uint16_t* kc;             // [L][B][nkv][T][hd]
+  uint16_t* kc;             // [L][B][nkv][T][hd], or paged: [L][n_pages][nkv][page][hd]
   uint16_t* vc;
+  const int32_t* bt;        // paged cache: block table [B][bt_stride], else nullptr
+  int page, n_pages, bt_stride;
   const float2* rope;       // [T][hd/2] (cos, sin)
   // batch > 1: TMA tensor maps (CUtensorMap, 128 bytes each) of every weight
   // matrix: [layer][wq wk wv wo w_gate w_up w_down], then the LM head, the K

@@ -508,8 +508,18 @@ struct Attn {
   int b, kvh, hg, S, p0, n_cached, nsub, P;
   int c, npieces;  // index of the piece within its row, pieces of the row
   bool active, owns_new;
-  size_t cache_base;  // element offset of (layer, b, kvh, position p0)
 };
+
+// Row (of head_dim elements) of (layer, sequence b, KV head, position) in
+// the K or V cache: contiguous [L][B][nkv][T], or paged [L][n_pages][nkv][page]
+// through the block table.
+__device__ __forceinline__ int64_t kv_row(const Params& p, int layer, int b, int kvh, int pos) {
+  if (p.bt) {
+    const int page = __ldg(p.bt + (size_t)b * p.bt_stride + pos / p.page);
+    return (((int64_t)layer * p.n_pages + page) * p.nkv + kvh) * p.page + pos % p.page;
+  }
+  return (((int64_t)layer * p.B + b) * p.nkv + kvh) * p.T + pos;
+}
 
 __device__ __forceinline__ Attn attn_geo(const Params& p, const AttnPiece& pc, int layer, int head_dim) {
   Attn a;
@@ -527,7 +537,6 @@ __device__ __forceinline__ Attn attn_geo(const Params& p, const AttnPiece& pc, i
   a.nsub = (a.n_cached + a.P - 1) / a.P;
   a.c = pc.slot_in_row;
   a.npieces = pc.n_pieces;
-  a.cache_base = ((((size_t)layer * p.B + a.b) * p.nkv + a.kvh) * p.T + a.p0) * head_dim;
   return a;
 }
 
@@ -740,7 +749,7 @@ struct Cursor {
   __device__ __forceinline__ void attn_box(const uint8_t** map, int* row) const {
     const Params& p = *pp;
     *map = p.tmaps + ((size_t)p.L * kTmapsPerLayer + 1 + kv) * 128;
-    *row = (int)(a.cache_base / (size_t)p.hd) + sub * a.P;
+    *row = (int)kv_row(p, layer, a.b, a.kvh, a.p0 + sub * a.P);
   }
 
   __device__ __forceinline__ uint32_t stage_bytes() const {
@@ -1870,7 +1879,7 @@ struct Consumer {
           // the new row (bf16): kept for this instruction's own use, and
           // appended at index S by head group 0 (every group computes the
           // same bits)
-          uint16_t* cache = (is_v ? p.vc : p.kc) + a.cache_base + (size_t)(a.S - a.p0) * HD;
+          uint16_t* cache = (is_v ? p.vc : p.kc) + (size_t)kv_row(p, layer, a.b, a.kvh, a.S) * HD;
           uint16_t* keep = is_v ? ctl->vnew : ctl->knew;
 #pragma unroll
           for (int j = 0; j < NP; ++j) {
@@ -2037,6 +2046,14 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
       if (S < 0 || S >= p.T || pos < 0 || pos >= p.T || tok < 0 || tok >= p.V) {
         set_status(p, MK_ERR_RANGE, b);
         bad = 1;
+      }
+      // paged cache: every page the step reads or writes is in the pool
+      for (int j = 0; p.bt && !bad && j <= S / p.page; ++j) {
+        const int pg = p.bt[(size_t)b * p.bt_stride + j];
+        if (pg < 0 || pg >= p.n_pages) {
+          set_status(p, MK_ERR_RANGE, b);
+          bad = 1;
+        }
       }
     }
     // the swizzled TMA boxes of the batched GEMV need 1024-byte aligned slots

@@ -53,6 +53,12 @@ bool encode_one(EncodeTiledFn enc, const void* w, int64_t rows, int K, uint8_t* 
   return true;
 }
 
+// Rows of head_dim elements in each KV cache (or page pool).
+int64_t kv_cache_rows(const mk_model_desc& d, const mk_kv& kv) {
+  return kv.block_table ? (int64_t)d.n_layers * kv.n_pages * d.n_kv_heads * kv.page_size
+                        : (int64_t)d.n_layers * d.batch * d.n_kv_heads * d.max_ctx;
+}
+
 }  // namespace
 
 cudaError_t encode_tmaps(const mk_model_desc& d, const mk_weights& w, const mk_kv& kv, uint8_t* out) {
@@ -61,7 +67,7 @@ cudaError_t encode_tmaps(const mk_model_desc& d, const mk_weights& w, const mk_k
   if (!batched(d)) {  // CUDA-core GEMVs read weights with 1-D copies: only the KV caches' maps
     memset(out, 0, (size_t)(kTmapsPerLayer * d.n_layers + 3) * 128);
     uint8_t* g = out + (size_t)d.n_layers * kTmapsPerLayer * 128;
-    const int64_t kv_rows = (int64_t)d.n_layers * d.batch * d.n_kv_heads * d.max_ctx;
+    const int64_t kv_rows = kv_cache_rows(d, kv);
     const int P = attn_stage_positions(d.head_dim);
     return encode_one(enc, kv.k, kv_rows, d.head_dim, g + 128, P, d.head_dim / 64) &&
                    encode_one(enc, kv.v, kv_rows, d.head_dim, g + 256, P, d.head_dim / 64)
@@ -88,7 +94,7 @@ cudaError_t encode_tmaps(const mk_model_desc& d, const mk_weights& w, const mk_k
   if (!encode_one(enc, lm, d.vocab, H, g)) return cudaErrorInvalidValue;
   // KV caches: rows are (layer, sequence, KV head, position), head_dim columns;
   // a box is one attention stage of positions
-  const int64_t kv_rows = (int64_t)d.n_layers * d.batch * d.n_kv_heads * d.max_ctx;
+  const int64_t kv_rows = kv_cache_rows(d, kv);
   const int P = attn_stage_positions(d.head_dim);
   if (!encode_one(enc, kv.k, kv_rows, d.head_dim, g + 128, P, d.head_dim / 64) ||
       !encode_one(enc, kv.v, kv_rows, d.head_dim, g + 256, P, d.head_dim / 64))

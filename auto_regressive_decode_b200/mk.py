@@ -49,7 +49,7 @@ class mk_weights(ctypes.Structure):
 
 
 class mk_kv(ctypes.Structure):
-    _fields_ = [("k", _P), ("v", _P)]
+    _fields_ = [("k", _P), ("v", _P), ("block_table", _P), ("page_size", _i32), ("n_pages", _i32)]
 
 
 class mk_instr(ctypes.Structure):
@@ -198,10 +198,12 @@ class Decoder:
     """Owns one mk_handle.  weights: dict of device tensors (see include/mk.h for shapes);
     k_cache / v_cache: device bf16 tensors [L][B][n_kv][max_ctx][hd]."""
 
-    def __init__(self, cfg, weights, k_cache, v_cache, wait_timeout_ns=0):
+    def __init__(self, cfg, weights, k_cache, v_cache, wait_timeout_ns=0, block_table=None, page_size=0):
+        """block_table (device int32 [B][ceil(max_ctx/page_size)]) with page_size: k_cache / v_cache are
+        page pools [L][n_pages][n_kv][page_size][hd]."""
         import torch
         self.cfg = cfg
-        self._keep = (weights, k_cache, v_cache)
+        self._keep = (weights, k_cache, v_cache, block_table)
         self.desc = model_desc(cfg, wait_timeout_ns=wait_timeout_ns)
         L = cfg.n_layers
         layers = (mk_layer_weights * L)()
@@ -214,7 +216,10 @@ class Decoder:
                 setattr(layers[l], name, ptr(lw.get(name)))
         self._layers = layers
         w = mk_weights(ptr(weights["embed"]), ptr(weights["final_norm"]), ptr(weights.get("lm_head")), layers)
-        kv = mk_kv(k_cache.data_ptr(), v_cache.data_ptr())
+        if block_table is None:
+            kv = mk_kv(k_cache.data_ptr(), v_cache.data_ptr(), None, 0, 0)
+        else:
+            kv = mk_kv(k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(), page_size, k_cache.shape[1])
         h = _P()
         check(mk_create(ctypes.byref(self.desc), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(h)), "mk_create")
         self.h = h
@@ -283,7 +288,7 @@ def weight_structs(cfg, weights, k_cache, v_cache):
     lm = weights.get("lm_head")
     w = mk_weights(weights["embed"].data_ptr(), weights["final_norm"].data_ptr(),
                    None if lm is None else lm.data_ptr(), layers)
-    kv = mk_kv(k_cache.data_ptr(), v_cache.data_ptr())
+    kv = mk_kv(k_cache.data_ptr(), v_cache.data_ptr(), None, 0, 0)
     return model_desc(cfg), w, kv, (layers, weights, k_cache, v_cache)
 
 

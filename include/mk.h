@@ -72,10 +72,21 @@ typedef struct mk_weights {
   const mk_layer_weights* layers;
 } mk_weights;
 
-/* KV cache (device, bf16, caller-owned): k and v are each
- * [n_layers][batch][n_kv_heads][max_ctx][head_dim]. */
+/* KV cache (device, bf16, caller-owned).
+ * Contiguous (block_table == NULL): k and v are each
+ *   [n_layers][batch][n_kv_heads][max_ctx][head_dim].
+ * Paged (block_table != NULL): k and v are page pools
+ *   [n_layers][n_pages][n_kv_heads][page_size][head_dim], and block_table
+ *   (device int32 [batch][ceil(max_ctx / page_size)], caller-owned, may be
+ *   rewritten between steps) maps page j of a sequence (positions
+ *   [j*page_size, (j+1)*page_size)) to a pool page.  page_size must be a
+ *   multiple of one attention stage, 32768 / (2*head_dim) positions (128 at
+ *   head_dim 128); every page a step reads or writes must be < n_pages
+ *   (checked on the device: MK_ERR_RANGE). */
 typedef struct mk_kv {
   void *k, *v;
+  const int32_t* block_table;
+  int32_t page_size, n_pages;
 } mk_kv;
 
 typedef struct mk_handle mk_handle;
