@@ -272,7 +272,26 @@ def run_mk(args, cfg, rank, world):
     toks = fx.tokens(cfg, seed)
     w = device_model(cfg, seed)
     kc, vc = device_caches(cfg, S0, seed)
-    dec = mk.Decoder(cfg, w, kc, vc)
+    if args.paged:
+        # the same cache as a page pool: one attention stage per page, pages in a seeded random order
+        page = 32768 // (2 * cfg.head_dim)
+        stride = -(-cfg.max_ctx // page)
+        table = np.random.default_rng(seed).permutation(cfg.batch * stride).reshape(cfg.batch, stride)
+        pools = []
+        for c in (kc, vc):
+            L, B_, nkv, T, hd = c.shape
+            pool = torch.empty((L, cfg.batch * stride, nkv, page, hd), dtype=c.dtype, device=c.device)
+            for b in range(B_):
+                for j in range(stride):
+                    lo, hi = j * page, min(T, (j + 1) * page)
+                    pool[:, int(table[b, j]), :, :hi - lo] = c[:, b, :, lo:hi]
+            pools.append(pool)
+        del kc, vc
+        kc, vc = pools
+        d_table = torch.from_numpy(table.astype(np.int32)).to(dev)
+        dec = mk.Decoder(cfg, w, kc, vc, block_table=d_table, page_size=page)
+    else:
+        dec = mk.Decoder(cfg, w, kc, vc)
     B, V = cfg.batch, cfg.vocab
     n_total = args.warmup + args.steps
     # per-step inputs, resident on the device (teacher forcing; positions wrap after cfg.steps)
@@ -391,7 +410,9 @@ def run_mk(args, cfg, rank, world):
         "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded random-init weights and KV cache, uniform token ids)",
-        "config": dict(workload_config(cfg), parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
+        "config": dict(workload_config(cfg), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
+                       **({"kv_layout": f"paged, {32768 // (2 * cfg.head_dim)}-position pages in a shuffled pool"}
+                          if args.paged else {})),
         "step_latency_ms": {"median": statistics.median(per_step_ms), "p10": float(np.percentile(per_step_ms, 10)),
                             "p90": float(np.percentile(per_step_ms, 90))},
         "bytes_per_step": bytes_step,
@@ -421,6 +442,7 @@ def main():
     ap.add_argument("--config", default="dense-8b", choices=sorted(fx.CONFIGS))
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--paged", action="store_true", help="run the KV cache as a paged pool (block table)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: the config with this many layers (same shapes); not a bench line")
     args = ap.parse_args()
