@@ -205,6 +205,21 @@ def cpu_baseline(cfg, seed=fx.DEFAULT_SEED, max_layers=2):
             "step_s": step_s}
 
 
+def max_over_ranks(values, world, device="cpu"):
+    """Each value's maximum over the ranks (a job's time is its slowest rank's); identity for one rank."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_tokens_per_s(world, batch, steps, total_ms):
+    """Whole-job tokens/s: every rank (replica) decodes `batch` tokens per step."""
+    return world * batch * steps / (total_ms / 1e3)
+
+
 def run_reference(args, cfg, rank):
     """The oracle timed on the host: each step is one layer of the decode step (a bounded sample);
     the step time is the median layer time x L plus the LM head, timed once."""
@@ -386,18 +401,14 @@ def run_mk(args, cfg, rank, world):
         raise RuntimeError(f"device status {mk.mk_status_string(st)}")
 
     # ---- max over ranks
-    t = torch.tensor([total_ms, e2e_ms, greedy_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, greedy_ms = float(t[0]), float(t[1]), float(t[2])
+    total_ms, e2e_ms, greedy_ms = max_over_ranks([total_ms, e2e_ms, greedy_ms], world, dev)
     dec.close()
     if rank != 0:
         return
 
     ms = total_ms / args.steps
-    tok_s = world * B * args.steps / (total_ms / 1e3)
-    e2e_tok_s = world * B * args.steps / (e2e_ms / 1e3)
+    tok_s = job_tokens_per_s(world, B, args.steps, total_ms)
+    e2e_tok_s = job_tokens_per_s(world, B, args.steps, e2e_ms)
     lens = [S0 + (k % cfg.steps) for k in range(args.warmup, n_total)]
     bytes_step = weight_bytes_read(cfg) + float(np.mean([kv_bytes(cfg, s) for s in lens]))
     if cfg.n_experts:
@@ -423,12 +434,12 @@ def run_mk(args, cfg, rank, world):
                      else "fallback", "traffic": traffic, "kernel": "mk_persistent"},
         "e2e": {"value": e2e_tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 3 * 4 * B,
                 "d2h_bytes_per_step": 4 * B * V},
-        "greedy_loop": {"value": world * B * args.steps / (greedy_ms / 1e3), "unit": "tokens/s",
+        "greedy_loop": {"value": job_tokens_per_s(world, B, args.steps, greedy_ms), "unit": "tokens/s",
                         "note": "mk_decode_greedy: K steps in one call, arg-max fed back on the device"},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:  # the oracle baseline: rank 0 at one GPU only
         base = cpu_baseline(cfg)
         out["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
     print(json.dumps(out), flush=True)
