@@ -38,6 +38,17 @@ MUTANTS = [
     ("qk-norm gain", "ora_rmsnorm(k + (size_t)h * hd, hd, W->k_norm", "ora_rmsnorm(k + (size_t)h * hd, hd, W->q_norm",
      ["test_whole_step_matches_torch_reference"]),
     ("moe weighting", "acc[i] += wsel[j] * o[i];", "acc[i] += o[i];", ["test_moe_step_matches_torch_reference"]),
+    ("silu sign", "return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));", ["test_silu_values"]),
+    ("mlp norm gain", "ora_rmsnorm(xb, H, W->mlp_norm,", "ora_rmsnorm(xb, H, W->attn_norm,",
+     ["test_whole_step_matches_torch_reference"]),
+    ("mlp residual", "xn, o);\n      for (int i = 0; i < H; ++i) xb[i] += o[i];",
+     "xn, o);\n      for (int i = 0; i < H; ++i) xb[i] = o[i];", ["test_whole_step_matches_torch_reference"]),
+    ("final norm skipped", "ora_gemv(m->lm_head, m->d.vocab, H, xn, logits);",
+     "ora_gemv(m->lm_head, m->d.vocab, H, x, logits);", ["test_whole_step_matches_torch_reference"]),
+    ("key rope position", "ora_rope(k + (size_t)h * hd, hd, pos, d->rope_theta);",
+     "ora_rope(k + (size_t)h * hd, hd, pos + 1, d->rope_theta);", ["test_whole_step_matches_torch_reference"]),
+    ("router input", "ora_gemv(W->router, E, H, xn, r);", "ora_gemv(W->router, E, H, xb, r);",
+     ["test_moe_step_matches_torch_reference"]),
 ]
 
 
