@@ -97,8 +97,20 @@ typedef struct mk_handle mk_handle;
  * counters, activation scratch, RoPE cos/sin table) on the current device.
  * Weight and cache pointers are borrowed: they must stay valid until
  * mk_destroy and are never freed by the library.
- * Returns MK_ERR_UNSUPPORTED for shapes the kernel cannot run (e.g. a matrix
- * row wider than one pipeline stage, head_dim not 64/128, misaligned pointers).
+ * Returns MK_ERR_UNSUPPORTED for shapes the kernel cannot run:
+ *   - head_dim not 64 or 128; n_q_heads not 1, 2, 4 or 8 times n_kv_heads;
+ *   - batch > 8;
+ *   - hidden above 8192 (a gate/up row pair of the norm-fused GEMVs must fit
+ *     one 32 KB pipeline stage); a GEMV width (hidden, n_q_heads*head_dim,
+ *     ffn_dim) not a multiple of 8, or too wide to cut into at most four
+ *     slices of one stage each (e.g. ffn_dim above 65536);
+ *   - batch > 1 or MoE (the tensor-core kernel) with hidden, n_q_heads*head_dim,
+ *     ffn_dim or expert_ffn_dim not a multiple of 64;
+ *   - MoE with more than 256 experts, top_k > 8, or batch * top_k > 64;
+ *   - max_ctx * head_dim above 2^31; misaligned pointers; a device without
+ *     cooperative launch or the shared memory the kernel needs.
+ * MK_ERR_INVALID_ARG for a malformed description (non-positive sizes, a
+ * negative eps, a non-positive rope_theta, top_k outside 1..n_experts).
  */
 int mk_create(const mk_model_desc* desc, const mk_weights* weights, const mk_kv* kv, mk_handle** out);
 

@@ -176,6 +176,23 @@ def test_invalid_and_unsupported_shapes():
         mk.Plan(mk.model_desc(base), 0)
 
 
+@pytest.mark.parametrize("kw,ok", [
+    ({"hidden": 8192}, True), ({"hidden": 8200}, False),           # a gate/up row pair fits one 32 KB stage
+    ({"ffn_dim": 65536}, True), ({"ffn_dim": 65544}, False),       # at most four one-stage slices
+    ({"ffn_dim": 700}, False),                                     # widths are multiples of 8
+    ({"n_q_heads": 4, "n_kv_heads": 3}, False), ({"n_q_heads": 32, "n_kv_heads": 2}, False),  # group 1/2/4/8
+    ({"batch": 8, "ffn_dim": 704}, True), ({"batch": 9, "ffn_dim": 704}, False),
+])
+def test_documented_shape_limits(kw, ok):
+    # the limits include/mk.h states for mk_create (host-side lowering, no GPU)
+    cfg = fx.CONFIGS["tiny"].replace(**kw)
+    if ok:
+        mk.Plan(mk.model_desc(cfg), 8)
+    else:
+        with pytest.raises(mk.MkError):
+            mk.Plan(mk.model_desc(cfg), 8)
+
+
 def test_batched_shapes_need_64_column_blocks():
     # the tensor-core GEMV views K (hidden, q width, ffn width) as blocks of 64 columns
     base = fx.CONFIGS["tiny"].replace(batch=4)
