@@ -88,7 +88,14 @@ def _setup(lib):
     lib.ora_decode_step.restype = _I
     lib.ora_decode_step.argtypes = [ctypes.POINTER(_Model), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
     lib.ora_lm_head.argtypes = [ctypes.POINTER(_Model), _P, _P]
-    for f in ("ora_rmsnorm", "ora_rope", "ora_gemv", "ora_attention", "ora_swiglu", "ora_topk", "ora_lm_head"):
+    lib.ora_e4m3_to_double.restype = _D
+    lib.ora_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    lib.ora_e2m1_to_double.restype = _D
+    lib.ora_e2m1_to_double.argtypes = [ctypes.c_uint8]
+    lib.ora_gemv_fp8.argtypes = [_P, _P, _I, _I, _I, _P, _P]
+    lib.ora_gemv_nvfp4.argtypes = [_P, _P, ctypes.c_float, _I, _I, _P, _P]
+    for f in ("ora_rmsnorm", "ora_rope", "ora_gemv", "ora_attention", "ora_swiglu", "ora_topk", "ora_lm_head",
+              "ora_gemv_fp8", "ora_gemv_nvfp4"):
         getattr(lib, f).restype = None
     return lib
 
@@ -141,6 +148,33 @@ def gemv(w, x, L=None):
     w = _u16(w); x = _f64(x)
     y = np.empty(w.shape[0], dtype=np.float64)
     (L or lib()).ora_gemv(_ptr(w), w.shape[0], w.shape[1], _ptr(x), _ptr(y))
+    return y
+
+
+def e4m3_to_double(code: int, L=None) -> float:
+    return (L or lib()).ora_e4m3_to_double(int(code))
+
+
+def e2m1_to_double(nibble: int, L=None) -> float:
+    return (L or lib()).ora_e2m1_to_double(int(nibble))
+
+
+def gemv_fp8(w, scale, block, x, L=None):
+    """w uint8 [rows][cols] E4M3 codes, scale fp32 [rows][ceil(cols / block)] -> y [rows]."""
+    w = np.ascontiguousarray(w, dtype=np.uint8); scale = np.ascontiguousarray(scale, dtype=np.float32)
+    x = _f64(x)
+    y = np.empty(w.shape[0], dtype=np.float64)
+    (L or lib()).ora_gemv_fp8(_ptr(w), _ptr(scale), w.shape[0], w.shape[1], int(block), _ptr(x), _ptr(y))
+    return y
+
+
+def gemv_nvfp4(w, scale, tensor_scale, x, L=None):
+    """w uint8 [rows][cols / 2] E2M1 pairs, scale uint8 [rows][cols / 16] E4M3 -> y [rows]."""
+    w = np.ascontiguousarray(w, dtype=np.uint8); scale = np.ascontiguousarray(scale, dtype=np.uint8)
+    x = _f64(x)
+    rows, cols = w.shape[0], 2 * w.shape[1]
+    y = np.empty(rows, dtype=np.float64)
+    (L or lib()).ora_gemv_nvfp4(_ptr(w), _ptr(scale), float(tensor_scale), rows, cols, _ptr(x), _ptr(y))
     return y
 
 

@@ -76,6 +76,46 @@ void ora_gemv(const uint16_t* w, int rows, int cols, const double* x, double* y)
   }
 }
 
+/* ---- low-bit weights ---------------------------------------------------------
+ * The pages name fp8 and nvfp4 weight streams (per-block scales) without
+ * fixing a block shape; the decodes below are the OCP 8-bit and 4-bit
+ * floating-point definitions, written out field by field. */
+double ora_e4m3_to_double(uint8_t code) {
+  const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double mag = e == 0 ? ldexp((double)m / 8.0, 1 - 7) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -mag : mag;
+}
+
+double ora_e2m1_to_double(uint8_t nibble) {
+  const int sign = (nibble >> 3) & 1, e = (nibble >> 1) & 3, m = nibble & 1;
+  const double mag = e == 0 ? (double)m / 2.0 : ldexp(1.0 + (double)m / 2.0, e - 1);
+  return sign ? -mag : mag;
+}
+
+void ora_gemv_fp8(const uint8_t* w, const float* scale, int rows, int cols, int block, const double* x, double* y) {
+  const int nb = (cols + block - 1) / block;
+  for (int r = 0; r < rows; ++r) {
+    double acc = 0.0;
+    for (int c = 0; c < cols; ++c)
+      acc += ora_e4m3_to_double(w[(size_t)r * cols + c]) * (double)scale[(size_t)r * nb + c / block] * x[c];
+    y[r] = acc;
+  }
+}
+
+void ora_gemv_nvfp4(const uint8_t* w, const uint8_t* scale, float tensor_scale, int rows, int cols,
+                    const double* x, double* y) {
+  for (int r = 0; r < rows; ++r) {
+    double acc = 0.0;
+    for (int c = 0; c < cols; ++c) {
+      const uint8_t byte = w[(size_t)r * (cols / 2) + c / 2];
+      const double v = ora_e2m1_to_double(c % 2 ? byte >> 4 : byte & 15);
+      acc += v * ora_e4m3_to_double(scale[(size_t)r * (cols / 16) + c / 16]) * (double)tensor_scale * x[c];
+    }
+    y[r] = acc;
+  }
+}
+
 /* SiLU (Hendrycks & Gimpel; Elfwing et al.): z * sigmoid(z) = z / (1 + e^-z). */
 double ora_silu(double z) { return z / (1.0 + exp(-z)); }
 

@@ -72,6 +72,22 @@ void ora_swiglu(const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_
                 const double* xn, double* y);
 void ora_topk(const double* logits, int n, int k, int32_t* sel, double* w);
 
+/* ---- low-bit weights (fp8 / nvfp4 weight streaming; not used by the decode step yet) ---------- */
+/* Exact decodes to double.  E4M3 is the OCP 8-bit floating-point format (sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent 0 is subnormal; 0x7F and 0xFF are NaN; no infinities; largest
+ * finite 448).  E2M1 is the OCP 4-bit format of the low nibble (sign, 2 exponent bits with bias 1,
+ * 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6). */
+double ora_e4m3_to_double(uint8_t code);
+double ora_e2m1_to_double(uint8_t nibble);
+/* fp8 weights with block scales: W[r][c] = e4m3(w[r][c]) * scale[r][c / block] (scale fp32
+ * [rows][ceil(cols / block)]); y_r = sum_c W[r][c] x_c in column order. */
+void ora_gemv_fp8(const uint8_t* w, const float* scale, int rows, int cols, int block, const double* x, double* y);
+/* nvfp4 weights: two E2M1 codes per byte (column 2j in the low nibble, 2j + 1 in the high one),
+ * one E4M3 scale per 16 columns (scale [rows][cols / 16]) and one fp32 scale for the whole matrix:
+ * W[r][c] = e2m1(code) * e4m3(scale[r][c / 16]) * tensor_scale.  cols is a multiple of 16. */
+void ora_gemv_nvfp4(const uint8_t* w, const uint8_t* scale, float tensor_scale, int rows, int cols,
+                    const double* x, double* y);
+
 /* ---- one layer and one step ------------------------------------------------ */
 /*
  * x: [B][hidden], the layer's input residual on entry and its output on return.

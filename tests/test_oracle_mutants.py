@@ -49,6 +49,15 @@ MUTANTS = [
      "ora_rope(k + (size_t)h * hd, hd, pos + 1, d->rope_theta);", ["test_whole_step_matches_torch_reference"]),
     ("router input", "ora_gemv(W->router, E, H, xn, r);", "ora_gemv(W->router, E, H, xb, r);",
      ["test_moe_step_matches_torch_reference"]),
+    ("e4m3 exponent bias", "ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)",
+     ["test_e4m3_every_code_matches_torch"]),
+    ("e4m3 subnormals", "ldexp((double)m / 8.0, 1 - 7)", "ldexp(1.0 + (double)m / 8.0, 0 - 7)",
+     ["test_e4m3_closed_forms"]),
+    ("fp8 block index", "scale[(size_t)r * nb + c / block]", "scale[(size_t)r * nb + c % nb]",
+     ["test_gemv_fp8_matches_dequantized_torch"]),
+    ("nvfp4 nibble order", "c % 2 ? byte >> 4 : byte & 15", "c % 2 ? byte & 15 : byte >> 4",
+     ["test_gemv_nvfp4_nibble_order_and_scales"]),
+    ("nvfp4 tensor scale", "* (double)tensor_scale * x[c]", "* x[c]", ["test_gemv_nvfp4_matches_dequantized"]),
 ]
 
 

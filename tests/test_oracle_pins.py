@@ -312,3 +312,76 @@ def test_step_rejects_out_of_range():
     g, ls, S, kc, vc, model = _run_oracle(cfg)
     with pytest.raises(ValueError):
         model.decode_step(kc, vc, [0], [cfg.max_ctx], [cfg.max_ctx])
+
+
+# ------------------------------------------------------------------ low-bit weights (fp8 / nvfp4)
+
+def _e4m3_torch(codes):
+    """E4M3 codes decoded by PyTorch's float8_e4m3fn (a library routine)."""
+    return torch.from_numpy(np.asarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_every_code_matches_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = _e4m3_torch(codes)
+    got = np.array([ora.e4m3_to_double(int(c)) for c in codes])
+    assert np.array_equal(np.isnan(got), np.isnan(ref)) and np.isnan(got).sum() == 2  # 0x7F, 0xFF
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))
+
+
+def test_e4m3_closed_forms():
+    assert ora.e4m3_to_double(0x38) == 1.0                 # exponent 7 = bias
+    assert ora.e4m3_to_double(0x7E) == 448.0               # largest finite: 2^8 * 1.75
+    assert ora.e4m3_to_double(0x01) == 2.0 ** -9           # smallest subnormal
+    assert ora.e4m3_to_double(0x07) == 7 * 2.0 ** -9       # largest subnormal
+    assert ora.e4m3_to_double(0x08) == 2.0 ** -6           # smallest normal
+    assert ora.e4m3_to_double(0xC0) == -2.0
+
+
+def test_e2m1_every_code():
+    # the OCP 4-bit floating-point format's magnitudes; bit 3 is the sign
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for n in range(16):
+        v = ora.e2m1_to_double(n)
+        assert abs(v) == mags[n & 7] and (math.copysign(1.0, v) < 0) == bool(n & 8)
+
+
+def test_gemv_fp8_matches_dequantized_torch():
+    rows, cols, block = 7, 300, 128                        # a ragged last block of 44 columns
+    w = RNG.integers(0, 256, size=(rows, cols)).astype(np.uint8)
+    w[(w & 0x7F) == 0x7F] = 0x3C                           # no NaN codes
+    nb = (cols + block - 1) // block
+    scale = RNG.uniform(0.01, 2.0, size=(rows, nb)).astype(np.float32)
+    x = RNG.normal(0, 1, size=cols)
+    wd = _e4m3_torch(w.reshape(-1)).reshape(rows, cols) * np.repeat(scale.astype(np.float64), block, axis=1)[:, :cols]
+    ref = (torch.from_numpy(wd) @ torch.from_numpy(x)).numpy()
+    y = ora.gemv_fp8(w, scale, block, x)
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_gemv_nvfp4_nibble_order_and_scales():
+    # one row: byte 0x21 holds column 0 = 0.5 (low nibble 1) and column 1 = 1.0 (high nibble 2)
+    w = np.zeros((1, 8), dtype=np.uint8)
+    w[0, 0] = 0x21
+    scale = np.array([[0x40]], dtype=np.uint8)             # E4M3 0x40 = 2.0, for columns 0..15
+    x = np.zeros(16)
+    x[0], x[1] = 3.0, 5.0
+    y = ora.gemv_nvfp4(w, scale, 0.25, x)
+    assert y[0] == (0.5 * 3.0 + 1.0 * 5.0) * 2.0 * 0.25
+
+
+def test_gemv_nvfp4_matches_dequantized():
+    rows, cols = 5, 64
+    nib = RNG.integers(0, 16, size=(rows, cols)).astype(np.uint8)
+    w = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    sc = RNG.integers(0x20, 0x50, size=(rows, cols // 16)).astype(np.uint8)   # finite E4M3 scales
+    ts = 0.0625
+    x = RNG.normal(0, 1, size=cols)
+    table = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    vals = np.where(nib & 8, -1.0, 1.0) * table[nib & 7]
+    wd = vals * np.repeat(_e4m3_torch(sc.reshape(-1)).reshape(rows, -1), 16, axis=1) * ts
+    ref = wd @ x
+    y = ora.gemv_nvfp4(w, sc, ts, x)
+    assert np.max(np.abs(y - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
