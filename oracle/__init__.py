@@ -32,12 +32,16 @@ _D = ctypes.c_double
 class _Desc(ctypes.Structure):
     _fields_ = [(n, _I) for n in ("n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn_dim", "vocab",
                                   "n_experts", "top_k", "expert_ffn_dim", "qk_norm", "batch", "max_ctx")] + \
-               [("rms_eps", _D), ("rope_theta", _D)]
+               [("rms_eps", _D), ("rope_theta", _D), ("fp8_block", _I)]
+
+
+FP8_MATRICES = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down")  # in ora_layer's order of fp8 forms
 
 
 class _Layer(ctypes.Structure):
     _fields_ = [(n, _P) for n in ("attn_norm", "wq", "wk", "wv", "q_norm", "k_norm", "wo", "mlp_norm", "w_gate",
-                                  "w_up", "w_down", "router")]
+                                  "w_up", "w_down", "router")] + \
+               [(f"{n}_fp8_{part}", _P) for n in FP8_MATRICES for part in ("codes", "scale")]
 
 
 _EXPERT_FN = ctypes.CFUNCTYPE(_P, _P, _I, _I, _I)
@@ -218,7 +222,7 @@ class Model:
     dict with w_gate, w_up, w_down for MoE configs.
     """
 
-    def __init__(self, cfg, embed, final_norm, lm_head, layers, expert_fn=None, L=None):
+    def __init__(self, cfg, embed, final_norm, lm_head, layers, expert_fn=None, L=None, fp8_block=0):
         self.cfg = cfg
         self.L = L or lib()
         self._keep = [embed, final_norm, lm_head]
@@ -227,17 +231,27 @@ class Model:
             if lw is None:
                 continue
             for name in _Layer._fields_:
+                if "_fp8_" in name[0]:
+                    continue
                 a = lw.get(name[0])
                 if a is not None:
                     a = _u16(a)
                     self._keep.append(a)
                     setattr(self._layers[i], name[0], a.ctypes.data)
+            if fp8_block:  # fp8 forms: lw[name + "_fp8"] = (E4M3 codes uint8 [out][in], fp32 scales)
+                for n in FP8_MATRICES:
+                    codes, scale = lw[n + "_fp8"]
+                    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+                    scale = np.ascontiguousarray(scale, dtype=np.float32)
+                    self._keep += [codes, scale]
+                    setattr(self._layers[i], n + "_fp8_codes", codes.ctypes.data)
+                    setattr(self._layers[i], n + "_fp8_scale", scale.ctypes.data)
         self._expert_fn = expert_fn
         self._expert_cache = {}
         self._cb = _EXPERT_FN(self._expert)
         d = _Desc(cfg.n_layers, cfg.hidden, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.ffn_dim, cfg.vocab,
                   cfg.n_experts, cfg.top_k, cfg.expert_ffn_dim, int(cfg.qk_norm), cfg.batch, cfg.max_ctx,
-                  cfg.rms_eps, cfg.rope_theta)
+                  cfg.rms_eps, cfg.rope_theta, int(fp8_block))
         lm = embed if lm_head is None else lm_head
         self.m = _Model(d, embed.ctypes.data, final_norm.ctypes.data, lm.ctypes.data, self._layers, self._cb, None)
 

@@ -116,6 +116,15 @@ void ora_gemv_nvfp4(const uint8_t* w, const uint8_t* scale, float tensor_scale, 
   }
 }
 
+/* A layer's projection: its fp8 form when the model has one, else bf16. */
+static void gemv_w(const ora_desc* d, const uint16_t* w, const ora_fp8* w8, int rows, int cols, const double* x,
+                   double* y) {
+  if (d->fp8_block > 0)
+    ora_gemv_fp8(w8->codes, w8->scale, rows, cols, d->fp8_block, x, y);
+  else
+    ora_gemv(w, rows, cols, x, y);
+}
+
 /* SiLU (Hendrycks & Gimpel; Elfwing et al.): z * sigmoid(z) = z / (1 + e^-z). */
 double ora_silu(double z) { return z / (1.0 + exp(-z)); }
 
@@ -216,9 +225,9 @@ int ora_layer_forward(const ora_model* m, int layer, double* x, uint16_t* k_cach
 
     /* attention block */
     ora_rmsnorm(xb, H, W->attn_norm, d->rms_eps, xn);
-    ora_gemv(W->wq, nq * hd, H, xn, q);
-    ora_gemv(W->wk, nkv * hd, H, xn, k);
-    ora_gemv(W->wv, nkv * hd, H, xn, v);
+    gemv_w(d, W->wq, &W->wq8, nq * hd, H, xn, q);
+    gemv_w(d, W->wk, &W->wk8, nkv * hd, H, xn, k);
+    gemv_w(d, W->wv, &W->wv8, nkv * hd, H, xn, v);
     for (int h = 0; h < nq; ++h) {
       if (d->qk_norm) {
         ora_rmsnorm(q + (size_t)h * hd, hd, W->q_norm, d->rms_eps, tmp);
@@ -244,14 +253,23 @@ int ora_layer_forward(const ora_model* m, int layer, double* x, uint16_t* k_cach
       size_t base = (((size_t)b * nkv + kvh) * T) * hd;
       ora_attention(q + (size_t)h * hd, k_cache + base, v_cache + base, S + 1, hd, att + (size_t)h * hd, NULL);
     }
-    ora_gemv(W->wo, H, nq * hd, att, o);
+    gemv_w(d, W->wo, &W->wo8, H, nq * hd, att, o);
     for (int i = 0; i < H; ++i) xb[i] += o[i];
     if (h_attn) memcpy(h_attn + (size_t)b * H, xb, sizeof(double) * H);
 
     /* MLP block */
     ora_rmsnorm(xb, H, W->mlp_norm, d->rms_eps, xn);
     if (d->n_experts == 0) {
-      ora_swiglu(W->w_gate, W->w_up, W->w_down, d->ffn_dim, H, xn, o);
+      if (d->fp8_block > 0) {  /* SwiGLU as ora_swiglu, on the fp8 matrices */
+        double* gu = (double*)malloc(sizeof(double) * 2 * (size_t)d->ffn_dim);
+        gemv_w(d, W->w_gate, &W->gate8, d->ffn_dim, H, xn, gu);
+        gemv_w(d, W->w_up, &W->up8, d->ffn_dim, H, xn, gu + d->ffn_dim);
+        for (int i = 0; i < d->ffn_dim; ++i) gu[i] = ora_silu(gu[i]) * gu[d->ffn_dim + i];
+        gemv_w(d, W->w_down, &W->down8, H, d->ffn_dim, gu, o);
+        free(gu);
+      } else {
+        ora_swiglu(W->w_gate, W->w_up, W->w_down, d->ffn_dim, H, xn, o);
+      }
       for (int i = 0; i < H; ++i) xb[i] += o[i];
     } else {
       const int E = d->n_experts, K = d->top_k;

@@ -38,12 +38,23 @@ typedef struct ora_desc {
   int qk_norm;                          /* per-head RMSNorm of q and k before RoPE */
   int batch, max_ctx;
   double rms_eps, rope_theta;
+  int fp8_block; /* > 0: the layers' projections are fp8 (ora_layer.*8) with one scale per row per
+                    fp8_block columns; 0: bf16 */
 } ora_desc;
+
+/* An fp8 weight matrix: E4M3 codes [out][in] and fp32 scales [out][ceil(in / fp8_block)]. */
+typedef struct ora_fp8 {
+  const uint8_t* codes;
+  const float* scale;
+} ora_fp8;
 
 typedef struct ora_layer {
   const uint16_t *attn_norm, *wq, *wk, *wv, *q_norm, *k_norm, *wo, *mlp_norm;
   const uint16_t *w_gate, *w_up, *w_down; /* dense MLP; unused for MoE */
   const uint16_t *router;                 /* [n_experts][hidden]; MoE only */
+  /* fp8 forms of wq wk wv wo and of the dense gate / up / down (ora_desc.fp8_block > 0): they then
+     replace the bf16 matrices; norms, router, experts, embedding and LM head stay bf16 */
+  ora_fp8 wq8, wk8, wv8, wo8, gate8, up8, down8;
 } ora_layer;
 
 /* Returns expert weights on demand: which = 0 gate, 1 up, 2 down. */

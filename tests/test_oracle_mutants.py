@@ -41,8 +41,8 @@ MUTANTS = [
     ("silu sign", "return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));", ["test_silu_values"]),
     ("mlp norm gain", "ora_rmsnorm(xb, H, W->mlp_norm,", "ora_rmsnorm(xb, H, W->attn_norm,",
      ["test_whole_step_matches_torch_reference"]),
-    ("mlp residual", "xn, o);\n      for (int i = 0; i < H; ++i) xb[i] += o[i];",
-     "xn, o);\n      for (int i = 0; i < H; ++i) xb[i] = o[i];", ["test_whole_step_matches_torch_reference"]),
+    ("mlp residual", "      }\n      for (int i = 0; i < H; ++i) xb[i] += o[i];",
+     "      }\n      for (int i = 0; i < H; ++i) xb[i] = o[i];", ["test_whole_step_matches_torch_reference"]),
     ("final norm skipped", "ora_gemv(m->lm_head, m->d.vocab, H, xn, logits);",
      "ora_gemv(m->lm_head, m->d.vocab, H, x, logits);", ["test_whole_step_matches_torch_reference"]),
     ("key rope position", "ora_rope(k + (size_t)h * hd, hd, pos, d->rope_theta);",
@@ -58,6 +58,10 @@ MUTANTS = [
     ("nvfp4 nibble order", "c % 2 ? byte >> 4 : byte & 15", "c % 2 ? byte & 15 : byte >> 4",
      ["test_gemv_nvfp4_nibble_order_and_scales"]),
     ("nvfp4 tensor scale", "* (double)tensor_scale * x[c]", "* x[c]", ["test_gemv_nvfp4_matches_dequantized"]),
+    ("fp8 step ignores fp8 o_proj", "gemv_w(d, W->wo, &W->wo8, H, nq * hd, att, o);",
+     "ora_gemv(W->wo, H, nq * hd, att, o);", ["test_fp8_step_uses_the_fp8_weights"]),
+    ("fp8 swiglu operands", "gu[i] = ora_silu(gu[i]) * gu[d->ffn_dim + i];",
+     "gu[i] = ora_silu(gu[d->ffn_dim + i]) * gu[i];", ["test_fp8_step_equals_bf16_step_when_the_weights_agree"]),
 ]
 
 

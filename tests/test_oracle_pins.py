@@ -385,3 +385,60 @@ def test_gemv_nvfp4_matches_dequantized():
     ref = wd @ x
     y = ora.gemv_nvfp4(w, sc, ts, x)
     assert np.max(np.abs(y - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_fp8_step_equals_bf16_step_when_the_weights_agree():
+    # fp8 projections whose E4M3 code x power-of-two block scale is exactly representable in bf16
+    # (4 significant bits): the oracle's fp8 step and its bf16 step on those bf16 values must agree
+    # bit for bit (same products, same summation order)
+    cfg = fx.CONFIGS["tiny"].replace(ffn_dim=320)
+    g, ls = host_model(cfg, gains="random")
+    block = 128
+    gen = torch.Generator().manual_seed(7)
+    for lw in ls:
+        for name in ora.FP8_MATRICES:
+            rows, cols = lw[name].shape
+            codes = (torch.randn(rows, cols, generator=gen, dtype=torch.float32) * 8).to(torch.float8_e4m3fn)
+            nb = (cols + block - 1) // block
+            k = torch.randint(-10, -6, (rows, nb), generator=gen)
+            scale = torch.pow(2.0, k.to(torch.float64)).to(torch.float32)
+            w = codes.to(torch.float64) * scale.to(torch.float64).repeat_interleave(block, dim=1)[:, :cols]
+            wb = w.to(torch.bfloat16)
+            assert torch.equal(wb.to(torch.float64), w)          # exact in bf16
+            lw[name] = wb.view(torch.int16).numpy().view(np.uint16)
+            lw[name + "_fp8"] = (codes.view(torch.uint8).numpy(), scale.numpy())
+    S = fx.context_lengths(cfg)
+    outs = []
+    for fp8 in (0, block):
+        kc, vc = host_caches(cfg, S)
+        model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls, fp8_block=fp8)
+        outs.append((model.decode_step(kc, vc, fx.tokens(cfg)[0], S, S), kc, vc))
+    (a, ka, va), (b, kb, vb) = outs
+    for key in ("h_attn", "h_mlp", "logits"):
+        assert np.array_equal(a[key], b[key]), key
+    assert np.array_equal(ka, kb) and np.array_equal(va, vb)
+
+
+def test_fp8_step_uses_the_fp8_weights():
+    # the same model with its fp8 codes perturbed (bf16 matrices unchanged) must change the fp8 step only
+    cfg = fx.CONFIGS["tiny"].replace(ffn_dim=320, n_layers=1)
+    g, ls = host_model(cfg)
+    gen = torch.Generator().manual_seed(3)
+    for lw in ls:
+        for name in ora.FP8_MATRICES:
+            rows, cols = lw[name].shape
+            codes = (torch.randn(rows, cols, generator=gen) * 8).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            lw[name + "_fp8"] = (codes, np.full((rows, (cols + 127) // 128), 2.0 ** -8, dtype=np.float32))
+    S = fx.context_lengths(cfg)
+    res = []
+    for bump in (False, True):
+        if bump:
+            c, s = ls[0]["wo_fp8"]
+            c = c.copy()
+            c[0, 0] ^= 0x08                                     # one code of o_proj
+            ls[0]["wo_fp8"] = (c, s)
+        kc, vc = host_caches(cfg, S)
+        m = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls, fp8_block=128)
+        res.append(m.decode_step(kc, vc, fx.tokens(cfg)[0], S, S)["h_attn"])
+    d = np.abs(res[1] - res[0]).reshape(-1)
+    assert d[0] > 0 and np.count_nonzero(d) == 1                # o_proj row 0 only
