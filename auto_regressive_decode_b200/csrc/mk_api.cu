@@ -325,7 +325,8 @@ __global__ void greedy_init(const int32_t* tok0, const int32_t* len0, int B, int
 }
 
 // After a step: the arg-max token (the key's low word holds ~token) becomes the
-// next step's input and output, every sequence moves one position on.
+// next step's input and output, every sequence moves one position on.  A step
+// that did no work (a sticky device status) leaves the key at 0: token -1.
 __global__ void greedy_advance(int B, int32_t* tok, int32_t* len, unsigned long long* amax, int32_t* out_tok) {
   const int b = threadIdx.x;
   if (b < B) {

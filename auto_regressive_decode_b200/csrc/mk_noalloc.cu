@@ -159,7 +159,7 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   const size_t o_off = take(sizeof(int32_t) * offsets.size());
   const size_t o_lay = take(sizeof(mk::LayerPtrs) * (size_t)L);
   const size_t o_rope = take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
-  const size_t n_tmaps = (size_t)mk::kTmapsPerLayer * L + 3;  // KV caches always; weights on the tensor-core kernel  // batch > 1: TMA tensor maps
+  const size_t n_tmaps = (size_t)mk::kTmapsPerLayer * L + 3;  // KV caches always; weights on the tensor-core kernel
   const size_t o_tmap = n_tmaps ? take(128 * n_tmaps) : 0;
   if (off > kStaticScratchBytes) return MK_ERR_UNSUPPORTED;  // model needs more than the 8 MiB array
   std::vector<uint8_t> tmaps(128 * n_tmaps);

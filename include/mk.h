@@ -142,9 +142,13 @@ int mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions
  *   out_tokens device int32[n_steps][batch]: x_1 .. x_{n_steps}
  *   out_logits device fp32[batch][vocab] for the last step's logits, or NULL
  * Asynchronous on `stream`; device-side errors (e.g. a length reaching
- * max_ctx, MK_ERR_RANGE) are reported by mk_get_status.  Each step is the
- * same kernel as mk_decode_step; the pick folds the LM head's outputs into
- * per-sequence maxima on the device and a one-warp kernel advances the state.
+ * max_ctx, MK_ERR_RANGE) are reported by mk_get_status, which the caller must
+ * check after the loop: the return value only covers argument checks and
+ * launches.  Once a step fails, the later steps of the call do no work and
+ * out_tokens holds -1 for the failing step and every step after it.  Each step
+ * is the same kernel as mk_decode_step; the pick folds the LM head's outputs
+ * into per-sequence maxima on the device and a one-warp kernel advances the
+ * state.
  */
 int mk_decode_greedy(mk_handle* h, int n_steps, const int32_t* tokens, const int32_t* seq_lens, void* stream,
                      int32_t* out_tokens, float* out_logits);

@@ -223,6 +223,9 @@ class Model:
     """
 
     def __init__(self, cfg, embed, final_norm, lm_head, layers, expert_fn=None, L=None, fp8_block=0):
+        if fp8_block and cfg.n_experts:
+            raise ValueError("fp8 weights are modelled for the attention projections and the dense MLP only, "
+                             "not for a mixture-of-experts model")
         self.cfg = cfg
         self.L = L or lib()
         self._keep = [embed, final_norm, lm_head]

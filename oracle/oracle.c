@@ -206,6 +206,9 @@ int ora_layer_forward(const ora_model* m, int layer, double* x, uint16_t* k_cach
                       const int32_t* positions, const int32_t* seq_lens, double* h_attn, double* router_logits,
                       int32_t* sel, double* sel_w) {
   const ora_desc* d = &m->d;
+  /* fp8 weights are modelled for the attention projections and the dense MLP only: a MoE model
+   * with fp8_block set has no fp8 router or experts to run, so it is refused rather than run in bf16 */
+  if (d->fp8_block > 0 && d->n_experts > 0) return -1;
   const ora_layer* W = &m->layers[layer];
   const int H = d->hidden, hd = d->head_dim, nq = d->n_q_heads, nkv = d->n_kv_heads, T = d->max_ctx;
   const int group = nq / nkv;

@@ -83,7 +83,9 @@ void ora_swiglu(const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_
                 const double* xn, double* y);
 void ora_topk(const double* logits, int n, int k, int32_t* sel, double* w);
 
-/* ---- low-bit weights (fp8 / nvfp4 weight streaming; not used by the decode step yet) ---------- */
+/* ---- low-bit weights (fp8 / nvfp4 weight streaming) -------------------------------------------- */
+/* The decode step runs wq, wk, wv, wo and the dense gate / up / down in fp8 when ora_desc.fp8_block
+ * is set (a MoE model with fp8_block set is refused); nvfp4 is used by ora_gemv_nvfp4 only. */
 /* Exact decodes to double.  E4M3 is the OCP 8-bit floating-point format (sign, 4 exponent bits with
  * bias 7, 3 mantissa bits; exponent 0 is subnormal; 0x7F and 0xFF are NaN; no infinities; largest
  * finite 448).  E2M1 is the OCP 4-bit format of the low nibble (sign, 2 exponent bits with bias 1,

@@ -4,12 +4,17 @@ Tolerances (stated by the decode-step parity contract this library is held to):
 per-layer hidden-state relative L2 <= 1e-2, logits max abs <= 5e-2,
 appended K/V relative L2 <= 1e-2, top-1 token identical on >= 99% of steps.
 
-Top-1 reading: with seeded random weights the logits are flat (standard
-deviation ~0.5 over the vocabulary), so the oracle's two best tokens are often
-closer than the bf16 rounding of the activations moves a logit.  A step agrees
-when the GPU's pick is a top-1 token of the oracle up to TOP1_TIE: its oracle
-logit is within TOP1_TIE of the oracle's maximum.  The exact-argmax rate is
-recorded beside it ("top1_exact").
+Top-1.  The batch-1 CUDA-core kernel keeps every activation in fp32, so its
+logits sit within a few 1e-6 of the oracle's: there the GPU's arg-max must
+equal the oracle's arg-max exactly on >= 99% of (step, sequence) pairs.  The
+tensor-core kernel (batch > 1, or any MoE model) rounds its mma operands to
+bf16, which moves a logit by up to ~1e-2; with seeded random weights the
+logits are flat (standard deviation ~0.5 over the vocabulary), so the
+oracle's two best tokens are sometimes closer than that.  On that kernel a
+step agrees when the GPU's pick is an oracle top-1 token up to TOP1_TIE (its
+oracle logit within TOP1_TIE of the oracle maximum).  Both rates are recorded
+on every run ("top1_exact", "top1"), and so is the oracle gap of every
+exact-argmax miss ("top1_gaps").
 
 MoE selection reading ("bit-exact" selection): (i) the GPU's picks and their
 order equal the oracle's top-k applied to the GPU's own router logits, for
@@ -17,8 +22,15 @@ every (layer, sequence); (ii) the GPU's router logits match the oracle's
 within the hidden-state tolerance; (iii) the end-to-end pick sets agree
 except where the oracle's k-th and (k+1)-th logits are closer than twice the
 measured router-logit error (a near-tie either side may resolve).
+
+Paged runs put each sequence's cache into a page pool through a seeded random
+block table, with the spare pages poisoned with NaN; the GPU then reads and
+appends through the table while the oracle keeps its contiguous cache.
 """
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 import torch
@@ -33,13 +45,61 @@ TOL_LOGITS_ABS = 5e-2
 TOL_KV = 1e-2
 MIN_TOP1 = 0.99
 TOP1_TIE = 1e-2
+NAN_BITS = 0x7FC0  # bf16 quiet NaN
 
 
 def bits(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def run_teacher_forced(cfg, steps=None, gains="ones", seed=fx.DEFAULT_SEED, seq_lens=None, wait_timeout_ns=0):
+def tensor_core_kernel(cfg) -> bool:
+    """The library runs batch > 1 and every MoE model on its tensor-core kernel."""
+    return cfg.batch > 1 or cfg.n_experts > 0
+
+
+# ---- paged cache ------------------------------------------------------------------------------
+
+def page_size(cfg) -> int:
+    """One attention stage of positions per page (32 KB of K or V)."""
+    return 32768 // (2 * cfg.head_dim)
+
+
+def block_table(cfg, seed=7, spare=5):
+    """(table int32 [B][pages per sequence], pool pages): a seeded random permutation with spare pages."""
+    stride = -(-cfg.max_ctx // page_size(cfg))
+    n_pages = cfg.batch * stride + spare
+    table = np.random.default_rng(seed).permutation(n_pages)[:cfg.batch * stride].reshape(cfg.batch, stride)
+    return table.astype(np.int32), n_pages
+
+
+def to_pool(cache, page, n_pages, table):
+    """Contiguous [L][B][nkv][T][hd] -> pool [L][n_pages][nkv][page][hd] by the block table (spares NaN)."""
+    L, B, nkv, T, hd = cache.shape
+    pool = torch.full((L, n_pages, nkv, page, hd), NAN_BITS, dtype=torch.int16, device=cache.device)
+    c16 = cache.view(torch.int16)
+    for b in range(B):
+        for j in range(table.shape[1]):
+            lo, hi = j * page, min(T, (j + 1) * page)
+            pool[:, int(table[b, j]), :, :hi - lo] = c16[:, b, :, lo:hi]
+    return pool.view(torch.bfloat16)
+
+
+def from_pool(pool, shape, page, table):
+    """Pool -> contiguous [L][B][nkv][T][hd] (int16 bits) through the block table."""
+    L, B, nkv, T, hd = shape
+    out = torch.empty(shape, dtype=torch.int16, device=pool.device)
+    p16 = pool.view(torch.int16)
+    for b in range(B):
+        for j in range(table.shape[1]):
+            lo, hi = j * page, min(T, (j + 1) * page)
+            out[:, b, :, lo:hi] = p16[:, int(table[b, j]), :, :hi - lo]
+    return out
+
+
+# ---- teacher-forced run -----------------------------------------------------------------------
+
+def run_teacher_forced(cfg, steps=None, gains="ones", seed=fx.DEFAULT_SEED, seq_lens=None, wait_timeout_ns=0,
+                       paged=False):
     """Run `steps` decode steps on the GPU and in the oracle; return per-step error metrics."""
     import auto_regressive_decode_b200.mk as mk
     steps = cfg.steps if steps is None else steps
@@ -48,8 +108,24 @@ def run_teacher_forced(cfg, steps=None, gains="ones", seed=fx.DEFAULT_SEED, seq_
     # GPU side: poisoned cache tail, so that a read past a sequence's length shows up as NaN
     w = device_model(cfg, seed, gains)
     kc, vc = device_caches(cfg, S0, seed, poison=True)
-    k_init, v_init = kc.clone(), vc.clone()
-    dec = mk.Decoder(cfg, w, kc, vc, wait_timeout_ns=wait_timeout_ns)
+    shape = tuple(kc.shape)
+    if paged:
+        page = page_size(cfg)
+        table, n_pages = block_table(cfg)
+        kp, vp = to_pool(kc, page, n_pages, table), to_pool(vc, page, n_pages, table)
+        del kc, vc
+        k_init, v_init = kp.clone(), vp.clone()
+        d_table = torch.from_numpy(table).cuda()
+        dec = mk.Decoder(cfg, w, kp, vp, wait_timeout_ns=wait_timeout_ns, block_table=d_table, page_size=page)
+
+        def gpu_caches():
+            return from_pool(kp, shape, page, table), from_pool(vp, shape, page, table)
+    else:
+        k_init, v_init = kc.clone(), vc.clone()
+        dec = mk.Decoder(cfg, w, kc, vc, wait_timeout_ns=wait_timeout_ns)
+
+        def gpu_caches():
+            return kc.view(torch.int16), vc.view(torch.int16)
     # oracle side: its own caches from the same generator
     g, ls = host_model(cfg, seed, gains)
     okc, ovc = host_caches(cfg, S0, seed)
@@ -57,7 +133,8 @@ def run_teacher_forced(cfg, steps=None, gains="ones", seed=fx.DEFAULT_SEED, seq_
                       expert_loader(cfg, seed) if cfg.n_experts else None)
     B, L = cfg.batch, cfg.n_layers
     logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
-    res = {"hidden": [], "logits_abs": [], "kv": [], "top1": [], "top1_exact": [], "status": [],
+    res = {"config": cfg.name, "kernel": "tensor-core" if tensor_core_kernel(cfg) else "cuda-core", "paged": paged,
+           "hidden": [], "logits_abs": [], "kv": [], "top1": [], "top1_exact": [], "top1_gaps": [], "status": [],
            "router": [], "sel_own": [], "sel_w": [], "sel_e2e": [], "sel_e2e_unexplained": 0, "count_ok": []}
     for t in range(steps):
         S = (S0 + t).astype(np.int32)
@@ -76,25 +153,46 @@ def run_teacher_forced(cfg, steps=None, gains="ones", seed=fx.DEFAULT_SEED, seq_
             errs.append(rel_l2(hid[2 * l + 2], ref["h_mlp"][l]))
         res["hidden"].append(max(errs))
         res["logits_abs"].append(float(np.max(np.abs(lg - ref["logits"]))))
+        gk_all, gv_all = gpu_caches()
         kv_err = 0.0
         for b in range(B):
-            gk = bf16_f64(bits(kc[:, b, :, S[b]].contiguous()))
-            gv = bf16_f64(bits(vc[:, b, :, S[b]].contiguous()))
+            gk = bf16_f64(bits(gk_all[:, b, :, S[b]].contiguous()))
+            gv = bf16_f64(bits(gv_all[:, b, :, S[b]].contiguous()))
             kv_err = max(kv_err, rel_l2(gk, bf16_f64(okc[:, b, :, S[b]])), rel_l2(gv, bf16_f64(ovc[:, b, :, S[b]])))
         res["kv"].append(kv_err)
         if cfg.n_experts:
             check_routing(res, dec.routing(), ref, cfg)
-        res["top1"].extend(top1_agree(lg, ref["logits"]))
-        res["top1_exact"].extend(list(np.argmax(lg, axis=1) == np.argmax(ref["logits"], axis=1)))
+        record_top1(res, lg, ref["logits"])
     # cache bytes other than the appended rows are untouched
-    kc_h, vc_h, ki, vi = bits(kc), bits(vc), bits(k_init), bits(v_init)
+    gk_all, gv_all = gpu_caches()
+    if paged:
+        ki, vi = from_pool(k_init, shape, page, table), from_pool(v_init, shape, page, table)
+        spare = sorted(set(range(n_pages)) - set(table.ravel().tolist()))
+        spare_ok = (torch.equal(kp.view(torch.int16)[:, spare], k_init.view(torch.int16)[:, spare]) and
+                    torch.equal(vp.view(torch.int16)[:, spare], v_init.view(torch.int16)[:, spare]))
+    else:
+        ki, vi = k_init.view(torch.int16), v_init.view(torch.int16)
+        spare_ok = True
+    kc_h, vc_h, ki, vi = bits(gk_all), bits(gv_all), bits(ki), bits(vi)
     touched = np.zeros(kc_h.shape[:4], dtype=bool)   # [L][B][nkv][T]
     for b in range(B):
         touched[:, b, :, S0[b]:S0[b] + steps] = True
-    res["untouched_ok"] = bool(np.array_equal(kc_h[~touched], ki[~touched]) and
+    res["untouched_ok"] = bool(spare_ok and np.array_equal(kc_h[~touched], ki[~touched]) and
                                np.array_equal(vc_h[~touched], vi[~touched]))
     dec.close()
+    log_result(res)
     return res
+
+
+def record_top1(res, gpu_logits: np.ndarray, ref_logits: np.ndarray):
+    """Per sequence: exact arg-max agreement, agreement up to TOP1_TIE, and the oracle gap of a miss."""
+    pick = np.argmax(gpu_logits, axis=1)
+    best = ref_logits.max(axis=1)
+    got = ref_logits[np.arange(ref_logits.shape[0]), pick]
+    exact = pick == np.argmax(ref_logits, axis=1)
+    res["top1"].extend(list(got >= best - TOP1_TIE))
+    res["top1_exact"].extend(list(exact))
+    res["top1_gaps"].extend([float(x) for x in (best - got)[~exact]])
 
 
 def top1_agree(gpu_logits: np.ndarray, ref_logits: np.ndarray) -> list:
@@ -102,6 +200,11 @@ def top1_agree(gpu_logits: np.ndarray, ref_logits: np.ndarray) -> list:
     pick = np.argmax(gpu_logits, axis=1)
     got = ref_logits[np.arange(ref_logits.shape[0]), pick]
     return list(got >= ref_logits.max(axis=1) - TOP1_TIE)
+
+
+def top1_exact(gpu_logits: np.ndarray, ref_logits: np.ndarray) -> list:
+    """Per sequence: the GPU's argmax is the oracle's argmax."""
+    return list(np.argmax(gpu_logits, axis=1) == np.argmax(ref_logits, axis=1))
 
 
 def check_routing(res, gpu, ref, cfg):
@@ -124,12 +227,39 @@ def check_routing(res, gpu, ref, cfg):
                     res["sel_e2e_unexplained"] += 1
 
 
+def summary(res) -> dict:
+    """The figures a parity run is judged on (also written to MK_PARITY_LOG when that is set)."""
+    out = {"config": res.get("config"), "kernel": res.get("kernel"), "paged": res.get("paged", False),
+           "steps_x_seqs": len(res["top1_exact"]), "top1_exact": float(np.mean(res["top1_exact"])),
+           "top1_tie": float(np.mean(res["top1"])), "top1_miss_gaps": res["top1_gaps"],
+           "hidden_max": max(res["hidden"]), "logits_abs_max": max(res["logits_abs"]), "kv_max": max(res["kv"])}
+    if res["router"]:
+        out["router_max"] = max(res["router"])
+        out["sel_e2e"] = float(np.mean(res["sel_e2e"]))
+    return out
+
+
+def log_result(res):
+    path = os.environ.get("MK_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(summary(res)) + "\n")
+
+
+def assert_top1(res):
+    """Exact arg-max identity on the batch-1 CUDA-core kernel; the tie reading on the tensor-core kernel."""
+    if res.get("kernel") == "cuda-core":
+        assert np.mean(res["top1_exact"]) >= MIN_TOP1, (np.mean(res["top1_exact"]), res["top1_gaps"])
+    else:
+        assert np.mean(res["top1"]) >= MIN_TOP1, (np.mean(res["top1"]), np.mean(res["top1_exact"]))
+
+
 def assert_parity(res):
     assert all(s == 0 for s in res["status"]), res["status"]
     assert max(res["hidden"]) <= TOL_HIDDEN, res["hidden"]
     assert max(res["logits_abs"]) <= TOL_LOGITS_ABS, res["logits_abs"]
     assert max(res["kv"]) <= TOL_KV, res["kv"]
-    assert np.mean(res["top1"]) >= MIN_TOP1, np.mean(res["top1"])
+    assert_top1(res)
     assert res["untouched_ok"]
     if res["router"]:
         assert max(res["router"]) <= TOL_HIDDEN, max(res["router"])

@@ -442,3 +442,18 @@ def test_fp8_step_uses_the_fp8_weights():
         res.append(m.decode_step(kc, vc, fx.tokens(cfg)[0], S, S)["h_attn"])
     d = np.abs(res[1] - res[0]).reshape(-1)
     assert d[0] > 0 and np.count_nonzero(d) == 1                # o_proj row 0 only
+
+
+def test_fp8_step_refuses_a_mixture_of_experts_model():
+    # fp8 forms exist for wq wk wv wo and the dense gate / up / down only: a MoE model asked to run
+    # in fp8 is refused on both sides of the binding instead of silently running its experts in bf16
+    cfg = fx.CONFIGS["tiny"].replace(ffn_dim=0, n_experts=4, top_k=2, expert_ffn_dim=64, n_layers=1)
+    g, ls = host_model(cfg)
+    with pytest.raises(ValueError):
+        ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls, expert_loader(cfg), fp8_block=128)
+    model = ora.Model(cfg, g["embed"], g["final_norm"], g["lm_head"], ls, expert_loader(cfg))
+    model.m.d.fp8_block = 128                                   # the C entry point's own check
+    kc, vc = host_caches(cfg, fx.context_lengths(cfg))
+    S = fx.context_lengths(cfg)
+    with pytest.raises(ValueError):
+        model.layer_forward(0, np.zeros((cfg.batch, cfg.hidden)), kc[0], vc[0], S, S)

@@ -38,8 +38,26 @@ def test_tiny_last_cache_slot():
     assert_parity(run_teacher_forced(cfg))
 
 
-def test_dense_0_6b_first_steps():
-    assert_parity(run_teacher_forced(fx.CONFIGS["dense-0.6b"], steps=3))
+def test_dense_0_6b_all_steps():
+    """The 0.6B shape (qk-norm, tied embeddings) end to end over all 64 of its decode steps."""
+    assert_parity(run_teacher_forced(fx.CONFIGS["dense-0.6b"]))
+
+
+# ---- paged KV cache through the oracle ---------------------------------------------------------
+
+@pytest.mark.parametrize("kw,gains", [
+    ({"n_q_heads": 4, "n_kv_heads": 2, "head_dim": 128, "ctx": 200, "steps": 4}, "random"),           # batch 1
+    ({"n_q_heads": 8, "n_kv_heads": 2, "head_dim": 128, "batch": 3, "ffn_dim": 704, "ctx": 0, "ctx_lo": 5,
+      "ctx_hi": 260, "steps": 3}, "random"),                                                          # tensor cores
+    ({"n_q_heads": 4, "n_kv_heads": 2, "head_dim": 128, "batch": 2, "ffn_dim": 0, "n_experts": 8, "top_k": 2,
+      "expert_ffn_dim": 128, "ctx": 0, "ctx_lo": 100, "ctx_hi": 300, "steps": 3}, "random"),          # MoE
+])
+def test_paged_cache_against_the_oracle(kw, gains):
+    """Every sequence's cache in a shuffled page pool (spare pages NaN): the oracle keeps its own
+    contiguous cache, the GPU reads and appends through the block table."""
+    cfg = fx.CONFIGS["tiny"].replace(**kw)
+    res = run_teacher_forced(cfg, gains=gains, paged=True)
+    assert_parity(res)
 
 
 # ---- batch > 1 (tensor-core projections) -------------------------------------------------------
