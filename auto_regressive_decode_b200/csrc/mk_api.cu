@@ -165,6 +165,8 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   const size_t o_rope = cv.take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
   const size_t n_tmaps = (size_t)mk::kTmapsPerLayer * L + 3;  // KV caches always; weights on the tensor-core kernel
   const size_t o_tmap = n_tmaps ? cv.take(128 * n_tmaps) : 0;
+  const size_t n_tb1 = mk::batched(d) ? 0 : mk::n_tmaps_b1(d);  // the batch-1 kernel's weight maps
+  const size_t o_tb1 = n_tb1 ? cv.take(128 * n_tb1) : 0;
   const char* trace_env = getenv("MK_TRACE");
   const bool tracing = trace_env && atoi(trace_env) > 0;
   const size_t o_trace = tracing ? cv.take(sizeof(uint64_t) * mk::kTraceStamps * instrs.size()) : 0;
@@ -204,17 +206,17 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
       rope[(size_t)pos * (hd / 2) + i] = make_float2((float)cos(ang), (float)sin(ang));
     }
 
-  std::vector<uint8_t> tmaps(128 * n_tmaps);
-  if (n_tmaps) {
-    const cudaError_t te = mk::encode_tmaps(d, *w, *kv, tmaps.data());
-    if (te != cudaSuccess) {
-      cudaFree(h->region);
-      delete h;
-      return te == cudaErrorInvalidValue ? MK_ERR_UNSUPPORTED : MK_ERR_CUDA;
-    }
+  std::vector<uint8_t> tmaps(128 * n_tmaps), tb1(128 * n_tb1);
+  cudaError_t te = n_tmaps ? mk::encode_tmaps(d, *w, *kv, tmaps.data()) : cudaSuccess;
+  if (te == cudaSuccess && n_tb1) te = mk::encode_tmaps_b1(d, *w, tb1.data());
+  if (te != cudaSuccess) {
+    cudaFree(h->region);
+    delete h;
+    return te == cudaErrorInvalidValue ? MK_ERR_UNSUPPORTED : MK_ERR_CUDA;
   }
   bool ok = cudaMemset(base, 0, h->region_bytes) == cudaSuccess &&
             (!n_tmaps || cudaMemcpy(base + o_tmap, tmaps.data(), tmaps.size(), cudaMemcpyHostToDevice) == cudaSuccess) &&
+            (!n_tb1 || cudaMemcpy(base + o_tb1, tb1.data(), tb1.size(), cudaMemcpyHostToDevice) == cudaSuccess) &&
             cudaMemcpy(base + o_ins, instrs.data(), sizeof(mk_instr) * instrs.size(), cudaMemcpyHostToDevice) ==
                 cudaSuccess &&
             cudaMemcpy(base + o_off, offsets.data(), sizeof(int32_t) * offsets.size(), cudaMemcpyHostToDevice) ==
@@ -258,6 +260,7 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   }
   p.rope = (const float2*)(base + o_rope);
   p.tmaps = n_tmaps ? base + o_tmap : nullptr;
+  p.tmaps_b1 = n_tb1 ? base + o_tb1 : nullptr;
   p.xres = (float*)(base + o_xres);
   p.qkv = (float*)(base + o_qkv);
   p.attn = (float*)(base + o_attn);
@@ -287,8 +290,8 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   h->loop_len = (int32_t*)(base + o_llen);
   h->amax = (unsigned long long*)(base + o_amax);
   h->loop_logits = (float*)(base + o_llog);
-  const char* piece_env = getenv("MK_COPY_PIECE_KB");  // diagnostic knob: bytes per bulk copy
-  p.copy_piece = piece_env && atoi(piece_env) > 0 ? (uint32_t)atoi(piece_env) * 1024u : mk::kDefaultCopyPiece;
+  const char* ahead_env = getenv("MK_L2_AHEAD_KB");  // tuning knob: the batch-1 kernel's L2 runway (0: off)
+  p.l2_ahead = ahead_env ? (uint32_t)atoi(ahead_env) * 1024u : mk::kDefaultL2Ahead;
   *out = h;
   return MK_OK;
 }

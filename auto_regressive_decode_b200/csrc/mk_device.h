@@ -33,6 +33,10 @@ struct Params {
   // matrix: [layer][wq wk wv wo w_gate w_up w_down], then the LM head, the K
   // cache and the V cache
   const uint8_t* tmaps;
+  // batch-1 kernel: 2-D TMA maps of every weight matrix, kB1BoxHeights per
+  // matrix (boxes of kB1Chunk columns x 16, 8, 4, 2, 1 rows): [layer][wq wk wv
+  // wo w_gate w_up w_down], then the LM head
+  const uint8_t* tmaps_b1;
   // library scratch (device)
   float* xres;              // [2L+1][B][H]
   float* qkv;               // [B][nq*hd + 2*nkv*hd]
@@ -66,7 +70,7 @@ struct Params {
   uint32_t epoch;
   uint64_t timeout_ns;
   uint64_t* trace;          // [n_instr][kTraceStamps] timestamps, or nullptr
-  uint32_t copy_piece;      // bytes per bulk copy (a multiple of 16); a stage is split into pieces
+  uint32_t l2_ahead;        // batch-1 kernel: weight bytes kept prefetched into L2 beyond the ring's instruction
 };
 
 // Encode the 3-D tensor maps of the batch > 1 kernel (one per weight matrix,
@@ -74,6 +78,11 @@ struct Params {
 // maps of 128 bytes).  Returns cudaErrorInvalidValue when the driver rejects a
 // map (alignment, sizes).
 cudaError_t encode_tmaps(const mk_model_desc& d, const mk_weights& w, const mk_kv& kv, uint8_t* out);
+
+// Maps of the batch-1 kernel's row-stationary tiles (kB1MapsPerLayer * L + 2
+// maps of 128 bytes) into host memory `out`.
+cudaError_t encode_tmaps_b1(const mk_model_desc& d, const mk_weights& w, uint8_t* out);
+inline size_t n_tmaps_b1(const mk_model_desc& d) { return (size_t)kB1MapsPerLayer * d.n_layers + kB1BoxHeights; }
 
 // Dynamic shared memory of one CTA.
 size_t kernel_smem_bytes(bool batched);

@@ -43,14 +43,12 @@ constexpr int kStagesBatched = 5;                      // ring depth of the tens
 // shared memory, kXsSlots chunks of [kMaxBatch][kBChunk] at a padded pitch
 constexpr int kXsPitchBytes = 1024 * 2 + 16;
 constexpr int kXsSlots = 3;
-constexpr int kMaxRows = 256;                          // rows per GEMV instruction
 constexpr int kRedFloats = 4096;                       // cross-warp reduction buffer
 constexpr int kMaxBatch = 8;
 constexpr int kMaxGroup = 8;                           // query heads per KV head
 constexpr int kMaxHeadDim = 128;
 constexpr int kTraceStamps = 8;                        // per-instruction trace words
-constexpr uint32_t kDefaultCopyPiece = 32 * 1024;  // bytes per bulk copy
-constexpr uint32_t kL2AheadBytes = 256 * 1024;     // batch-1 kernel: L2 prefetch beyond the ring per instruction
+constexpr uint32_t kDefaultL2Ahead = 512 * 1024;  // batch-1 kernel: weight bytes prefetched into L2 ahead
 
 // ---- dependency counters -----------------------------------------------------
 // Each counter is bumped once per producing instruction per step; a waiter
@@ -73,45 +71,28 @@ inline int counter_embed(int n_layers) { return n_layers * C_PER_LAYER; }
 inline int counter_lmhead(int n_layers) { return n_layers * C_PER_LAYER + 1; }
 inline int n_counters(int n_layers) { return n_layers * C_PER_LAYER + 2; }
 
-// ---- GEMV tiling (host and device agree on it) -------------------------------
-// A GEMV instruction streams full rows of K bf16.  The 256 consumer threads
-// split each row over `tpr` threads (16-byte vectors, round-robin), so rpp =
-// 256 / tpr rows are in flight at once and each thread keeps nv = ceil(K/8/tpr)
-// input vectors of 8 floats in registers for the whole instruction.
-struct GemvTile {
-  int tpr, rpp, nv, rows_per_stage;
-};
-
-MK_HD GemvTile gemv_tile(int K, int n_mats) {
-  GemvTile t;
-  int vt = K / 8;
-  int tpr = 32;
-  while (tpr < vt && tpr < kConsumerThreads) tpr *= 2;
-  t.tpr = tpr;
-  t.rpp = kConsumerThreads / tpr;
-  t.nv = (vt + tpr - 1) / tpr;
-  int r = kStageBytes / (K * 2 * n_mats);
-  // rows per thread per stage: at most 16 / (vectors x matrices), so that the
-  // loads in flight and the accumulators stay within the register budget
-  const int nvp = t.nv > 2 ? 4 : t.nv > 1 ? 2 : 1;
-  int rpt = 16 / (nvp * n_mats);
-  if (rpt > 8) rpt = 8;
-  int cap = rpt * t.rpp;
-  if (r > cap) r = cap;
-  t.rows_per_stage = r;
-  return t;
-}
-
-// Rows longer than 8 vectors per thread are streamed in ks column slices of
-// K/ks (each slice a separate pass over the same rows); 0 = unsupported.
-MK_HD int gemv_ksplit(int K, int n_mats) {
-  for (int ks = 1; ks <= 4; ks *= 2) {
-    if (K % (8 * ks)) break;
-    const GemvTile t = gemv_tile(K / ks, n_mats);
-    if (t.nv <= 8 && t.rows_per_stage >= 1) return ks;
-  }
-  return 0;
-}
+// ---- batch-1 GEMV tiling (host and device agree on it) -----------------------
+// Row-stationary tiles: an instruction owns `lines` weight rows (rows x matrices;
+// gate/up pairs count twice) and streams K in chunks of kB1Chunk columns.  A
+// stage holds every line of the instruction for `nc` consecutive chunks, each
+// line a 512-byte row of shared memory, moved by 2-D TMA boxes of 8 rows or 1
+// row (no swizzle).  Consumer warp w owns the rows r == w (mod 8) of every
+// stage and keeps their partial dot products in registers across all chunks:
+// one warp reduction per instruction, none per stage.
+constexpr int kB1Chunk = 256;          // columns per chunk (the TMA box width)
+constexpr int kB1LineBytes = kB1Chunk * 2;
+constexpr int kB1MaxLines = 64;        // lines per instruction (64 x 512 B = one stage)
+constexpr int kB1BoxHeights = 5;       // box maps of 16, 8, 4, 2 and 1 rows per matrix
+constexpr int kB1MapsPerLayer = 7 * kB1BoxHeights;  // wq wk wv wo w_gate w_up w_down
+// The input vector of a batch-1 GEMV sits in shared memory (fp32, the norm's
+// gain applied) in pieces of at most kB1XPieceFloats columns, loaded once per
+// piece with one round trip to L2: the same op's next instruction on the SM
+// reuses it, and a K longer than a piece reloads mid-instruction.
+constexpr int kB1XPieceFloats = 6144;
+MK_HD int b1_max_rows(int op) { return op == OP_GATEUP ? kB1MaxLines / 2 : kB1MaxLines; }
+// chunks per stage: as many as fill a stage with the instruction's lines
+MK_HD int b1_chunks_per_stage(int lines) { return lines > 32 ? 1 : (lines > 16 ? 2 : 4); }
+static_assert(kB1MaxLines * kB1LineBytes == kStageBytes, "a stage of 64 lines fills a ring slot");
 
 // ---- batch > 1 GEMV (tensor cores) -------------------------------------------------
 // A stage is one tile of 16 A-operand rows (16 weight rows, or 8 gate rows over
@@ -161,6 +142,10 @@ MK_HD int64_t even_begin(int64_t U, int n, int j) {
 // heads than this is split into head groups, each a separate instruction
 // over the same cache chunk (keeps the per-thread accumulators in registers).
 MK_HD int attn_heads_per_instr(int group) { return group > 4 ? 4 : group; }
+
+// The merging piece of an attention row loads the partial outputs of its
+// first kMergeAhead pieces together with their (m, l) pairs.
+constexpr int kMergeAhead = 8;
 
 // Positions of K (or V) that fit one ring slot.
 MK_HD int attn_stage_positions(int head_dim) { return kStageBytes / (head_dim * 2); }

@@ -43,6 +43,17 @@ struct Ctl {
   int waiting;    // the consumers are blocked on a dependency counter
   int last;       // attention: this CTA merges (broadcast)
   int flag;       // generic broadcast
+  uint32_t xtag;  // batch-1 GEMV: which input piece the reduction buffer holds (0: none)
+  float xss;      // and, for a norm-fused op, the sum of squares of its input
+  float b1red[kB1MaxLines * 4];  // batch-1 GEMV: per-warp sums of lines split over chunks
+  // batch-1 GEMV, the producer's current instruction: its TMA boxes for one
+  // chunk (tensor map, row, shared-memory offset within the chunk's lines)
+  struct B1Box {
+    const uint8_t* map;
+    int row;
+    uint32_t off;
+  } b1box[kB1MaxLines];
+  int b1nbox;
   float sred[kConsumerWarps * 2];
   float qs[kMaxGroup * kMaxHeadDim];
   float aml[kConsumerWarps * kMaxGroup * 2];  // attention: per-warp (m, l) of every head
@@ -68,8 +79,10 @@ struct Smem {
   static constexpr size_t kSlot = (size_t)kStageBytes;
   static_assert(2 * kBBoxBytes == kStageBytes, "a batched GEMV stage is two boxes");
   static constexpr size_t kRing = (size_t)kNst * kSlot;
-  // the reduction buffer doubles as the tensor-core kernel's input ring (never both at once)
-  static constexpr size_t kXs = BATCHED ? (size_t)kXsSlots * kMaxBatch * kXsPitchBytes : 0;
+  // the reduction buffer doubles as the GEMV input buffer (never both at once): the
+  // tensor-core kernel's input ring, the batch-1 kernel's input piece
+  static constexpr size_t kXs = BATCHED ? (size_t)kXsSlots * kMaxBatch * kXsPitchBytes
+                                        : (size_t)kB1XPieceFloats * sizeof(float);
   static constexpr size_t kRed = (size_t)kRedFloats * sizeof(float) > kXs ? (size_t)kRedFloats * sizeof(float) : kXs;
   static constexpr size_t kTotal = kRing + kRed + sizeof(Ctl);
   static_assert(kNst <= kStages, "Ctl holds kStages barrier pairs");
@@ -140,6 +153,16 @@ __device__ __forceinline__ void tma_box3(void* dst, const void* map, int c0, int
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
       "%3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
       "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar)), "l"(pol)
+      : "memory");
+}
+
+// One box of a 2-D tensor map (column c0, row c1) into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_box2(void* dst, const void* map, int c0, int c1, unsigned long long* bar,
+                                         uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
 }
 
@@ -333,6 +356,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// 16-byte loads from shared memory at a 32-bit shared address.
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+// The same, predicated: zeros where `pred` is 0 (no branch around the load).
+__device__ __forceinline__ uint4 lds_u4_if(uint32_t a, uint32_t pred) {
+  uint4 v;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %5, 0;\n\t"
+      "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+      "@p ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n\t}"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "r"(a), "r"(pred));
+  return v;
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+
 // Four 8x8 b16 matrices from shared memory, transposed on the way: lane
 // (g, c) receives elements (2c, g) and (2c + 1, g) of every stored matrix.
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t a[4], uint32_t saddr) {
@@ -376,94 +422,119 @@ __device__ __forceinline__ void set_status(const Params& p, int code, int detail
 // ---------------------------------------------------------------------------
 // A GEMV instruction covers rows [r0, r1) of its op's row space.  For QKV that
 // space is wq | wk | wv concatenated, so an instruction may span up to three
-// matrices ("segments"); a stage never crosses a segment.  Fields are named
-// (not arrays) so that the geometry stays in registers.
+// matrices ("segments").  Fields are named (not arrays) so that the geometry
+// stays in registers.
 struct Gemv {
-  const uint16_t *sw0, *sw1, *sw2;  // first row of each segment
-  const uint16_t* wup;              // gate/up: first row of the up matrix (one segment)
-  int sn0, sn1, sn2, nseg;          // rows per segment
   int K, r0, r1;
-  int ks, Kc;                       // column slices per row, slice width (K = ks * Kc)
-  GemvTile tile;                    // tiling of one slice
+  bool gated;  // gate/up: every row is a pair of lines, gate then up
   // batch > 1 (tensor cores): bnch chunks of kBChunk columns, bnt tiles of
   // btile_rows() output rows
   int bnch, bnt;
-  __device__ __forceinline__ const uint16_t* seg_ptr(int s) const { return s == 0 ? sw0 : (s == 1 ? sw1 : sw2); }
-  // first element of row r0 + rel (rel < r1 - r0), whichever matrix holds it
-  __device__ __forceinline__ const uint16_t* row_ptr(int rel) const {
-    if (rel < sn0) return sw0 + (size_t)rel * K;
-    rel -= sn0;
-    if (rel < sn1) return sw1 + (size_t)rel * K;
-    return sw2 + (size_t)(rel - sn1) * K;
-  }
-  __device__ __forceinline__ int seg_rows(int s) const { return s == 0 ? sn0 : (s == 1 ? sn1 : sn2); }
+  // batch 1 (row-stationary tiles): lines of the instruction, chunks of
+  // kB1Chunk columns, chunks per stage, stages; per segment its 8-row box map
+  // (the 1-row box map follows it), first row within its matrix, rows, first
+  // line within a stage and first weight of its first row (L2 prefetch)
+  int lines, nch, ncs, nst, nseg;
+  const uint8_t *bm0, *bm1, *bm2;
+  const uint16_t *bw0, *bw1, *bw2;
+  int brow0, brow1, brow2, bn0, bn1, bn2, bl0, bl1, bl2;
+  __device__ __forceinline__ int seg_rows(int s) const { return s == 0 ? bn0 : (s == 1 ? bn1 : bn2); }
+  __device__ __forceinline__ int seg_row(int s) const { return s == 0 ? brow0 : (s == 1 ? brow1 : brow2); }
+  __device__ __forceinline__ int seg_line(int s) const { return s == 0 ? bl0 : (s == 1 ? bl1 : bl2); }
+  __device__ __forceinline__ const uint8_t* seg_map(int s) const { return s == 0 ? bm0 : (s == 1 ? bm1 : bm2); }
+  __device__ __forceinline__ const uint16_t* seg_w(int s) const { return s == 0 ? bw0 : (s == 1 ? bw1 : bw2); }
 };
+
+// Batch-1 box maps of matrix `mat` (0..6: wq wk wv wo w_gate w_up w_down) of
+// a layer: kB1BoxHeights maps, of 16, 8, 4, 2 and 1 rows.
+__device__ __forceinline__ const uint8_t* b1_map(const Params& p, int layer, int mat) {
+  return p.tmaps_b1 + ((size_t)layer * kB1MapsPerLayer + kB1BoxHeights * mat) * 128;
+}
 
 __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, int op, int layer) {
   Gemv g;
-  g.wup = nullptr;
   g.r0 = in.a;
   g.r1 = in.b;
+  g.gated = op == OP_GATEUP;
+  const int R = g.r1 - g.r0;
   g.nseg = 1;
-  g.sn0 = g.r1 - g.r0;
-  g.sn1 = g.sn2 = 0;
-  g.sw1 = g.sw2 = nullptr;
+  g.bn0 = R;
+  g.bn1 = g.bn2 = 0;
+  g.brow0 = g.r0;
+  g.brow1 = g.brow2 = 0;
+  g.bl0 = 0;
+  g.bl1 = g.bl2 = 0;
+  g.bm0 = g.bm1 = g.bm2 = nullptr;
+  g.bw0 = g.bw1 = g.bw2 = nullptr;
   if (op == OP_LMHEAD) {
     g.K = p.H;
-    g.sw0 = p.lm_head + (size_t)g.r0 * g.K;
+    if (!p.tc) {
+      g.bm0 = p.tmaps_b1 + (size_t)p.L * kB1MapsPerLayer * 128;
+      g.bw0 = p.lm_head + (size_t)g.r0 * g.K;
+    }
   } else {
     const LayerPtrs& lp = p.layers[layer];
     switch (op) {
       case OP_QKV: {
         g.K = p.H;
-        const int qd = p.nq * p.hd, kvd = p.nkv * p.hd;
-        g.nseg = 0;
+        if (!p.tc) {
+          const int qd = p.nq * p.hd, kvd = p.nkv * p.hd;
+          g.nseg = 0;
 #pragma unroll
-        for (int m = 0; m < 3; ++m) {
-          const int base = m == 0 ? 0 : (m == 1 ? qd : qd + kvd);
-          const int end = m == 0 ? qd : (m == 1 ? qd + kvd : qd + 2 * kvd);
-          const uint16_t* mat = m == 0 ? lp.wq : (m == 1 ? lp.wk : lp.wv);
-          const int a = max(g.r0, base), b = min(g.r1, end);
-          if (a < b) {
-            const uint16_t* w = mat + (size_t)(a - base) * g.K;
-            if (g.nseg == 0) { g.sw0 = w; g.sn0 = b - a; }
-            else if (g.nseg == 1) { g.sw1 = w; g.sn1 = b - a; }
-            else { g.sw2 = w; g.sn2 = b - a; }
-            ++g.nseg;
+          for (int m = 0; m < 3; ++m) {
+            const int base = m == 0 ? 0 : (m == 1 ? qd : qd + kvd);
+            const int end = m == 0 ? qd : (m == 1 ? qd + kvd : qd + 2 * kvd);
+            const uint16_t* mat = m == 0 ? lp.wq : (m == 1 ? lp.wk : lp.wv);
+            const int a = max(g.r0, base), b = min(g.r1, end);
+            if (a < b) {
+              const uint8_t* map = b1_map(p, layer, m);
+              const uint16_t* w = mat + (size_t)(a - base) * g.K;
+              if (g.nseg == 0) { g.bm0 = map; g.bw0 = w; g.brow0 = a - base; g.bn0 = b - a; g.bl0 = a - g.r0; }
+              else if (g.nseg == 1) { g.bm1 = map; g.bw1 = w; g.brow1 = a - base; g.bn1 = b - a; g.bl1 = a - g.r0; }
+              else { g.bm2 = map; g.bw2 = w; g.brow2 = a - base; g.bn2 = b - a; g.bl2 = a - g.r0; }
+              ++g.nseg;
+            }
           }
         }
         break;
       }
       case OP_OPROJ:
         g.K = p.nq * p.hd;
-        g.sw0 = lp.wo + (size_t)g.r0 * g.K;
+        if (!p.tc) { g.bm0 = b1_map(p, layer, 3); g.bw0 = lp.wo + (size_t)g.r0 * g.K; }
         break;
       case OP_GATEUP:
         g.K = p.H;
-        g.sw0 = lp.w_gate + (size_t)g.r0 * g.K;
-        g.wup = lp.w_up + (size_t)g.r0 * g.K;
+        if (!p.tc) {  // gate rows, then the same rows of up
+          g.nseg = 2;
+          g.bm0 = b1_map(p, layer, 4);
+          g.bm1 = b1_map(p, layer, 5);
+          g.bw0 = lp.w_gate + (size_t)g.r0 * g.K;
+          g.bw1 = lp.w_up + (size_t)g.r0 * g.K;
+          g.brow1 = g.r0;
+          g.bn1 = R;
+          g.bl1 = R;
+        }
         break;
       case OP_ROUTER:
         g.K = p.H;
-        g.sw0 = lp.router + (size_t)g.r0 * g.K;
         break;
       case OP_EXP_DOWN:  // rows of every picked expert's down matrix (tensor maps)
         g.K = p.Ie;
-        g.sw0 = lp.w_down;
         break;
       default:  // OP_DOWN
         g.K = p.I;
-        g.sw0 = lp.w_down + (size_t)g.r0 * g.K;
+        if (!p.tc) { g.bm0 = b1_map(p, layer, 6); g.bw0 = lp.w_down + (size_t)g.r0 * g.K; }
         break;
     }
   }
-  g.ks = gemv_ksplit(g.K, g.wup ? 2 : 1);
-  g.Kc = g.K / g.ks;
-  g.tile = gemv_tile(g.Kc, g.wup ? 2 : 1);
+  g.lines = R * (g.gated ? 2 : 1);
+  g.nch = (g.K + kB1Chunk - 1) / kB1Chunk;
+  g.ncs = b1_chunks_per_stage(g.lines);
+  g.nst = (g.nch + g.ncs - 1) / g.ncs;
   if (p.tc) {
-    const int tr = btile_rows(g.wup != nullptr);
+    const int tr = btile_rows(g.gated);
     g.bnch = (g.K + kBChunk - 1) / kBChunk;
-    g.bnt = (g.r1 - g.r0 + tr - 1) / tr;
+    g.bnt = (R + tr - 1) / tr;
   }
   return g;
 }
@@ -482,19 +553,11 @@ __device__ __forceinline__ Gemv moe_gate_piece(const Params& p, const Ctl* ctl, 
   const int64_t left = g1 - g < (int64_t)(kBatchedMaxRowsGated / 8) ? g1 - g : (int64_t)(kBatchedMaxRowsGated / 8);
   const int t1 = (int)(nte - t0 < left ? nte : t0 + left);
   const int e = ctl->moe_uniq[s];
-  const LayerPtrs& lp = p.layers[layer];
   Gemv gm;
   gm.K = p.H;
   gm.r0 = e * p.Ie + t0 * 8;
   gm.r1 = e * p.Ie + t1 * 8;
-  gm.nseg = 1;
-  gm.sn0 = gm.r1 - gm.r0;
-  gm.sn1 = gm.sn2 = 0;
-  gm.sw0 = lp.w_gate;
-  gm.sw1 = gm.sw2 = nullptr;
-  gm.wup = lp.w_up;
-  gm.ks = 1;
-  gm.Kc = gm.K;
+  gm.gated = true;
   gm.bnch = (p.H + kBChunk - 1) / kBChunk;
   gm.bnt = t1 - t0;
   *slot = s;
@@ -653,56 +716,33 @@ struct Cursor {
       }
       return;
     }
-    rr += g.tile.rows_per_stage;
-    if (rr >= g.seg_rows(sg)) {
-      rr = 0;
-      if (++sg >= g.nseg) {
-        sg = 0;
-        if (++kc >= g.ks) seek(i + 1);
-      }
-    }
+    if (++kc >= g.nst) seek(i + 1);  // batch-1 GEMV: stage kc of the row-stationary tiles
   }
 
-  // f(src, bytes, smem offset) for every copy of the current stage; returns the stage's bytes.
-  template <typename F>
-  __device__ __forceinline__ uint32_t copies(F&& f) const {
-    const int R = g.tile.rows_per_stage;
-    const int nr = min(R, g.seg_rows(sg) - rr);
-    const uint32_t seg = (uint32_t)g.Kc * 2u;
-    const size_t off = (size_t)rr * g.K + (size_t)kc * g.Kc;
-    const uint32_t bytes = (uint32_t)nr * seg;
-    for (int m = 0; m < (g.wup ? 2 : 1); ++m) {
-      const uint16_t* src = (m ? g.wup : g.seg_ptr(sg)) + off;
-      const uint32_t base = (uint32_t)m * R * seg;
-      if (g.ks == 1) {
-        // several concurrent bulk copies per stage keep more requests in flight
-        const uint32_t piece = pp->copy_piece;
-        for (uint32_t o = 0; o < bytes; o += piece)
-          f(src + o / 2, min(piece, bytes - o), base + o);
-      } else {
-        for (int r = 0; r < nr; ++r) f(src + (size_t)r * g.K, seg, base + r * seg);
+  // Batch-1 GEMV: the TMA boxes of one chunk of every line, into `box` (the
+  // same for every chunk but for the column): a segment's rows as boxes of 16,
+  // 8, 4, 2 and 1 rows, largest first (single rows only when K is narrower
+  // than a chunk, whose boxes are K wide).  Chunk j's line l lands at
+  // shared-memory line (j - first chunk of the stage) * lines + l.  Returns
+  // the number of boxes.
+  __device__ __forceinline__ int b1_box_list(Ctl::B1Box* box) const {
+    const bool wide = g.K >= kB1Chunk;
+    int nb = 0;
+    for (int s2 = 0; s2 < g.nseg; ++s2) {
+      const uint8_t* map = g.seg_map(s2);
+      const int n = g.seg_rows(s2), row = g.seg_row(s2), line = g.seg_line(s2);
+      int r = 0;
+      for (int m = wide ? 0 : kB1BoxHeights - 1; m < kB1BoxHeights; ++m) {
+        const int h = 16 >> m;
+        for (; r + h <= n; r += h) {
+          box[nb].map = map + 128 * m;
+          box[nb].row = row + r;
+          box[nb].off = (uint32_t)(line + r) * kB1LineBytes;
+          ++nb;
+        }
       }
     }
-    return g.wup ? 2 * bytes : bytes;
-  }
-
-  // Batch-1 GEMV: bring into L2 up to `budget` bytes of the rows the ring
-  // has not reached yet (whole rows from the current one to the end of the
-  // instruction; the gate/up pair's up rows alongside).  Row blocks are
-  // contiguous, so this is one prefetch per matrix segment.
-  __device__ __forceinline__ void prefetch_rest(uint32_t budget) const {
-    if (op == OP_ATTN || pp->tc || i >= n) return;
-    const size_t rowb = (size_t)g.K * 2;
-    for (int s2 = sg; s2 < g.nseg && budget >= 16; ++s2) {
-      const int from = s2 == sg ? rr : 0;
-      const size_t left = (size_t)(g.seg_rows(s2) - from) * rowb * (g.wup ? 2 : 1);
-      if (left == 0) continue;
-      const uint32_t take = (uint32_t)(left < budget ? left : budget) / (g.wup ? 2u : 1u) & ~15u;
-      if (take == 0) break;
-      prefetch_l2(g.seg_ptr(s2) + (size_t)from * g.K, take);
-      if (g.wup) prefetch_l2(g.wup + (size_t)from * g.K, take);
-      budget -= take * (g.wup ? 2u : 1u);
-    }
+    return nb;
   }
 
   // Batched GEMV stage: f(tensor map, row, column block, shared-memory
@@ -713,7 +753,7 @@ struct Cursor {
   __device__ __forceinline__ uint32_t boxes(F&& f) const {
     const Params& p = *pp;
     const int kb = kc * (kBChunk / 64);
-    if (g.wup) {
+    if (g.gated) {
       const uint8_t* m = p.tmaps + ((size_t)layer * kTmapsPerLayer + 4) * 128;
       const int row = g.r0 + sg * 8;
       f(m, row, kb, 0u);
@@ -755,9 +795,10 @@ struct Cursor {
   __device__ __forceinline__ uint32_t stage_bytes() const {
     if (op == OP_ATTN)
       return (uint32_t)kStageBytes;  // a TMA box: always a whole stage of positions
-    if (pp->tc) return (g.wup || g.r1 - g.r0 - sg * 16 > 8) ? 2u * kBBoxBytes : (uint32_t)kBBoxBytes;
-    const uint32_t b = (uint32_t)min(g.tile.rows_per_stage, g.seg_rows(sg) - rr) * (uint32_t)g.Kc * 2u;
-    return g.wup ? 2 * b : b;
+    if (pp->tc) return (g.gated || g.r1 - g.r0 - sg * 16 > 8) ? 2u * kBBoxBytes : (uint32_t)kBBoxBytes;
+    // batch 1: every line of every chunk of the stage, one box width each
+    const int j0 = kc * g.ncs, nj = min(g.nch, j0 + g.ncs) - j0;
+    return (uint32_t)(g.lines * nj) * (uint32_t)min(g.K, kB1Chunk) * 2u;
   }
 };
 
@@ -830,15 +871,64 @@ struct Producer {
   }
 };
 
+// The cached K and V bytes an attention slot instruction streams this step
+// (its pieces' positions before the new token), optionally prefetched into L2
+// one ring stage at a time.
+__device__ __noinline__ uint64_t attn_kv_bytes(const Params& p, const mk_instr& in, int layer, bool prefetch) {
+  AttnSched sc;
+  attn_sched(p, in, sc);
+  const int j = in.a;
+  uint64_t total = 0;
+  for (int64_t gg = attn_slot_begin(sc, j), g1 = attn_slot_begin(sc, j + 1); gg < g1;) {
+    const AttnPiece pc = attn_piece_at(sc, gg, j);
+    gg += pc.ub - pc.ua;
+    const Attn a = attn_geo(p, pc, layer, p.hd);
+    for (int sub = 0; sub < a.nsub; ++sub) {
+      const uint32_t bytes = (uint32_t)min(a.P, a.n_cached - sub * a.P) * (uint32_t)p.hd * 2u;
+      if (prefetch) {
+        const int64_t row = kv_row(p, layer, a.b, a.kvh, a.p0 + sub * a.P);
+        prefetch_l2(p.kc + row * p.hd, bytes);
+        prefetch_l2(p.vc + row * p.hd, bytes);
+      }
+      total += 2u * bytes;
+    }
+  }
+  return total;
+}
+
+// Batch-1 GEMV instruction: its weight bytes (every segment's row block),
+// optionally prefetched into L2 (each segment's rows are one contiguous block).
+__device__ __noinline__ uint64_t b1_weight_bytes(const Params& p, const mk_instr& in, bool prefetch) {
+  const int op = op_of(in.op_layer);
+  const Gemv g = gemv_geo(p, in, op, layer_of(in.op_layer));
+  if (prefetch)
+    for (int s2 = 0; s2 < g.nseg; ++s2) {
+      const uint32_t bytes = (uint32_t)g.seg_rows(s2) * (uint32_t)g.K * 2u;
+      if (bytes) prefetch_l2(g.seg_w(s2), bytes);
+    }
+  return (uint64_t)g.lines * g.K * 2u;
+}
+
 // One thread (lane 0 of the producer warp) issues every copy.
+//
+// Batch-1 kernel: besides the ring, the producer keeps an L2 runway: the
+// weight blocks of the instructions after the current one are prefetched into
+// L2, up to p.l2_ahead bytes ahead of the instruction the ring is filling, so
+// that HBM keeps streaming while the consumers wait on a dependency and the
+// ring is full; an attention slot's runway is the cached K/V positions of its
+// pieces.
 template <bool BATCHED>
 __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
   Producer<BATCHED> pr(p, ctl, ring);
   uint64_t* trace = p.trace ? p.trace + (size_t)p.offsets[blockIdx.x] * kTraceStamps : nullptr;
   Cursor cur(p, list, n, &ctl->psched, ctl);
   cur.seek(0);
+  // runway (batch 1): instructions [.., pf_i) prefetched; cum_pf / cum_cur =
+  // their bytes / the bytes of the instructions up to the current one
+  int pf_i = 0, entered = -1;
+  uint64_t cum_pf = 0, cum_cur = 0;
   bool ok = true;
-  int last = -1, pf_instr = -1;
+  int last = -1;
   while (cur.i < n) {
     if (cur.pending) {  // an expert instruction: its weights follow from the routing
       if (!(ok = pr.wait_routing(cur.layer))) break;
@@ -852,18 +942,53 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
       for (int j = last + 1; j <= cur.i; ++j) trace[j * kTraceStamps + 3] = now;
       last = cur.i;
     }
+    if (!BATCHED) {
+      if (p.l2_ahead && cur.i != entered) {
+        entered = cur.i;
+        cum_cur += cur.op == OP_ATTN ? attn_kv_bytes(p, list[cur.i], cur.layer, false)
+                                     : b1_weight_bytes(p, list[cur.i], false);
+        if (pf_i <= cur.i) {  // the runway restarts after the current instruction
+          pf_i = cur.i + 1;
+          cum_pf = cum_cur;
+        }
+        while (pf_i < n && cum_pf < cum_cur + p.l2_ahead) {
+          const mk_instr in = list[pf_i];
+          const int op = op_of(in.op_layer);
+          if (op == OP_ATTN)
+            cum_pf += attn_kv_bytes(p, in, layer_of(in.op_layer), true);
+          else if (op >= OP_QKV && op <= OP_LMHEAD)
+            cum_pf += b1_weight_bytes(p, in, true);
+          ++pf_i;
+        }
+      }
+      if (cur.op != OP_ATTN) {
+        // a batch-1 GEMV instruction: its box list once, then every stage from it
+        Ctl::B1Box* box = ctl->b1box;
+        const int nbox = cur.b1_box_list(box);
+        const int nch = cur.g.nch, ncs = cur.g.ncs, nst = cur.g.nst;
+        const uint32_t chunk_stride = (uint32_t)cur.g.lines * kB1LineBytes;
+        const uint32_t chunk_bytes = (uint32_t)cur.g.lines * (uint32_t)min(cur.g.K, kB1Chunk) * 2u;
+        for (int kc = 0; kc < nst && ok; ++kc) {
+          uint8_t* dst;
+          unsigned long long* bar;
+          if (!(ok = pr.claim(&dst, &bar, [&]() {}))) break;
+          const int j0 = kc * ncs, nj = min(nch - j0, ncs);
+          mbar_arrive_expect_tx(bar, chunk_bytes * (uint32_t)nj);
+          for (int jj = 0; jj < nj; ++jj) {
+            uint8_t* dj = dst + jj * chunk_stride;
+            const int col = (j0 + jj) * kB1Chunk;
+            for (int b = 0; b < nbox; ++b) tma_box2(dj + box[b].off, box[b].map, col, box[b].row, bar, pr.pol);
+          }
+          ++pr.k;
+        }
+        if (!ok) break;
+        cur.seek(cur.i + 1);
+        continue;
+      }
+    }
     uint8_t* dst;
     unsigned long long* bar;
-    // While the consumers wait on another SM with the ring full, HBM would
-    // idle: bring the rest of this instruction's weights into L2 (once per
-    // instruction), so the ring refills from L2 when the wait ends.
-    if (!(ok = pr.claim(&dst, &bar, [&]() {
-          if (!BATCHED && cur.i != pf_instr) {
-            pf_instr = cur.i;
-            cur.prefetch_rest(kL2AheadBytes);
-          }
-        })))
-      break;
+    if (!(ok = pr.claim(&dst, &bar, [&]() {}))) break;
     const uint32_t bytes = cur.stage_bytes();
     mbar_arrive_expect_tx(bar, bytes);
     if (cur.op == OP_ATTN) {
@@ -871,12 +996,10 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
       int row;
       cur.attn_box(&map, &row);
       tma_box3(dst, map, 0, row, 0, bar, pr.pol);
-    } else if (BATCHED) {
+    } else {
       cur.boxes([&](const uint8_t* map, int row, int kb, uint32_t off) {
         tma_box3(dst + off, map, 0, row, kb, bar, pr.pol);
       });
-    } else {
-      cur.copies([&](const uint16_t* src, uint32_t b, uint32_t off) { bulk_g2s(dst + off, src, b, bar, pr.pol); });
     }
     ++pr.k;
     cur.advance();
@@ -993,179 +1116,189 @@ struct Consumer {
     }
   }
 
-  // ---- GEMV ------------------------------------------------------------------
-  // Input vector x (fp32, written by other CTAs) optionally RMS-normalised
-  // with a bf16 gain; each thread keeps its NVT vectors in registers.
-  // Gains of the RMSNorm prologue are weights: fetch them before the dependency wait.
-  template <int NVT, bool NORM>
-  __device__ __forceinline__ void load_gain(const uint16_t* gain, int K, const GemvTile& tl, uint4 graw[NVT]) {
-    const int ct = t % tl.tpr, vt = K / 8;
-#pragma unroll
-    for (int j = 0; j < NVT; ++j) {
-      const int v = ct + j * tl.tpr;
-      graw[j] = NORM && v < vt ? __ldg(reinterpret_cast<const uint4*>(gain + v * 8)) : make_uint4(0, 0, 0, 0);
-    }
-  }
-
-  template <int NVT, bool NORM>
-  __device__ __forceinline__ void load_x(const float* src, const uint4 graw[NVT], int K, const GemvTile& tl,
-                                         float xr[NVT][8]) {
-    // One pass: every group of tpr threads holds all of x, so the block sum
-    // of the per-thread squares counts each element rpp times (a power of 2).
-    const int ct = t % tl.tpr, vt = K / 8;
-
-    float ss = 0.f;
-#pragma unroll
-    for (int j = 0; j < NVT; ++j) {
-      const int v = ct + j * tl.tpr;
-      if (v < vt) {
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(src + v * 8));
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(src + v * 8) + 1);
-        xr[j][0] = a.x; xr[j][1] = a.y; xr[j][2] = a.z; xr[j][3] = a.w;
-        xr[j][4] = b.x; xr[j][5] = b.y; xr[j][6] = b.z; xr[j][7] = b.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
-      }
-      if (NORM) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
-      }
-    }
-    if (NORM) {
-      ss = block_sum(ss) / (float)tl.rpp;
-      const float scale = 1.f / sqrtf(ss / (float)K + p.eps);
-#pragma unroll
-      for (int j = 0; j < NVT; ++j)
-        if (ct + j * tl.tpr < vt) {
-          float gf[8];
-          unpack8(graw[j], gf);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xr[j][e] = xr[j][e] * scale * gf[e];
-        }
-    }
-  }
-
-  // Stream the instruction's stages, leaving per-(row, warp) partial dots in red.
-  // Each thread accumulates RPT rows of the stage (rows rs, rs+rpp, ...) and
-  // the warp reduces all of them at once with warp_reduce_multi.
-  template <int NVT, int RPT, bool GATED>
-  __device__ __forceinline__ void gemv_stream(const Gemv& g, const float xr[NVT][8], int kc) {
-    constexpr int NM = GATED ? 2 : 1;
-    const GemvTile& tl = g.tile;
-    const int R = tl.rows_per_stage, K = g.Kc, vt = K / 8;
-    const int rs = t / tl.tpr, ct = t % tl.tpr, wpr = tl.tpr / 32, wir = ct / 32;
-    const int q = row_of_lane<RPT * NM>(lane);
-    const bool writer = (lane & (32 / (RPT * NM) - 1)) == 0;
-    unsigned long long xp[NVT][4];  // the input slice as fp32 pairs
-#pragma unroll
-    for (int j = 0; j < NVT; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) xp[j][e] = pack2(xr[j][2 * e], xr[j][2 * e + 1]);
-    int rl = 0;  // first row of the segment within the instruction
-#pragma unroll 1
-    for (int sg = 0; sg < g.nseg; ++sg) {
-      const int nr = g.seg_rows(sg);
-#pragma unroll 1
-    for (int rr = 0; rr < nr; rr += R) {
-      const int n = min(R, nr - rr);
-      const uint16_t* w0 = reinterpret_cast<const uint16_t*>(wait_full());
-      if (tr && kc == 0 && sg == 0 && rr == 0) tr[5] = globaltimer();
-      const uint16_t* w1 = w0 + (size_t)R * K;
-      float acc[RPT * NM];
-#pragma unroll
-      for (int k = 0; k < RPT; ++k) {
-        const int i = rs + k * tl.rpp;
-        unsigned long long a0 = 0ull, a1 = 0ull;  // (+0.0f, +0.0f) pairs
-#pragma unroll
-        for (int j = 0; j < NVT; ++j) {
-          const int v = ct + j * tl.tpr;
-          if (i < n && v < vt) {
-            a0 = dot8x2(*reinterpret_cast<const uint4*>(w0 + (size_t)i * K + v * 8), xp[j], a0);
-            if (GATED) a1 = dot8x2(*reinterpret_cast<const uint4*>(w1 + (size_t)i * K + v * 8), xp[j], a1);
-          }
-        }
-        acc[k] = sum2(a0);
-        if (GATED) acc[RPT + k] = sum2(a1);
-      }
-      const float sum = warp_reduce_multi<RPT * NM>(acc, lane);
-      if (writer) {
-        const int k = q % RPT, which = q / RPT;
-        const int i = rs + k * tl.rpp;
-        if (i < n) {
-          float* dst = red + ((rl + rr + i) * NM + which) * wpr + wir;
-          *dst = (kc ? *dst : 0.f) + sum;  // the same thread owns this slot in every slice pass
-        }
-      }
-      release();
-    }
-      rl += nr;
-    }
-    if (tr) tr[6] = globaltimer();
-    consumer_bar();
-  }
-
-  template <int NVT, int RPT, bool NORM, bool GATED>
-  __device__ __forceinline__ bool gemv_run(const mk_instr& in, int op, int layer) {
+  // ---- GEMV, batch 1: row-stationary tiles ------------------------------------
+  // Stage s holds chunks [s * ncs, ...) of every line of the instruction, each
+  // line kB1Chunk bf16 weights (512 bytes); a stage holds at most 64 line
+  // chunks, so each warp has at most 8 of them.  With ncs chunks per stage,
+  // warp w takes chunk w % ncs of every stage and the lines w / ncs, w / ncs +
+  // 8 / ncs, ... (gate/up: those neurons, each a gate line and an up line);
+  // lane l covers the columns [8l, 8l + 8) of its chunk.  Partial dot products
+  // stay in registers (packed fp32 pairs) across all stages; at the end each
+  // warp reduces its lines across its lanes, and the ncs warps that share a
+  // line add their sums in a fixed order.  The input vector (fp32; times the
+  // RMSNorm gain for the norm-fused ops) is in the reduction buffer, loaded
+  // with one round trip to L2 per piece of kB1XPieceFloats columns and kept
+  // for the op's next instruction on this SM; the stream itself has no block
+  // barrier.  The norm's 1/rms is constant along K, so it scales the outputs;
+  // its sum of squares is taken from the same loads.
+  template <bool NORM, bool GATED>
+  __device__ __forceinline__ bool gemv_b1(const mk_instr& in, int op, int layer) {
     const Gemv g = gemv_geo(p, in, op, layer);
-    const int BH = p.B * p.H;
-    // input vector and prologue
+    const int H = p.H, K = g.K, lines = g.lines, R = g.r1 - g.r0, nch = g.nch, NCS = g.ncs;
     const float* src;
     const uint16_t* gain = nullptr;
     if (op == OP_QKV) {
-      src = p.xres + (size_t)(2 * layer) * BH;
+      src = p.xres + (size_t)(2 * layer) * H;
       gain = p.layers[layer].attn_norm;
     } else if (op == OP_OPROJ) {
       src = p.attn;
     } else if (op == OP_GATEUP) {
-      src = p.xres + (size_t)(2 * layer + 1) * BH;
+      src = p.xres + (size_t)(2 * layer + 1) * H;
       gain = p.layers[layer].mlp_norm;
     } else if (op == OP_DOWN) {
       src = p.act;
     } else {  // LM head
-      src = p.xres + (size_t)(2 * p.L) * BH;
+      src = p.xres + (size_t)(2 * p.L) * H;
       gain = p.final_norm;
     }
-    uint4 graw[NVT];
-    load_gain<NVT, NORM>(gain, g.Kc, g.tile, graw);
+    const int LSTEP = kConsumerWarps / NCS;  // warps per chunk: a warp's lines are LSTEP apart
+    const int cw = warp % NCS, lw = warp / NCS;
+    // this warp's item k: gate/up, neuron lw + LSTEP (k & 3) (gate line for k < 4,
+    // up line for k >= 4); otherwise line lw + LSTEP k.  own: the items that exist.
+    uint32_t own = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (GATED ? lw + LSTEP * (k & 3) < R : lw + LSTEP * k < lines) own |= 1u << k;
+    auto line_of = [&](int k) {
+      return GATED ? (k < 4 ? 0 : R) + lw + LSTEP * (k & 3) : lw + LSTEP * k;
+    };
+    // output rows: with one chunk per stage every warp finishes its own lines
+    // (writer lanes: the reduced item lane / 4); otherwise thread t < rows
+    // finishes row t from the per-warp sums
+    const int q = lane >> 2;
+    const bool writer = (lane & 3) == 0;
+    int orow = -1;
+    if (NCS == 1) {
+      if (writer && (GATED ? q < 4 : true) && ((own >> q) & 1u)) orow = g.r0 + lw + LSTEP * (q & (GATED ? 3 : 7));
+    } else if (t < R) {
+      orow = g.r0 + t;
+    }
     if (!wait_counter(in.wait_idx, in.wait_count)) return false;
     if (tr) tr[1] = globaltimer();
-    // residual rows for the epilogue, fetched before the weights stream
+    // residual row of the epilogue, fetched before the stream
     float resid = 0.f;
-    if ((op == OP_OPROJ || op == OP_DOWN) && t < g.r1 - g.r0)
-      resid = __ldcg(p.xres + (size_t)(2 * layer + (op == OP_DOWN ? 1 : 0)) * BH + g.r0 + t);
-    for (int kc = 0; kc < g.ks; ++kc) {  // ks > 1 only without a norm prologue
-      float xr[NVT][8];
-      load_x<NVT, NORM>(src + (size_t)kc * g.Kc, graw, g.Kc, g.tile, xr);
-      if (tr && kc == 0) tr[4] = globaltimer();
-      gemv_stream<NVT, RPT, GATED>(g, xr, kc);
+    if ((op == OP_OPROJ || op == OP_DOWN) && orow >= 0)
+      resid = __ldcg(p.xres + (size_t)(2 * layer + (op == OP_DOWN ? 1 : 0)) * H + orow);
+    // input piece: [chunk][half][lane] float4 (lane l's 8 columns of a chunk in two halves)
+    float4* xb = reinterpret_cast<float4*>(red);
+    const uint32_t xs0 = smem_addr(red);
+    const int pch = kB1XPieceFloats / kB1Chunk / NCS * NCS;  // chunks per piece, whole stages
+    const bool narrow = K < kB1Chunk;  // lines are K wide: lanes past K hold stale bytes
+    unsigned long long acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0ull;  // (+0.0f, +0.0f) pairs
+    int s = 0;  // stage
+    for (int c0 = 0; c0 < nch; c0 += pch) {
+      const int c1 = min(nch, c0 + pch);
+      const uint32_t tag = ((uint32_t)layer << 12 | (uint32_t)op << 6 | (uint32_t)(c0 / pch)) + 1u;
+      if (ctl->xtag != tag) {
+        if (c0 > 0) consumer_bar();  // every warp is done with the previous piece
+        float ss = 0.f;
+        for (int f = t; f < (c1 - c0) * 64; f += kConsumerThreads) {
+          const int col = c0 * kB1Chunk + 4 * f;
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (col < K) {
+            v = __ldcg(reinterpret_cast<const float4*>(src + col));
+            if (NORM) {
+              const uint2 gv = __ldg(reinterpret_cast<const uint2*>(gain + col));
+              ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+              v.x *= bf16_lo(gv.x);
+              v.y *= bf16_hi(gv.x);
+              v.z *= bf16_lo(gv.y);
+              v.w *= bf16_hi(gv.y);
+            }
+          }
+          const int ff = f & 63;
+          xb[((f >> 6) * 2 + (ff & 1)) * 32 + (ff >> 1)] = v;
+        }
+        if (NORM) {
+          ss = warp_sum(ss);
+          if (lane == 0) ctl->sred[warp] = ss;
+        }
+        consumer_bar();
+        if (t == 0) {
+          if (NORM) {
+            float s2 = 0.f;
+#pragma unroll
+            for (int w2 = 0; w2 < kConsumerWarps; ++w2) s2 += ctl->sred[w2];
+            ctl->xss = (c0 == 0 ? 0.f : ctl->xss) + s2;  // pieces of the same input, in order
+          }
+          ctl->xtag = tag;
+        }
+        consumer_bar();
+      }
+      if (tr && c0 == 0) tr[4] = globaltimer();
+      const int s1 = (c1 + NCS - 1) / NCS;
+#pragma unroll 1
+      for (; s < s1; ++s) {
+        const uint8_t* w = wait_full();
+        if (tr && s == 0) tr[5] = globaltimer();
+        const int c = s * NCS + cw;  // this warp's chunk
+        if (c < nch) {
+          // every load of the stage first (x, then the warp's own lines), then the arithmetic;
+          // shared-space loads on 32-bit shared addresses
+          const uint32_t xa = xs0 + (uint32_t)((c - c0) * 2 * 32 + lane) * 16u;
+          const float4 x0 = lds_f4(xa), x1 = lds_f4(xa + 512u);
+          const uint32_t wj = smem_addr(w) + (uint32_t)(cw * lines * kB1LineBytes + lane * 16);
+          // items the warp does not own (and, for a K narrower than a chunk, the
+          // lanes past K) load zeros: no branch, so the eight chains interleave
+          const uint32_t lanes_ok = !narrow || c * kB1Chunk + lane * 8 < K;
+          uint4 wv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            wv[k] = lds_u4_if(wj + (uint32_t)line_of(k) * kB1LineBytes, ((own >> k) & 1u) & lanes_ok);
+          const unsigned long long xp[4] = {pack2(x0.x, x0.y), pack2(x0.z, x0.w), pack2(x1.x, x1.y),
+                                            pack2(x1.z, x1.w)};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = dot8x2(wv[k], xp, acc[k]);
+        }
+        release();
+      }
     }
-    // epilogue: fixed-order sum of the per-warp partials, then the op's output
-    const int wpr = g.tile.tpr / 32, n = g.r1 - g.r0;
+    if (tr) tr[6] = globaltimer();
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = sum2(acc[k]);
+    float tot = warp_reduce_multi<8>(v, lane);  // item lane / 4 of this warp
+    float up = GATED ? __shfl_xor_sync(0xffffffffu, tot, 16) : 0.f;  // item q + 4: the up line of neuron q
+    if (NCS > 1) {
+      // the warps sharing a line add their sums in chunk order
+      if (writer && ((own >> q) & 1u) && (GATED ? q < 4 : true)) {
+        const int li = lw + LSTEP * (q & (GATED ? 3 : 7));
+        ctl->b1red[li * 4 + cw] = tot;
+        if (GATED) ctl->b1red[(kB1MaxLines / 2 + li) * 4 + cw] = up;
+      }
+      consumer_bar();
+      tot = up = 0.f;
+      if (orow >= 0) {
+        const int li = t;
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) {
+          if (c2 >= NCS) break;
+          tot += ctl->b1red[li * 4 + c2];
+          if (GATED) up += ctl->b1red[(kB1MaxLines / 2 + li) * 4 + c2];
+        }
+      }
+    }
+    const float scale = NORM ? 1.f / sqrtf(ctl->xss / (float)K + p.eps) : 1.f;
     const bool amx = op == OP_LMHEAD && p.argmax;
     unsigned long long best = 0ull;
-    for (int i = t; i < n; i += kConsumerThreads) {
-      const int row = g.r0 + i;
+    if (orow >= 0) {
       if (GATED) {
-        float gs = 0.f, us = 0.f;
-        for (int w = 0; w < wpr; ++w) {
-          gs += red[(i * 2) * wpr + w];
-          us += red[(i * 2 + 1) * wpr + w];
-        }
-        p.act[row] = gs / (1.f + expf(-gs)) * us;
-        continue;
-      }
-      float y = 0.f;
-      for (int w = 0; w < wpr; ++w) y += red[i * wpr + w];
-      if (op == OP_QKV) {
-        p.qkv[row] = y;  // q | k | v concatenated, like the instruction's rows
-      } else if (op == OP_OPROJ) {
-        p.xres[(size_t)(2 * layer + 1) * BH + row] = resid + y;
-      } else if (op == OP_DOWN) {
-        p.xres[(size_t)(2 * layer + 2) * BH + row] = resid + y;
+        const float gs = tot * scale, us = up * scale;
+        p.act[orow] = gs / (1.f + expf(-gs)) * us;
       } else {
-        p.logits[row] = y;
-        if (amx) best = max(best, argmax_key(y, row));
+        const float y = tot * scale;
+        if (op == OP_QKV) {
+          p.qkv[orow] = y;  // q | k | v concatenated, like the instruction's rows
+        } else if (op == OP_OPROJ) {
+          p.xres[(size_t)(2 * layer + 1) * H + orow] = resid + y;
+        } else if (op == OP_DOWN) {
+          p.xres[(size_t)(2 * layer + 2) * H + orow] = resid + y;
+        } else {
+          p.logits[orow] = y;
+          if (amx) best = argmax_key(y, orow);
+        }
       }
     }
     if (amx) {  // the instruction's arg-max: warps, then shared memory, then one global atomic
@@ -1179,24 +1312,6 @@ struct Consumer {
       }
     }
     return true;
-  }
-
-  // gemv_tile caps rows per thread at 16 / (NVT * matrices), at most 8.
-  template <int NVT, bool NORM, bool GATED>
-  __device__ __forceinline__ bool gemv_nv(const mk_instr& in, int op, int layer, int rpt) {
-    constexpr int CAP = 16 / (NVT * (GATED ? 2 : 1)) > 8 ? 8 : 16 / (NVT * (GATED ? 2 : 1));
-    if (rpt <= 1 || CAP == 1) return gemv_run<NVT, 1, NORM, GATED>(in, op, layer);
-    if (rpt <= 2 || CAP == 2) return gemv_run<NVT, 2, NORM, GATED>(in, op, layer);
-    if (rpt <= 4 || CAP == 4) return gemv_run<NVT, (CAP < 4 ? CAP : 4), NORM, GATED>(in, op, layer);
-    return gemv_run<NVT, CAP, NORM, GATED>(in, op, layer);
-  }
-
-  template <bool NORM, bool GATED>
-  __device__ __forceinline__ bool gemv_nvsel(const mk_instr& in, int op, int layer, int nv, int rpt) {
-    if (nv <= 1) return gemv_nv<1, NORM, GATED>(in, op, layer, rpt);
-    if (nv <= 2) return gemv_nv<2, NORM, GATED>(in, op, layer, rpt);
-    if (NORM || nv <= 4) return gemv_nv<4, NORM, GATED>(in, op, layer, rpt);
-    return gemv_nv<(NORM ? 4 : 8), NORM, GATED>(in, op, layer, rpt);
   }
 
   // ---- GEMV, batch > 1: tensor cores ---------------------------------------
@@ -1459,14 +1574,9 @@ struct Consumer {
         return gemv_tc<true, false>(g, op, layer, in.wait_idx, in.wait_count, -1);
       return gemv_tc<false, false>(g, op, layer, in.wait_idx, in.wait_count, -1);
     }
-    const bool norm = op == OP_QKV || op == OP_GATEUP || op == OP_LMHEAD;
-    const int K = op == OP_OPROJ ? p.nq * p.hd : (op == OP_DOWN ? p.I : p.H);
-    const int nm = op == OP_GATEUP ? 2 : 1;
-    const GemvTile tl = gemv_tile(K / gemv_ksplit(K, nm), nm);
-    const int rpt = (tl.rows_per_stage + tl.rpp - 1) / tl.rpp;
-    if (op == OP_GATEUP) return gemv_nvsel<true, true>(in, op, layer, tl.nv, rpt);
-    if (norm) return gemv_nvsel<true, false>(in, op, layer, tl.nv, rpt);
-    return gemv_nvsel<false, false>(in, op, layer, tl.nv, rpt);
+    if (op == OP_GATEUP) return gemv_b1<true, true>(in, op, layer);
+    if (op == OP_QKV || op == OP_LMHEAD) return gemv_b1<true, false>(in, op, layer);
+    return gemv_b1<false, false>(in, op, layer);
   }
 
   // ---- MoE routing ---------------------------------------------------------------
@@ -1592,6 +1702,9 @@ struct Consumer {
     constexpr int MT = P / 16 / kConsumerWarps;  // key tiles per warp per stage
     constexpr int KS = HD / 16;                  // k-steps of the score mma
     constexpr int DT = HD / 16;                  // dimension tiles of the P.V mma
+    // the batch-1 kernel unrolls its inner loops less: fewer fragments in
+    // flight keep its registers within the budget of the fp32 GEMV loops
+    constexpr int KU = BATCHED ? KS : 2, DU = BATCHED ? DT : 4;
     constexpr uint32_t CBB = (uint32_t)P * 128u;  // bytes of one 64-column block of a stage
     const int gq = lane >> 2, cq = lane & 3;
     // The batch-1 kernel (fp32 activations elsewhere) takes q and the
@@ -1634,7 +1747,7 @@ struct Consumer {
         const int key0 = (warp * MT + mt) * 16;
         if (key0 < np) {
           float sc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll KU
           for (int ks = 0; ks < KS; ++ks) {
             const uint32_t ch = ((uint32_t)(ks & 3) << 1) | (uint32_t)(lane >> 4);
             uint32_t af[4];
@@ -1666,7 +1779,7 @@ struct Consumer {
           l1 = l1 * c1 + y1;
           m0 = n0;
           m1 = n1;
-#pragma unroll
+#pragma unroll DU
           for (int dt = 0; dt < DT; ++dt) {
             o[dt][0] *= c0;
             o[dt][1] *= c1;
@@ -1691,7 +1804,7 @@ struct Consumer {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
           }
-#pragma unroll
+#pragma unroll DU
           for (int dt = 0; dt < DT; ++dt) {
             const uint32_t ch = ((uint32_t)(dt & 3) << 1) | (uint32_t)((lane >> 3) & 1);
             uint32_t af[4];
@@ -1915,8 +2028,12 @@ struct Consumer {
     }
     consumer_bar();
     if (ctl->last) {
-      // (m, l) of every (head, piece) into shared memory with one parallel
-      // pass, then each output element reads its pieces' o with independent loads
+      // One round trip for the merge: the (m, l) of every (head, piece) go to
+      // shared memory while each thread's output elements load the partial o
+      // of their first kMergeAhead pieces into registers (the rest, for rows of
+      // more pieces, load in the combine loop).
+      constexpr int NOUT = (G * HD + kConsumerThreads - 1) / kConsumerThreads;
+      constexpr int MA = kMergeAhead;
       const int nvalid = a.npieces;
       const size_t pg = ((size_t)a.b * p.nq + q0) * p.n_chunks;
       for (int idx = t; idx < G * nvalid; idx += kConsumerThreads) {
@@ -1925,24 +2042,44 @@ struct Consumer {
         red[2 * idx] = ml.x;
         red[2 * idx + 1] = ml.y;
       }
+      float po_r[NOUT][MA];
+#pragma unroll
+      for (int o = 0; o < NOUT; ++o) {
+        const int idx = t + o * kConsumerThreads;
+        const float* po = p.part_o + (pg + (size_t)(idx / HD) * p.n_chunks) * HD + idx % HD;
+#pragma unroll
+        for (int c = 0; c < MA; ++c) po_r[o][c] = idx < G * HD && c < nvalid ? __ldcg(po + (size_t)c * HD) : 0.f;
+      }
       consumer_bar();
-      for (int idx = t; idx < G * HD; idx += kConsumerThreads) {
-        const int h = idx / HD, d = idx % HD;
-        const float* ml = red + 2 * h * nvalid;
-        float M = -1e30f;
-        for (int c = 0; c < nvalid; ++c) M = fmaxf(M, ml[2 * c]);
-        const float* po = p.part_o + (pg + (size_t)h * p.n_chunks) * HD + d;
-        float den = 0.f, num = 0.f;
+#pragma unroll
+      for (int o = 0; o < NOUT; ++o) {
+        const int idx = t + o * kConsumerThreads;
+        if (idx < G * HD) {
+          const int h = idx / HD, d = idx % HD;
+          const float* ml = red + 2 * h * nvalid;
+          float M = -1e30f;
+          for (int c = 0; c < nvalid; ++c) M = fmaxf(M, ml[2 * c]);
+          float den = 0.f, num = 0.f;
+#pragma unroll
+          for (int c = 0; c < MA; ++c) {
+            if (c < nvalid) {
+              const float w = exp2f(ml[2 * c] - M);
+              den = fmaf(w, ml[2 * c + 1], den);
+              num = fmaf(w, po_r[o][c], num);
+            }
+          }
+          const float* po = p.part_o + (pg + (size_t)h * p.n_chunks) * HD + d;
 #pragma unroll 8
-        for (int c = 0; c < nvalid; ++c) {
-          const float w = exp2f(ml[2 * c] - M);
-          den = fmaf(w, ml[2 * c + 1], den);
-          num = fmaf(w, __ldcg(po + (size_t)c * HD), num);
+          for (int c = MA; c < nvalid; ++c) {
+            const float w = exp2f(ml[2 * c] - M);
+            den = fmaf(w, ml[2 * c + 1], den);
+            num = fmaf(w, __ldcg(po + (size_t)c * HD), num);
+          }
+          if constexpr (BATCHED)
+            p.attn_bf[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = f32_to_bf16_bits(num / den);
+          else
+            p.attn[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = num / den;
         }
-        if constexpr (BATCHED)
-          p.attn_bf[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = f32_to_bf16_bits(num / den);
-        else
-          p.attn[(size_t)a.b * qd + (size_t)(q0 + h) * HD + d] = num / den;
       }
       signal(sig_idx);
     }
@@ -1950,6 +2087,7 @@ struct Consumer {
 
   __device__ __forceinline__ bool attn(const mk_instr& in, int layer, int sig_idx) {
     const int G = attn_heads_per_instr(p.nq / p.nkv);
+    if (t == 0) ctl->xtag = 0u;  // the reduction buffer is about to be overwritten (ordered by the prologue's barrier)
     if (p.hd == 128) {
       switch (G) {
         case 1: return attn_run<128, 1>(in, layer, sig_idx);
@@ -2037,6 +2175,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
     ctl->dead = 0;
     ctl->waiting = 0;
     ctl->last = 0;
+    ctl->xtag = 0u;
     for (int b = 0; b < kMaxBatch; ++b) ctl->amax[b] = 0ull;
     ctl->moe_pub = 0;
     // a sticky error from an earlier step, or out-of-range inputs: do nothing

@@ -161,12 +161,13 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   const size_t o_rope = take(sizeof(float2) * (size_t)d.max_ctx * (hd / 2));
   const size_t n_tmaps = (size_t)mk::kTmapsPerLayer * L + 3;  // KV caches always; weights on the tensor-core kernel
   const size_t o_tmap = n_tmaps ? take(128 * n_tmaps) : 0;
+  const size_t n_tb1 = mk::batched(d) ? 0 : mk::n_tmaps_b1(d);  // the batch-1 kernel's weight maps
+  const size_t o_tb1 = n_tb1 ? take(128 * n_tb1) : 0;
   if (off > kStaticScratchBytes) return MK_ERR_UNSUPPORTED;  // model needs more than the 8 MiB array
-  std::vector<uint8_t> tmaps(128 * n_tmaps);
-  if (n_tmaps) {
-    const cudaError_t te = mk::encode_tmaps(d, *w, *kv, tmaps.data());
-    if (te != cudaSuccess) return te == cudaErrorInvalidValue ? MK_ERR_UNSUPPORTED : MK_ERR_CUDA;
-  }
+  std::vector<uint8_t> tmaps(128 * n_tmaps), tb1(128 * n_tb1);
+  cudaError_t te = n_tmaps ? mk::encode_tmaps(d, *w, *kv, tmaps.data()) : cudaSuccess;
+  if (te == cudaSuccess && n_tb1) te = mk::encode_tmaps_b1(d, *w, tb1.data());
+  if (te != cudaSuccess) return te == cudaErrorInvalidValue ? MK_ERR_UNSUPPORTED : MK_ERR_CUDA;
 
   std::vector<mk::LayerPtrs> lp(L);
   for (int l = 0; l < L; ++l) {
@@ -194,7 +195,8 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
       cudaMemcpyAsync(base + o_lay, lp.data(), sizeof(mk::LayerPtrs) * L, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(base + o_rope, rope.data(), sizeof(float2) * rope.size(), cudaMemcpyHostToDevice, s) !=
           cudaSuccess ||
-      (n_tmaps && cudaMemcpyAsync(base + o_tmap, tmaps.data(), tmaps.size(), cudaMemcpyHostToDevice, s) != cudaSuccess))
+      (n_tmaps && cudaMemcpyAsync(base + o_tmap, tmaps.data(), tmaps.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) ||
+      (n_tb1 && cudaMemcpyAsync(base + o_tb1, tb1.data(), tb1.size(), cudaMemcpyHostToDevice, s) != cudaSuccess))
     return MK_ERR_CUDA;
 
   mk::Params p;
@@ -227,6 +229,7 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   }
   p.rope = (const float2*)(base + o_rope);
   p.tmaps = n_tmaps ? base + o_tmap : nullptr;
+  p.tmaps_b1 = n_tb1 ? base + o_tb1 : nullptr;
   p.xres = (float*)(base + o_xres);
   p.qkv = (float*)(base + o_qkv);
   p.attn = (float*)(base + o_attn);
@@ -256,7 +259,7 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   p.seq_lens = seq_lens;
   p.logits = out_logits;
   p.epoch = 1;  // counters were just cleared
-  p.copy_piece = mk::kDefaultCopyPiece;
+  p.l2_ahead = mk::kDefaultL2Ahead;
   if (mk::launch_step(p, n_sm, s) != cudaSuccess) {
     cudaGetLastError();
     return MK_ERR_CUDA;

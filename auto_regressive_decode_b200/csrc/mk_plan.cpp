@@ -29,13 +29,6 @@ struct mk_plan {
 
 namespace mk {
 
-static bool aligned_ok(int K, int n_mats) {
-  // a row (or a gate+up row pair), possibly cut into column slices, must fit
-  // one ring slot with at most 4 input vectors per thread
-  if (K <= 0 || K % 8) return false;
-  return gemv_ksplit(K, n_mats) > 0;
-}
-
 int validate_desc(const mk_model_desc* d) {
   if (!d) return MK_ERR_INVALID_ARG;
   if (d->n_layers <= 0 || d->hidden <= 0 || d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0 ||
@@ -56,18 +49,18 @@ int validate_desc(const mk_model_desc* d) {
     const int ks[3] = {d->hidden, qd, d->expert_ffn_dim};
     for (int K : ks)
       if (K % 64) return MK_ERR_UNSUPPORTED;
-  } else {
-    if (d->ffn_dim <= 0) return MK_ERR_INVALID_ARG;
-    if (!aligned_ok(d->ffn_dim, 1)) return MK_ERR_UNSUPPORTED;
+  } else if (d->ffn_dim <= 0) {
+    return MK_ERR_INVALID_ARG;
   }
-  if (!aligned_ok(d->hidden, 1) || !aligned_ok(d->hidden, 2) || !aligned_ok(qd, 1)) return MK_ERR_UNSUPPORTED;
-  // GEMVs with an RMSNorm prologue (K = hidden) read whole rows in one pass
-  if (gemv_ksplit(d->hidden, 1) != 1 || gemv_ksplit(d->hidden, 2) != 1) return MK_ERR_UNSUPPORTED;
+  // GEMV widths: rows of whole 16-byte vectors (the TMA maps' row pitch)
+  const int ks[3] = {d->hidden, qd, d->n_experts ? d->expert_ffn_dim : d->ffn_dim};
+  for (int K : ks)
+    if (K % 8) return MK_ERR_UNSUPPORTED;
   if ((int64_t)d->max_ctx * d->head_dim > (1ll << 31)) return MK_ERR_UNSUPPORTED;
   if (d->batch > 1 && !d->n_experts) {
     // tensor-core GEMVs: the weight tensor maps view K as blocks of 64 columns
-    const int ks[3] = {d->hidden, qd, d->ffn_dim};
-    for (int K : ks)
+    const int kb[3] = {d->hidden, qd, d->ffn_dim};
+    for (int K : kb)
       if (K % 64) return MK_ERR_UNSUPPORTED;
   }
   return MK_OK;
@@ -91,31 +84,31 @@ struct Builder {
     return 1;
   }
   // Rows [0, N) of one op split evenly over the SMs, each SM's share cut
-  // into instructions of at most kMaxRows rows (and at the boundaries in
-  // `cuts`, e.g. between wq/wk/wv).  Returns the number of instructions.
-  int rows_op(int op, int layer, int N, const std::vector<int>& cuts, int wait_idx, int wait_count, int sig_idx) {
-    int n = 0;
+  // into equal instructions of at most max_rows rows.  Only the last
+  // instruction of an SM's share signals (its release covers the earlier
+  // ones' outputs), so the counter's per-step target is the number of SMs
+  // holding rows of the op, which this returns.
+  int rows_op(int op, int layer, int N, int wait_idx, int wait_count, int sig_idx) {
+    int n_sig = 0;
     const int n_sm = p->n_sm;
-    const int max_rows = batched(p->d) ? batched_max_rows(op) : kMaxRows;
+    const int max_rows = batched(p->d) ? batched_max_rows(op) : b1_max_rows(op);
     // batch > 1: row ranges start at multiples of kBBoxRows (a TMA box
-    // never reaches into another SM's rows or across wq | wk | wv)
+    // never reaches into another SM's rows); batch 1: any row
     const int unit = batched(p->d) ? kBBoxRows : 1;
     const int64_t NU = (N + unit - 1) / unit;
     for (int s = 0; s < n_sm; ++s) {
-      int r0 = (int)std::min<int64_t>(N, NU * s / n_sm * unit);
-      int r1 = (int)std::min<int64_t>(N, NU * (s + 1) / n_sm * unit);
-      while (r0 < r1) {
-        int e = std::min(r1, r0 + max_rows);
-        int seg = 0, base = 0;
-        for (size_t k = 0; k < cuts.size(); ++k) {
-          if (r0 >= cuts[k]) { seg = (int)k + 1; base = cuts[k]; }
-        }
-        if (seg < (int)cuts.size()) e = std::min(e, cuts[seg]);
-        n += emit(s, op, layer, wait_idx, wait_count, sig_idx, r0 - base, e - base, seg);
-        r0 = e;
+      const int64_t u0 = NU * s / n_sm, u1 = NU * (s + 1) / n_sm;
+      if (u0 >= u1) continue;
+      const int64_t units = u1 - u0, cap = std::max(1, max_rows / unit);
+      const int64_t n_i = (units + cap - 1) / cap;
+      for (int64_t i = 0; i < n_i; ++i) {
+        const int r0 = (int)std::min<int64_t>(N, (u0 + units * i / n_i) * unit);
+        const int r1 = (int)std::min<int64_t>(N, (u0 + units * (i + 1) / n_i) * unit);
+        emit(s, op, layer, wait_idx, wait_count, i + 1 == n_i ? sig_idx : -1, r0, r1);
       }
+      ++n_sig;
     }
-    return n;
+    return n_sig;
   }
 };
 
@@ -159,37 +152,37 @@ int build_plan(const mk_model_desc* d, int n_sm, mk_plan* p) {
     const int cq = counter_index(l, C_QKV), ca = counter_index(l, C_ATTN), co = counter_index(l, C_OPROJ);
     const int cg = counter_index(l, C_GATEUP), cd = counter_index(l, C_DOWN);
     // rows of wq | wk | wv concatenated; an instruction may span matrices
-    int n_qkv = b.rows_op(OP_QKV, l, qd + 2 * kvd, {}, prev_idx, prev_count, cq);
+    int n_qkv = b.rows_op(OP_QKV, l, qd + 2 * kvd, prev_idx, prev_count, cq);
     p->targets[cq] = n_qkv;
     // attention: slot j = SM j; the kernel deals the step's units to the slots
     const int group = d->n_q_heads / d->n_kv_heads, nhg = group / attn_heads_per_instr(group);
     for (int s = 0; s < n_sm; ++s) b.emit(s, OP_ATTN, l, cq, n_qkv, ca, s, n_sm, 0, 0);
     p->targets[ca] = d->batch * d->n_kv_heads * nhg;  // one bump per merged (sequence, KV head, head group)
-    int n_o = b.rows_op(OP_OPROJ, l, H, {}, ca, p->targets[ca], co);
+    int n_o = b.rows_op(OP_OPROJ, l, H, ca, p->targets[ca], co);
     p->targets[co] = n_o;
     if (d->n_experts) {
       // router rows; one expert gate/up slot per SM; down by output rows
       const int cr = counter_index(l, C_ROUTER), ceg = counter_index(l, C_EXP_GATEUP);
       const int ced = counter_index(l, C_EXP_DOWN);
-      int n_r = b.rows_op(OP_ROUTER, l, d->n_experts, {}, co, n_o, cr);
+      int n_r = b.rows_op(OP_ROUTER, l, d->n_experts, co, n_o, cr);
       p->targets[cr] = n_r;
       for (int s = 0; s < n_sm; ++s) b.emit(s, OP_EXP_GATEUP, l, cr, n_r, ceg, s, n_sm, 0, 0);
       p->targets[ceg] = n_sm;
-      int n_ed = b.rows_op(OP_EXP_DOWN, l, H, {}, ceg, n_sm, ced);
+      int n_ed = b.rows_op(OP_EXP_DOWN, l, H, ceg, n_sm, ced);
       p->targets[ced] = n_ed;
       prev_idx = ced;
       prev_count = n_ed;
       continue;
     }
-    int n_gu = b.rows_op(OP_GATEUP, l, d->ffn_dim, {}, co, n_o, cg);
+    int n_gu = b.rows_op(OP_GATEUP, l, d->ffn_dim, co, n_o, cg);
     p->targets[cg] = n_gu;
-    int n_dn = b.rows_op(OP_DOWN, l, H, {}, cg, n_gu, cd);
+    int n_dn = b.rows_op(OP_DOWN, l, H, cg, n_gu, cd);
     p->targets[cd] = n_dn;
     prev_idx = cd;
     prev_count = n_dn;
   }
   const int c_lm = counter_lmhead(L);
-  p->targets[c_lm] = b.rows_op(OP_LMHEAD, L, d->vocab, {}, prev_idx, prev_count, c_lm);
+  p->targets[c_lm] = b.rows_op(OP_LMHEAD, L, d->vocab, prev_idx, prev_count, c_lm);
   // Host-made fault for tests of the failure path (never set in normal use):
   // MK_FAULT_INJECT=wait makes SM 0's first instruction wait on a counter no
   // instruction ever raises far enough, so every bounded wait must run out.

@@ -68,15 +68,17 @@ def layer_breakdown(plan, trace, layer):
 
 
 def handoff_costs(plan, trace):
-    """Per op: median time (us) from an instruction's done stamp to the start of
-    the next instruction on the same SM -- its signal (barrier and release) and
-    the fetch of the next instruction."""
+    """Per op: median time (us) from a signalling instruction's done stamp (the
+    last of its op on an SM) to the start of the next instruction on the same
+    SM -- its signal (barrier and release) and the fetch of the next instruction."""
     t = trace.astype(np.int64)
     ops = plan.instrs[:, 0] & 0xFF
+    sig = plan.instrs[:, 3] >= 0
     off = np.asarray(plan.offsets)
     same = np.zeros(len(t), dtype=bool)
     for s in range(len(off) - 1):
         same[off[s]:off[s + 1] - 1] = True
+    same &= sig
     gap = np.full(len(t), np.nan)
     gap[:-1] = (t[1:, 0] - t[:-1, 2]) / 1e3
     return {OP_NAMES.get(op, str(op)): float(np.median(gap[same & (ops == op)]))

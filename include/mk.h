@@ -100,10 +100,8 @@ typedef struct mk_handle mk_handle;
  * Returns MK_ERR_UNSUPPORTED for shapes the kernel cannot run:
  *   - head_dim not 64 or 128; n_q_heads not 1, 2, 4 or 8 times n_kv_heads;
  *   - batch > 8;
- *   - hidden above 8192 (a gate/up row pair of the norm-fused GEMVs must fit
- *     one 32 KB pipeline stage); a GEMV width (hidden, n_q_heads*head_dim,
- *     ffn_dim) not a multiple of 8, or too wide to cut into at most four
- *     slices of one stage each (e.g. ffn_dim above 65536);
+ *   - a GEMV width (hidden, n_q_heads*head_dim, ffn_dim or expert_ffn_dim)
+ *     not a multiple of 8;
  *   - batch > 1 or MoE (the tensor-core kernel) with hidden, n_q_heads*head_dim,
  *     ffn_dim or expert_ffn_dim not a multiple of 64;
  *   - MoE with more than 256 experts, top_k > 8, or batch * top_k > 64;
