@@ -290,8 +290,6 @@ extern "C" int mk_create(const mk_model_desc* desc, const mk_weights* w, const m
   h->loop_len = (int32_t*)(base + o_llen);
   h->amax = (unsigned long long*)(base + o_amax);
   h->loop_logits = (float*)(base + o_llog);
-  const char* ahead_env = getenv("MK_L2_AHEAD_KB");  // tuning knob: the batch-1 kernel's L2 runway (0: off)
-  p.l2_ahead = ahead_env ? (uint32_t)atoi(ahead_env) * 1024u : mk::kDefaultL2Ahead;
   *out = h;
   return MK_OK;
 }

@@ -70,7 +70,6 @@ struct Params {
   uint32_t epoch;
   uint64_t timeout_ns;
   uint64_t* trace;          // [n_instr][kTraceStamps] timestamps, or nullptr
-  uint32_t l2_ahead;        // batch-1 kernel: weight bytes kept prefetched into L2 beyond the ring's instruction
 };
 
 // Encode the 3-D tensor maps of the batch > 1 kernel (one per weight matrix,

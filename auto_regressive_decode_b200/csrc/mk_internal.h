@@ -48,7 +48,6 @@ constexpr int kMaxBatch = 8;
 constexpr int kMaxGroup = 8;                           // query heads per KV head
 constexpr int kMaxHeadDim = 128;
 constexpr int kTraceStamps = 8;                        // per-instruction trace words
-constexpr uint32_t kDefaultL2Ahead = 512 * 1024;  // batch-1 kernel: weight bytes prefetched into L2 ahead
 
 // ---- dependency counters -----------------------------------------------------
 // Each counter is bumped once per producing instruction per step; a waiter
@@ -145,7 +144,7 @@ MK_HD int attn_heads_per_instr(int group) { return group > 4 ? 4 : group; }
 
 // The merging piece of an attention row loads the partial outputs of its
 // first kMergeAhead pieces together with their (m, l) pairs.
-constexpr int kMergeAhead = 8;
+constexpr int kMergeAhead = 24;
 
 // Positions of K (or V) that fit one ring slot.
 MK_HD int attn_stage_positions(int head_dim) { return kStageBytes / (head_dim * 2); }

@@ -43,6 +43,7 @@ struct Ctl {
   int waiting;    // the consumers are blocked on a dependency counter
   int last;       // attention: this CTA merges (broadcast)
   int flag;       // generic broadcast
+  int32_t slen[kMaxBatch], spos[kMaxBatch];  // this step's seq_lens and positions (read once per step)
   uint32_t xtag;  // batch-1 GEMV: which input piece the reduction buffer holds (0: none)
   float xss;      // and, for a norm-fused op, the sum of squares of its input
   float b1red[kB1MaxLines * 4];  // batch-1 GEMV: per-warp sums of lines split over chunks
@@ -55,7 +56,7 @@ struct Ctl {
   } b1box[kB1MaxLines];
   int b1nbox;
   float sred[kConsumerWarps * 2];
-  float qs[kMaxGroup * kMaxHeadDim];
+  alignas(16) float qs[kMaxGroup * kMaxHeadDim];
   float aml[kConsumerWarps * kMaxGroup * 2];  // attention: per-warp (m, l) of every head
   alignas(16) uint16_t knew[kMaxHeadDim];     // the new token's K/V rows (bf16, as appended)
   alignas(16) uint16_t vnew[kMaxHeadDim];
@@ -138,11 +139,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Bring a global range into L2 (no destination, no completion to wait for).
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // One box of a 3-D tensor map (coordinates c0, c1, c2) into shared memory,
@@ -431,18 +427,16 @@ struct Gemv {
   // btile_rows() output rows
   int bnch, bnt;
   // batch 1 (row-stationary tiles): lines of the instruction, chunks of
-  // kB1Chunk columns, chunks per stage, stages; per segment its 8-row box map
-  // (the 1-row box map follows it), first row within its matrix, rows, first
-  // line within a stage and first weight of its first row (L2 prefetch)
+  // kB1Chunk columns, chunks per stage, stages; per segment its first box map
+  // (the others follow it), first row within its matrix, rows and first line
+  // within a stage
   int lines, nch, ncs, nst, nseg;
   const uint8_t *bm0, *bm1, *bm2;
-  const uint16_t *bw0, *bw1, *bw2;
   int brow0, brow1, brow2, bn0, bn1, bn2, bl0, bl1, bl2;
   __device__ __forceinline__ int seg_rows(int s) const { return s == 0 ? bn0 : (s == 1 ? bn1 : bn2); }
   __device__ __forceinline__ int seg_row(int s) const { return s == 0 ? brow0 : (s == 1 ? brow1 : brow2); }
   __device__ __forceinline__ int seg_line(int s) const { return s == 0 ? bl0 : (s == 1 ? bl1 : bl2); }
   __device__ __forceinline__ const uint8_t* seg_map(int s) const { return s == 0 ? bm0 : (s == 1 ? bm1 : bm2); }
-  __device__ __forceinline__ const uint16_t* seg_w(int s) const { return s == 0 ? bw0 : (s == 1 ? bw1 : bw2); }
 };
 
 // Batch-1 box maps of matrix `mat` (0..6: wq wk wv wo w_gate w_up w_down) of
@@ -465,15 +459,12 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
   g.bl0 = 0;
   g.bl1 = g.bl2 = 0;
   g.bm0 = g.bm1 = g.bm2 = nullptr;
-  g.bw0 = g.bw1 = g.bw2 = nullptr;
   if (op == OP_LMHEAD) {
     g.K = p.H;
     if (!p.tc) {
       g.bm0 = p.tmaps_b1 + (size_t)p.L * kB1MapsPerLayer * 128;
-      g.bw0 = p.lm_head + (size_t)g.r0 * g.K;
     }
   } else {
-    const LayerPtrs& lp = p.layers[layer];
     switch (op) {
       case OP_QKV: {
         g.K = p.H;
@@ -484,14 +475,12 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
           for (int m = 0; m < 3; ++m) {
             const int base = m == 0 ? 0 : (m == 1 ? qd : qd + kvd);
             const int end = m == 0 ? qd : (m == 1 ? qd + kvd : qd + 2 * kvd);
-            const uint16_t* mat = m == 0 ? lp.wq : (m == 1 ? lp.wk : lp.wv);
             const int a = max(g.r0, base), b = min(g.r1, end);
             if (a < b) {
               const uint8_t* map = b1_map(p, layer, m);
-              const uint16_t* w = mat + (size_t)(a - base) * g.K;
-              if (g.nseg == 0) { g.bm0 = map; g.bw0 = w; g.brow0 = a - base; g.bn0 = b - a; g.bl0 = a - g.r0; }
-              else if (g.nseg == 1) { g.bm1 = map; g.bw1 = w; g.brow1 = a - base; g.bn1 = b - a; g.bl1 = a - g.r0; }
-              else { g.bm2 = map; g.bw2 = w; g.brow2 = a - base; g.bn2 = b - a; g.bl2 = a - g.r0; }
+              if (g.nseg == 0) { g.bm0 = map; g.brow0 = a - base; g.bn0 = b - a; g.bl0 = a - g.r0; }
+              else if (g.nseg == 1) { g.bm1 = map; g.brow1 = a - base; g.bn1 = b - a; g.bl1 = a - g.r0; }
+              else { g.bm2 = map; g.brow2 = a - base; g.bn2 = b - a; g.bl2 = a - g.r0; }
               ++g.nseg;
             }
           }
@@ -500,7 +489,7 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
       }
       case OP_OPROJ:
         g.K = p.nq * p.hd;
-        if (!p.tc) { g.bm0 = b1_map(p, layer, 3); g.bw0 = lp.wo + (size_t)g.r0 * g.K; }
+        if (!p.tc) g.bm0 = b1_map(p, layer, 3);
         break;
       case OP_GATEUP:
         g.K = p.H;
@@ -508,8 +497,6 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
           g.nseg = 2;
           g.bm0 = b1_map(p, layer, 4);
           g.bm1 = b1_map(p, layer, 5);
-          g.bw0 = lp.w_gate + (size_t)g.r0 * g.K;
-          g.bw1 = lp.w_up + (size_t)g.r0 * g.K;
           g.brow1 = g.r0;
           g.bn1 = R;
           g.bl1 = R;
@@ -523,7 +510,7 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
         break;
       default:  // OP_DOWN
         g.K = p.I;
-        if (!p.tc) { g.bm0 = b1_map(p, layer, 6); g.bw0 = lp.w_down + (size_t)g.r0 * g.K; }
+        if (!p.tc) g.bm0 = b1_map(p, layer, 6);
         break;
     }
   }
@@ -584,13 +571,13 @@ __device__ __forceinline__ int64_t kv_row(const Params& p, int layer, int b, int
   return (((int64_t)layer * p.B + b) * p.nkv + kvh) * p.T + pos;
 }
 
-__device__ __forceinline__ Attn attn_geo(const Params& p, const AttnPiece& pc, int layer, int head_dim) {
+__device__ __forceinline__ Attn attn_geo(const Params& p, const Ctl* ctl, const AttnPiece& pc, int layer, int head_dim) {
   Attn a;
   const int group = p.nq / p.nkv, nhg = group / attn_heads_per_instr(group);
   a.b = pc.b;
   a.kvh = pc.row / nhg;
   a.hg = pc.row % nhg;
-  a.S = p.seq_lens[a.b];
+  a.S = ctl->slen[a.b];
   a.p0 = pc.ua * p.chunk;
   const int p1 = pc.ub * p.chunk;
   a.active = true;
@@ -603,9 +590,9 @@ __device__ __forceinline__ Attn attn_geo(const Params& p, const AttnPiece& pc, i
   return a;
 }
 
-__device__ __forceinline__ void attn_sched(const Params& p, const mk_instr& in, AttnSched& sc) {
+__device__ __forceinline__ void attn_sched(const Params& p, const Ctl* ctl, const mk_instr& in, AttnSched& sc) {
   const int group = p.nq / p.nkv;
-  attn_sched_init(sc, p.seq_lens, p.B, p.nkv * (group / attn_heads_per_instr(group)), p.chunk, in.b);
+  attn_sched_init(sc, ctl->slen, p.B, p.nkv * (group / attn_heads_per_instr(group)), p.chunk, in.b);
 }
 
 // ---------------------------------------------------------------------------
@@ -642,7 +629,7 @@ struct Cursor {
       op = op_of(in.op_layer);
       layer = layer_of(in.op_layer);
       if (op == OP_ATTN) {
-        attn_sched(*pp, in, *sc);
+        attn_sched(*pp, ctl, in, *sc);
         aslot = in.a;
         ag = attn_slot_begin(*sc, aslot);
         ag1 = attn_slot_begin(*sc, aslot + 1);
@@ -685,7 +672,7 @@ struct Cursor {
   __device__ __forceinline__ bool next_piece() {
     while (ag < ag1) {
       const AttnPiece pc = attn_piece_at(*sc, ag, aslot);
-      a = attn_geo(*pp, pc, layer, pp->hd);
+      a = attn_geo(*pp, ctl, pc, layer, pp->hd);
       pieceu = pc.ub - pc.ua;
       if (a.nsub > 0) return true;
       ag += pieceu;
@@ -871,62 +858,13 @@ struct Producer {
   }
 };
 
-// The cached K and V bytes an attention slot instruction streams this step
-// (its pieces' positions before the new token), optionally prefetched into L2
-// one ring stage at a time.
-__device__ __noinline__ uint64_t attn_kv_bytes(const Params& p, const mk_instr& in, int layer, bool prefetch) {
-  AttnSched sc;
-  attn_sched(p, in, sc);
-  const int j = in.a;
-  uint64_t total = 0;
-  for (int64_t gg = attn_slot_begin(sc, j), g1 = attn_slot_begin(sc, j + 1); gg < g1;) {
-    const AttnPiece pc = attn_piece_at(sc, gg, j);
-    gg += pc.ub - pc.ua;
-    const Attn a = attn_geo(p, pc, layer, p.hd);
-    for (int sub = 0; sub < a.nsub; ++sub) {
-      const uint32_t bytes = (uint32_t)min(a.P, a.n_cached - sub * a.P) * (uint32_t)p.hd * 2u;
-      if (prefetch) {
-        const int64_t row = kv_row(p, layer, a.b, a.kvh, a.p0 + sub * a.P);
-        prefetch_l2(p.kc + row * p.hd, bytes);
-        prefetch_l2(p.vc + row * p.hd, bytes);
-      }
-      total += 2u * bytes;
-    }
-  }
-  return total;
-}
-
-// Batch-1 GEMV instruction: its weight bytes (every segment's row block),
-// optionally prefetched into L2 (each segment's rows are one contiguous block).
-__device__ __noinline__ uint64_t b1_weight_bytes(const Params& p, const mk_instr& in, bool prefetch) {
-  const int op = op_of(in.op_layer);
-  const Gemv g = gemv_geo(p, in, op, layer_of(in.op_layer));
-  if (prefetch)
-    for (int s2 = 0; s2 < g.nseg; ++s2) {
-      const uint32_t bytes = (uint32_t)g.seg_rows(s2) * (uint32_t)g.K * 2u;
-      if (bytes) prefetch_l2(g.seg_w(s2), bytes);
-    }
-  return (uint64_t)g.lines * g.K * 2u;
-}
-
 // One thread (lane 0 of the producer warp) issues every copy.
-//
-// Batch-1 kernel: besides the ring, the producer keeps an L2 runway: the
-// weight blocks of the instructions after the current one are prefetched into
-// L2, up to p.l2_ahead bytes ahead of the instruction the ring is filling, so
-// that HBM keeps streaming while the consumers wait on a dependency and the
-// ring is full; an attention slot's runway is the cached K/V positions of its
-// pieces.
 template <bool BATCHED>
 __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* list, int n, Ctl* ctl, uint8_t* ring) {
   Producer<BATCHED> pr(p, ctl, ring);
   uint64_t* trace = p.trace ? p.trace + (size_t)p.offsets[blockIdx.x] * kTraceStamps : nullptr;
   Cursor cur(p, list, n, &ctl->psched, ctl);
   cur.seek(0);
-  // runway (batch 1): instructions [.., pf_i) prefetched; cum_pf / cum_cur =
-  // their bytes / the bytes of the instructions up to the current one
-  int pf_i = 0, entered = -1;
-  uint64_t cum_pf = 0, cum_cur = 0;
   bool ok = true;
   int last = -1;
   while (cur.i < n) {
@@ -943,24 +881,6 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
       last = cur.i;
     }
     if (!BATCHED) {
-      if (p.l2_ahead && cur.i != entered) {
-        entered = cur.i;
-        cum_cur += cur.op == OP_ATTN ? attn_kv_bytes(p, list[cur.i], cur.layer, false)
-                                     : b1_weight_bytes(p, list[cur.i], false);
-        if (pf_i <= cur.i) {  // the runway restarts after the current instruction
-          pf_i = cur.i + 1;
-          cum_pf = cum_cur;
-        }
-        while (pf_i < n && cum_pf < cum_cur + p.l2_ahead) {
-          const mk_instr in = list[pf_i];
-          const int op = op_of(in.op_layer);
-          if (op == OP_ATTN)
-            cum_pf += attn_kv_bytes(p, in, layer_of(in.op_layer), true);
-          else if (op >= OP_QKV && op <= OP_LMHEAD)
-            cum_pf += b1_weight_bytes(p, in, true);
-          ++pf_i;
-        }
-      }
       if (cur.op != OP_ATTN) {
         // a batch-1 GEMV instruction: its box list once, then every stage from it
         Ctl::B1Box* box = ctl->b1box;
@@ -1058,8 +978,15 @@ struct Consumer {
     ++k;
   }
 
-  // Dependency wait on `idx` reaching epoch * count.  Uniform result.
+  // Dependency wait on `idx` reaching epoch * count.  Uniform result.  An
+  // instruction that waits on what the previous wait already saw (the later
+  // instructions of an op on this SM) skips the acquire round trip: the data
+  // it reads was ordered by that acquire.
+  int sat_idx = -1, sat_count = 0;
   __device__ __forceinline__ bool wait_counter(int idx, int count) {
+    if (idx >= 0 && idx == sat_idx && count == sat_count) return !consumer_bar_or(*(volatile int*)&ctl->dead != 0);
+    sat_idx = idx;
+    sat_count = count;
     bool fail = false;
     if (idx >= 0 && t == 0) {
       const uint32_t target = p.epoch * (uint32_t)count;
@@ -1686,6 +1613,256 @@ struct Consumer {
   }
 
   // ---- attention ---------------------------------------------------------------
+  // Batch 1: the cached positions of one piece on the CUDA cores, in fp32.  A
+  // stage holds P positions of K (or V) as [64-column block][position][64]
+  // with the 128-byte swizzle (16-byte chunk c of position row r at chunk
+  // position c ^ (r & 7)).  Warp w takes positions [w P/8, (w + 1) P/8) of
+  // every stage with its own online softmax (log2 units; q pre-scaled by
+  // log2(e)/sqrt(hd)).  Lane l covers the 8 dimensions (l % DS) * 8 .. + 8
+  // (DS = HD / 8) of the positions of its group l / DS: scores take the dot
+  // products of those slices, reduced over the DS lanes by halving shuffles;
+  // P.V accumulates o[head][its 8 dims] over its group's positions in packed
+  // fp32 pairs.  At the end the position groups of a warp, then the warps,
+  // merge into the piece's partial, the same partial the tensor-core path
+  // writes.
+  template <int HD, int G>
+  __device__ __forceinline__ void attn_ff(const Attn& a, int q0) {
+    constexpr int P = kStageBytes / (HD * 2);  // positions per stage
+    constexpr int DS = HD / 8;                 // lanes per position (8 dimensions each)
+    constexpr int PG = 32 / DS;                // position groups per warp
+    constexpr int PW = P / kConsumerWarps;     // positions per warp per stage
+    constexpr int NPL = PW / PG;               // positions per lane per stage (8)
+    constexpr int NB = 4;                      // positions per score batch
+    constexpr int VB = G * NB;                 // score values per batch (<= 16)
+    constexpr int RR = VB < DS ? VB : DS;      // values per reduction round
+    constexpr uint32_t CBB = (uint32_t)P * 128u;
+    constexpr int NJ = (G * PW + 31) / 32;     // softmax entries per lane
+    static_assert(NPL % NB == 0 && VB % RR == 0, "attention tiling");
+    const int ds = lane % DS, pg = lane / DS;
+    const uint32_t blk = (uint32_t)(ds >> 3) * CBB, chunk = (uint32_t)(ds & 7);
+    // q slices of the G heads (fp32 pairs)
+    unsigned long long qp[G][4];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float4 q0v = *reinterpret_cast<const float4*>(ctl->qs + h * HD + ds * 8);
+      const float4 q1v = *reinterpret_cast<const float4*>(ctl->qs + h * HD + ds * 8 + 4);
+      qp[h][0] = pack2(q0v.x, q0v.y);
+      qp[h][1] = pack2(q0v.z, q0v.w);
+      qp[h][2] = pack2(q1v.x, q1v.y);
+      qp[h][3] = pack2(q1v.z, q1v.w);
+    }
+    unsigned long long o[G][4];
+#pragma unroll
+    for (int h = 0; h < G; ++h) o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0ull;
+    float m[G], l[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) m[h] = -1e30f, l[h] = 0.f;
+    // this warp's scores / probabilities of a stage, [position][4 heads]
+    float* S = red + kRedFloats + warp * (PW * 4);
+    for (int s = 0; s < a.nsub; ++s) {
+      const int np = min(P, a.n_cached - s * P);
+      const uint32_t Ks = smem_addr(wait_stage(k));
+      const uint32_t Vs = smem_addr(wait_stage(k + 1));
+      if (tr && s == 0) tr[5] = globaltimer();
+      // -- scores of the lane's positions, NB at a time, reduced over the DS lanes
+#pragma unroll
+      for (int i0 = 0; i0 < NPL; i0 += NB) {
+        float part[VB];
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          const int pos = warp * PW + pg + PG * (i0 + i);
+          const uint4 kv = lds_u4_if(Ks + blk + (uint32_t)pos * 128u + ((chunk ^ (uint32_t)(pos & 7)) << 4), pos < np);
+          const unsigned long long kp[4] = {pack2(bf16_lo(kv.x), bf16_hi(kv.x)), pack2(bf16_lo(kv.y), bf16_hi(kv.y)),
+                                            pack2(bf16_lo(kv.z), bf16_hi(kv.z)), pack2(bf16_lo(kv.w), bf16_hi(kv.w))};
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            unsigned long long d = ffma2(kp[0], qp[h][0], 0ull);
+            d = ffma2(kp[1], qp[h][1], d);
+            d = ffma2(kp[2], qp[h][2], d);
+            d = ffma2(kp[3], qp[h][3], d);
+            part[h * NB + i] = sum2(d);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < VB / RR; ++r) {
+          float v[RR];
+#pragma unroll
+          for (int e = 0; e < RR; ++e) v[e] = part[r * RR + e];
+          const float tot = group_reduce_multi<RR, DS>(v, lane);  // value index (ds) >> log2(DS / RR)
+          const int vi = r * RR + (ds >> (ilog2c(DS) - ilog2c(RR)));
+          if ((ds & (DS / RR - 1)) == 0) {
+            const int h = vi / NB, i = vi % NB;
+            const int pl = pg + PG * (i0 + i);  // the position within the warp's share
+            S[pl * 4 + h] = warp * PW + pl < np ? tot : -1e30f;
+          }
+        }
+      }
+      __syncwarp();
+      // -- online softmax per head over the warp's PW positions: lane j handles
+      // entries j, j + 32, ... of [head][position]
+      float mt[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) mt[h] = -1e30f;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int idx = lane + 32 * j, h = min(idx / PW, G - 1), pl = idx % PW;
+        float x = idx < G * PW ? S[pl * 4 + h] : -1e30f;
+#pragma unroll
+        for (int off = PW / 2; off; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+          if (hh == h) mt[hh] = x;
+      }
+      // each head's maximum lives in the lanes of its entries: broadcast
+      float c[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float mx = __shfl_sync(0xffffffffu, mt[h], (h * PW) % 32);
+        const float mn = fmaxf(m[h], mx);
+        c[h] = exp2f(m[h] - mn);
+        m[h] = mn;
+      }
+      float lt[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) lt[h] = 0.f;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int idx = lane + 32 * j, h = min(idx / PW, G - 1), pl = idx % PW;
+        float mh = m[0];
+#pragma unroll
+        for (int hh = 1; hh < G; ++hh)
+          if (hh == h) mh = m[hh];
+        const bool act = idx < G * PW;
+        const float sc = act ? S[pl * 4 + h] : -1e30f;
+        const float pv = act && warp * PW + pl < np ? exp2f(sc - mh) : 0.f;
+        if (act) S[pl * 4 + h] = pv;
+        float y = pv;
+#pragma unroll
+        for (int off = PW / 2; off; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+          if (hh == h) lt[hh] = y;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) l[h] = l[h] * c[h] + __shfl_sync(0xffffffffu, lt[h], (h * PW) % 32);
+      __syncwarp();
+      // -- o = o * c + P . V over the lane's positions
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const unsigned long long cc = pack2(c[h], c[h]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[h][e] = ffma2(o[h][e], cc, 0ull);
+      }
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int pl = pg + PG * i, pos = warp * PW + pl;
+        const uint4 vv = lds_u4_if(Vs + blk + (uint32_t)pos * 128u + ((chunk ^ (uint32_t)(pos & 7)) << 4), pos < np);
+        const float4 pr = *reinterpret_cast<const float4*>(S + pl * 4);
+        const unsigned long long vp[4] = {pack2(bf16_lo(vv.x), bf16_hi(vv.x)), pack2(bf16_lo(vv.y), bf16_hi(vv.y)),
+                                          pack2(bf16_lo(vv.z), bf16_hi(vv.z)), pack2(bf16_lo(vv.w), bf16_hi(vv.w))};
+        const float ph[4] = {pr.x, pr.y, pr.z, pr.w};
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const unsigned long long pp = pack2(ph[h], ph[h]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[h][e] = ffma2(vp[e], pp, o[h][e]);
+        }
+      }
+      __syncwarp();
+      release();  // K slot
+      release();  // V slot
+    }
+    if (tr) tr[6] = globaltimer();
+    // -- the position groups of each warp: one o per warp (m, l are warp-uniform)
+#pragma unroll
+    for (int off = DS; off < 32; off <<= 1)
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x, y;
+          asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(o[h][e]));
+          x += __shfl_xor_sync(0xffffffffu, x, off);
+          y += __shfl_xor_sync(0xffffffffu, y, off);
+          o[h][e] = pack2(x, y);
+        }
+    if (a.owns_new && warp == 0) {
+      // the new token: its score for every head (the DS lanes of group 0 hold
+      // its dimension slices), folded into warp 0's state
+      const uint4 kv = *reinterpret_cast<const uint4*>(ctl->knew + ds * 8);
+      const unsigned long long kp[4] = {pack2(bf16_lo(kv.x), bf16_hi(kv.x)), pack2(bf16_lo(kv.y), bf16_hi(kv.y)),
+                                        pack2(bf16_lo(kv.z), bf16_hi(kv.z)), pack2(bf16_lo(kv.w), bf16_hi(kv.w))};
+      const uint4 vv = *reinterpret_cast<const uint4*>(ctl->vnew + ds * 8);
+      const unsigned long long vp[4] = {pack2(bf16_lo(vv.x), bf16_hi(vv.x)), pack2(bf16_lo(vv.y), bf16_hi(vv.y)),
+                                        pack2(bf16_lo(vv.z), bf16_hi(vv.z)), pack2(bf16_lo(vv.w), bf16_hi(vv.w))};
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        unsigned long long d = ffma2(kp[0], qp[h][0], 0ull);
+        d = ffma2(kp[1], qp[h][1], d);
+        d = ffma2(kp[2], qp[h][2], d);
+        d = ffma2(kp[3], qp[h][3], d);
+        float sn = sum2(d);
+#pragma unroll
+        for (int off = DS / 2; off; off >>= 1) sn += __shfl_xor_sync(0xffffffffu, sn, off);
+        const float mn = fmaxf(m[h], sn);
+        const float cc = exp2f(m[h] - mn), en = exp2f(sn - mn);
+        m[h] = mn;
+        l[h] = l[h] * cc + en;
+        const unsigned long long c2 = pack2(cc, cc), e2 = pack2(en, en);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[h][e] = ffma2(vp[e], e2, ffma2(o[h][e], c2, 0ull));
+      }
+    }
+    // -- merge the warps through shared memory (one round: G heads fit)
+    constexpr int HR = kRedFloats / (kConsumerWarps * HD) < G ? kRedFloats / (kConsumerWarps * HD) : G;
+    static_assert(HR == G, "one merge round");
+    const size_t pbase = ((size_t)a.b * p.nq + q0) * p.n_chunks + a.c;
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        ctl->aml[(warp * kMaxGroup + h) * 2] = m[h];
+        ctl->aml[(warp * kMaxGroup + h) * 2 + 1] = l[h];
+      }
+    }
+    if (pg == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float4 a0, a1;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(a0.x), "=f"(a0.y) : "l"(o[h][0]));
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(a0.z), "=f"(a0.w) : "l"(o[h][1]));
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(a1.x), "=f"(a1.y) : "l"(o[h][2]));
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(a1.z), "=f"(a1.w) : "l"(o[h][3]));
+        *reinterpret_cast<float4*>(red + (warp * HR + h) * HD + ds * 8) = a0;
+        *reinterpret_cast<float4*>(red + (warp * HR + h) * HD + ds * 8 + 4) = a1;
+      }
+    }
+    consumer_bar();
+    for (int id = t; id < G * HD; id += kConsumerThreads) {
+      const int h = id / HD, d = id % HD;
+      float M = -1e30f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ctl->aml[(w * kMaxGroup + h) * 2]);
+      float den = 0.f, num = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float cw = exp2f(ctl->aml[(w * kMaxGroup + h) * 2] - M);
+        den = fmaf(cw, ctl->aml[(w * kMaxGroup + h) * 2 + 1], den);
+        num = fmaf(cw, red[(w * HR + h) * HD + d], num);
+      }
+      if (a.npieces == 1) {  // the whole row: the output itself
+        p.attn[(size_t)a.b * p.nq * HD + (size_t)(q0 + h) * HD + d] = num / den;
+      } else {
+        const size_t pi = pbase + (size_t)h * p.n_chunks;
+        p.part_o[pi * HD + d] = num;
+        if (d == 0) {
+          p.part_ml[pi * 2] = M;
+          p.part_ml[pi * 2 + 1] = den;
+        }
+      }
+    }
+    consumer_bar();
+  }
+
   // Batch > 1: the cached positions of one chunk on tensor cores.  A stage is
   // a TMA box of P positions, [64-column block][position][64] with the 128-byte
   // swizzle.  Warp w owns key tiles of 16 positions of every stage:
@@ -1906,14 +2083,14 @@ struct Consumer {
     // and positions, not on its activations: fetch the first piece's before
     // the dependency wait.
     AttnSched sc;
-    attn_sched(p, in, sc);
+    attn_sched(p, ctl, in, sc);
     const int j = in.a;
     const int64_t g0 = attn_slot_begin(sc, j), g1 = attn_slot_begin(sc, j + 1);
     int rb = -1;  // sequence whose RoPE factors csr holds
     float2 csr[NP];
     if (g0 < g1) {
       rb = attn_piece_at(sc, g0, j).b;
-      const float2* cs = p.rope + (size_t)p.positions[rb] * (HD / 2);
+      const float2* cs = p.rope + (size_t)ctl->spos[rb] * (HD / 2);
 #pragma unroll
       for (int q = 0; q < NP; ++q) csr[q] = __ldg(cs + lane + 32 * q);
     }
@@ -1924,11 +2101,11 @@ struct Consumer {
       g += pc.ub - pc.ua;
       if (pc.b != rb) {
         rb = pc.b;
-        const float2* cs = p.rope + (size_t)p.positions[rb] * (HD / 2);
+        const float2* cs = p.rope + (size_t)ctl->spos[rb] * (HD / 2);
 #pragma unroll
         for (int q = 0; q < NP; ++q) csr[q] = __ldg(cs + lane + 32 * q);
       }
-      attn_piece<HD, G>(attn_geo(p, pc, layer, HD), layer, sig_idx, csr);
+      attn_piece<HD, G>(attn_geo(p, ctl, pc, layer, HD), layer, sig_idx, csr);
     }
     return true;
   }
@@ -2008,7 +2185,10 @@ struct Consumer {
       }
       consumer_bar();
       if (tr) tr[4] = globaltimer();
-      attn_tc<HD, G>(a, q0);
+      if constexpr (BATCHED)
+        attn_tc<HD, G>(a, q0);
+      else
+        attn_ff<HD, G>(a, q0);
     }
     if (a.npieces == 1) {  // written above: no partials to merge
       signal(sig_idx);
@@ -2182,6 +2362,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_persistent(const __grid_consta
     int bad = ld_relaxed_i32(p.status) != 0;
     for (int b = 0; b < p.B && !bad; ++b) {
       const int S = p.seq_lens[b], pos = p.positions[b], tok = p.tokens[b];
+      ctl->slen[b] = S;
+      ctl->spos[b] = pos;
       if (S < 0 || S >= p.T || pos < 0 || pos >= p.T || tok < 0 || tok >= p.V) {
         set_status(p, MK_ERR_RANGE, b);
         bad = 1;

@@ -259,7 +259,6 @@ extern "C" int mk_decode_step_noalloc(const mk_model_desc* desc, const mk_weight
   p.seq_lens = seq_lens;
   p.logits = out_logits;
   p.epoch = 1;  // counters were just cleared
-  p.l2_ahead = mk::kDefaultL2Ahead;
   if (mk::launch_step(p, n_sm, s) != cudaSuccess) {
     cudaGetLastError();
     return MK_ERR_CUDA;
