@@ -40,7 +40,11 @@ sys.path.insert(0, ROOT)
 
 import fixtures as fx  # noqa: E402
 
+METRIC = "decode tokens/s (batch tokens per decode step / step time)"
 SPEC_HBM_GBS = 8000.0
+# the default line's workload, then the other configurations it reports under "per_config"
+MAIN_CONFIG = "dense-8b"
+PER_CONFIG = ("dense-0.6b", "dense-13b-b8", "moe-128x8")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -221,8 +225,9 @@ def job_tokens_per_s(world, batch, steps, total_ms):
 
 
 def run_reference(args, cfg, rank):
-    """The oracle timed on the host: each step is one layer of the decode step (a bounded sample);
-    the step time is the median layer time x L plus the LM head, timed once."""
+    """The oracle timed on the host.  Each timed step is a bounded sample: one of the L layers of the
+    decode step (layers taken in turn).  `ms_per_step` and `steps` report those samples as timed; the
+    throughput extrapolates the median layer to the whole step (L layers plus the LM head, timed once)."""
     if rank != 0:
         return
     import oracle as ora
@@ -247,66 +252,82 @@ def run_reference(args, cfg, rank):
     for b in range(cfg.batch):
         model.lm_head(x[b])
     t_head = time.perf_counter() - t0
-    step_s = statistics.median(times) * cfg.n_layers + t_head
+    layer_s = statistics.median(times)
+    step_s = layer_s * cfg.n_layers + t_head
     value = cfg.batch / step_s
-    out = {"impl": "reference", "metric": "decode tokens/s (batch tokens per decode step / step time)",
+    out = {"impl": "reference", "metric": METRIC,
            "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+           "warmup": args.warmup, "ms_per_step": layer_s * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": workload_config(cfg),
+           "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "1 GPU",
+           "timed_unit": f"one of the {cfg.n_layers} layers of the decode step per timed step (a bounded "
+                         f"sample); value extrapolates: median layer x {cfg.n_layers} + LM head "
+                         f"= {step_s * 1e3:.1f} ms per decode step",
+           "extrapolated_ms_per_decode_step": step_s * 1e3,
            "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": "tokens/s",
-                            "sample": f"each step: one of {cfg.n_layers} layers (fp64, single thread); step time = "
-                                      f"median layer x {cfg.n_layers} + LM head = {step_s:.3f} s"},
+                            "sample": f"each timed step: one of {cfg.n_layers} layers (fp64, single thread); "
+                                      f"decode step = median layer x {cfg.n_layers} + LM head = {step_s:.3f} s"},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
-def workload_config(cfg):
+def workload_config(cfg, paged=False):
+    """The workload a line measures; the same dict in both arms."""
     ctx = f"ctx U[{cfg.ctx_lo},{cfg.ctx_hi}]" if cfg.ragged else f"ctx {cfg.ctx}"
-    return {"workload": f"{cfg.name}: {cfg.n_layers} layers, hidden {cfg.hidden}, {cfg.n_q_heads}q/{cfg.n_kv_heads}kv "
-                        f"heads x {cfg.head_dim}, ffn {cfg.ffn_dim or cfg.expert_ffn_dim}, vocab {cfg.vocab}; "
-                        f"batch {cfg.batch}, {ctx}, teacher-forced decode",
-            "batch": cfg.batch, "max_ctx": cfg.max_ctx, "weights": "bf16 ~N(0,0.02), seeded",
-            "kv_cache": "bf16 ~N(0,1), seeded", "accumulate": "fp32",
-            "l2": "inputs larger than L2 (weights stream from HBM every step)"}
+    out = {"workload": f"{cfg.name}: {cfg.n_layers} layers, hidden {cfg.hidden}, {cfg.n_q_heads}q/{cfg.n_kv_heads}kv "
+                       f"heads x {cfg.head_dim}, ffn {cfg.ffn_dim or cfg.expert_ffn_dim}, vocab {cfg.vocab}; "
+                       f"batch {cfg.batch}, {ctx}, teacher-forced decode",
+           "batch": cfg.batch, "max_ctx": cfg.max_ctx, "weights": "bf16 ~N(0,0.02), seeded",
+           "kv_cache": "bf16 ~N(0,1), seeded", "accumulate": "fp32",
+           "l2": "inputs larger than L2 (weights stream from HBM every step)"}
+    if paged:
+        out["kv_layout"] = f"paged, {32768 // (2 * cfg.head_dim)}-position pages in a shuffled pool"
+    return out
 
 
 # ---------------------------------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------------------------------
 
-def run_mk(args, cfg, rank, world):
+def make_decoder(cfg, seed, dev, paged):
+    """Seeded device weights and caches of cfg and a Decoder on them (the cache as a shuffled page pool
+    when paged)."""
     import torch
     import auto_regressive_decode_b200.mk as mk
     from fixtures.device import device_caches, device_model
-
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    seed = fx.DEFAULT_SEED + rank
     S0 = fx.context_lengths(cfg, seed)
-    toks = fx.tokens(cfg, seed)
     w = device_model(cfg, seed)
     kc, vc = device_caches(cfg, S0, seed)
-    if args.paged:
-        # the same cache as a page pool: one attention stage per page, pages in a seeded random order
-        page = 32768 // (2 * cfg.head_dim)
-        stride = -(-cfg.max_ctx // page)
-        table = np.random.default_rng(seed).permutation(cfg.batch * stride).reshape(cfg.batch, stride)
-        pools = []
-        for c in (kc, vc):
-            L, B_, nkv, T, hd = c.shape
-            pool = torch.empty((L, cfg.batch * stride, nkv, page, hd), dtype=c.dtype, device=c.device)
-            for b in range(B_):
-                for j in range(stride):
-                    lo, hi = j * page, min(T, (j + 1) * page)
-                    pool[:, int(table[b, j]), :, :hi - lo] = c[:, b, :, lo:hi]
-            pools.append(pool)
-        del kc, vc
-        kc, vc = pools
-        d_table = torch.from_numpy(table.astype(np.int32)).to(dev)
-        dec = mk.Decoder(cfg, w, kc, vc, block_table=d_table, page_size=page)
-    else:
-        dec = mk.Decoder(cfg, w, kc, vc)
+    if not paged:
+        return mk.Decoder(cfg, w, kc, vc), S0
+    # one attention stage per page, pages in a seeded random order
+    page = 32768 // (2 * cfg.head_dim)
+    stride = -(-cfg.max_ctx // page)
+    table = np.random.default_rng(seed).permutation(cfg.batch * stride).reshape(cfg.batch, stride)
+    pools = []
+    for c in (kc, vc):
+        L, B_, nkv, T, hd = c.shape
+        pool = torch.empty((L, cfg.batch * stride, nkv, page, hd), dtype=c.dtype, device=c.device)
+        for b in range(B_):
+            for j in range(stride):
+                lo, hi = j * page, min(T, (j + 1) * page)
+                pool[:, int(table[b, j]), :, :hi - lo] = c[:, b, :, lo:hi]
+        pools.append(pool)
+    del kc, vc
+    d_table = torch.from_numpy(table.astype(np.int32)).to(dev)
+    return mk.Decoder(cfg, w, pools[0], pools[1], block_table=d_table, page_size=page), S0
+
+
+def measure(args, cfg, rank, world, dev, full=True):
+    """Time args.steps decode steps of cfg after args.warmup untimed ones (CUDA events on the launching
+    stream, max over ranks).  full: also the end-to-end (host buffers) and greedy-loop numbers."""
+    import torch
+    import auto_regressive_decode_b200.mk as mk
+
+    seed = fx.DEFAULT_SEED + rank
+    dec, S0 = make_decoder(cfg, seed, dev, args.paged)
+    toks = fx.tokens(cfg, seed)
     B, V = cfg.batch, cfg.vocab
     n_total = args.warmup + args.steps
     # per-step inputs, resident on the device (teacher forcing; positions wrap after cfg.steps)
@@ -321,12 +342,15 @@ def run_mk(args, cfg, rank, world):
             import torch.distributed as dist
             dist.barrier()
 
+    def check():
+        st = dec.status()
+        if st != 0:
+            raise RuntimeError(f"{cfg.name}: device status {mk.mk_status_string(st)}")
+
     for i in range(args.warmup):
         dec.step(all_tok[i], all_len[i], all_len[i], logits)
     torch.cuda.synchronize()
-    st = dec.status()
-    if st != 0:
-        raise RuntimeError(f"device status {mk.mk_status_string(st)}")
+    check()
 
     # ---- device-resident timing: one event pair per step, on the launching stream
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
@@ -342,37 +366,9 @@ def run_mk(args, cfg, rank, world):
             ev[j + 1].record(stream)
         torch.cuda.synchronize()
     barrier()
-    st = dec.status()
-    if st != 0:
-        raise RuntimeError(f"device status {mk.mk_status_string(st)}")
+    check()
     per_step_ms = [ev[j].elapsed_time(ev[j + 1]) for j in range(args.steps)]
     total_ms = ev[0].elapsed_time(ev[-1])
-
-    # ---- end to end through the C ABI with host buffers
-    h_tok = torch.from_numpy(toks[steps_idx].astype(np.int32)).pin_memory()
-    h_len = torch.from_numpy((S0[None, :] + steps_idx[:, None]).astype(np.int32)).pin_memory()
-    h_logits = torch.empty((B, V), dtype=torch.float32).pin_memory()
-    d_tok = torch.empty(B, dtype=torch.int32, device=dev)
-    d_len = torch.empty(B, dtype=torch.int32, device=dev)
-    d_pos = torch.empty(B, dtype=torch.int32, device=dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for j in range(args.steps):
-        i = args.warmup + j
-        d_tok.copy_(h_tok[i], non_blocking=True)
-        d_len.copy_(h_len[i], non_blocking=True)
-        d_pos.copy_(h_len[i], non_blocking=True)
-        dec.step(d_tok, d_pos, d_len, logits)
-        h_logits.copy_(logits, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    st = dec.status()
-    if st != 0:
-        raise RuntimeError(f"device status {mk.mk_status_string(st)}")
 
     # ---- MoE: the distinct experts each timed step read (its routing, replayed untimed)
     distinct = []
@@ -382,48 +378,65 @@ def run_mk(args, cfg, rank, world):
             dec.step(all_tok[i], all_len[i], all_len[i], logits)
             distinct.append(int(dec.routing()[3].sum()))
 
-    # ---- on-device greedy decoding: K steps in one call, each step's arg-max fed back on the device
-    # (after the MoE replay: the loop rewrites cache rows below S0 to make room)
-    picks = torch.empty((args.steps, B), dtype=torch.int32, device=dev)
-    g_len = torch.from_numpy(np.maximum(S0 - args.steps, 0).astype(np.int32)).to(dev)  # room for K steps
-    g_tok = all_tok[0].clone()
-    dec.greedy(3, g_tok, g_len, picks)  # warm-up
-    torch.cuda.synchronize()
-    barrier()
-    e0.record(stream)
-    dec.greedy(args.steps, g_tok, g_len, picks)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    greedy_ms = e0.elapsed_time(e1)
-    st = dec.status()
-    if st != 0:
-        raise RuntimeError(f"device status {mk.mk_status_string(st)}")
+    e2e_ms = greedy_ms = float("nan")
+    if full:
+        # ---- end to end through the C ABI with host buffers
+        h_tok = torch.from_numpy(toks[steps_idx].astype(np.int32)).pin_memory()
+        h_len = torch.from_numpy((S0[None, :] + steps_idx[:, None]).astype(np.int32)).pin_memory()
+        h_logits = torch.empty((B, V), dtype=torch.float32).pin_memory()
+        d_tok = torch.empty(B, dtype=torch.int32, device=dev)
+        d_len = torch.empty(B, dtype=torch.int32, device=dev)
+        d_pos = torch.empty(B, dtype=torch.int32, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for j in range(args.steps):
+            i = args.warmup + j
+            d_tok.copy_(h_tok[i], non_blocking=True)
+            d_len.copy_(h_len[i], non_blocking=True)
+            d_pos.copy_(h_len[i], non_blocking=True)
+            dec.step(d_tok, d_pos, d_len, logits)
+            h_logits.copy_(logits, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        check()
+
+        # ---- on-device greedy decoding: K steps in one call, each step's arg-max fed back on the device
+        # (after the MoE replay: the loop rewrites cache rows below S0 to make room)
+        picks = torch.empty((args.steps, B), dtype=torch.int32, device=dev)
+        g_len = torch.from_numpy(np.maximum(S0 - args.steps, 0).astype(np.int32)).to(dev)  # room for K steps
+        g_tok = all_tok[0].clone()
+        dec.greedy(3, g_tok, g_len, picks)  # warm-up
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        dec.greedy(args.steps, g_tok, g_len, picks)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        greedy_ms = e0.elapsed_time(e1)
+        check()
 
     # ---- max over ranks
     total_ms, e2e_ms, greedy_ms = max_over_ranks([total_ms, e2e_ms, greedy_ms], world, dev)
     dec.close()
-    if rank != 0:
-        return
+    del dec, all_tok, all_len, logits
+    torch.cuda.empty_cache()
 
     ms = total_ms / args.steps
-    tok_s = job_tokens_per_s(world, B, args.steps, total_ms)
-    e2e_tok_s = job_tokens_per_s(world, B, args.steps, e2e_ms)
     lens = [S0 + (k % cfg.steps) for k in range(args.warmup, n_total)]
     bytes_step = weight_bytes_read(cfg) + float(np.mean([kv_bytes(cfg, s) for s in lens]))
     if cfg.n_experts:
         bytes_step += expert_bytes_read(cfg, distinct)
     peak, peak_kind = measured_peaks()
     achieved = bytes_step / (ms / 1e3) / 1e9
-    traffic = ncu_traffic(cfg.name)
-    out = {
-        "metric": "decode tokens/s (batch tokens per decode step / step time)",
-        "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded random-init weights and KV cache, uniform token ids)",
-        "config": dict(workload_config(cfg), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
-                       **({"kv_layout": f"paged, {32768 // (2 * cfg.head_dim)}-position pages in a shuffled pool"}
-                          if args.paged else {})),
+    r = {
+        "workload": workload_config(cfg)["workload"],
+        "ms_per_step": ms,
+        "tokens_per_s": job_tokens_per_s(world, B, args.steps, total_ms),
         "step_latency_ms": {"median": statistics.median(per_step_ms), "p10": float(np.percentile(per_step_ms, 10)),
                             "p90": float(np.percentile(per_step_ms, 90))},
         "bytes_per_step": bytes_step,
@@ -431,14 +444,55 @@ def run_mk(args, cfg, rank, world):
         "mbu": {"vs_spec_8tbs": achieved / SPEC_HBM_GBS, f"vs_{peak_kind}_{peak:.0f}gbs": achieved / peak},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                     else "fallback", "traffic": traffic, "kernel": "mk_persistent"},
-        "e2e": {"value": e2e_tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 3 * 4 * B,
-                "d2h_bytes_per_step": 4 * B * V},
-        "greedy_loop": {"value": job_tokens_per_s(world, B, args.steps, greedy_ms), "unit": "tokens/s",
-                        "note": "mk_decode_greedy: K steps in one call, arg-max fed back on the device"},
-        "gpu_launches": args.steps,
+                     else "fallback", "traffic": ncu_traffic(cfg.name), "kernel": "mk_persistent"},
         "clocks": clk.summary(),
     }
+    if full:
+        r["e2e_ms"] = e2e_ms
+        r["greedy_ms"] = greedy_ms
+    return r
+
+
+def run_mk(args, cfg, rank, world):
+    import torch
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    m = measure(args, cfg, rank, world, dev, full=True)
+    per_config = {}
+    if args.per_config and not args.layers and cfg.name == MAIN_CONFIG:
+        for name in PER_CONFIG:
+            c = fx.CONFIGS[name]
+            pc = measure(args, c, rank, world, dev, full=False)
+            per_config[name] = {k: pc[k] for k in ("workload", "ms_per_step", "tokens_per_s", "step_latency_ms",
+                                                   "bytes_per_step", "mbu", "roofline", "clocks")}
+            if c.n_experts:
+                per_config[name]["moe_distinct_experts_per_layer"] = pc["moe_distinct_experts_per_layer"]
+    if rank != 0:
+        return
+    B, V = cfg.batch, cfg.vocab
+    out = {
+        "metric": METRIC,
+        "value": m["tokens_per_s"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights and KV cache, uniform token ids)",
+        "config": workload_config(cfg, args.paged),
+        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+        "step_latency_ms": m["step_latency_ms"],
+        "bytes_per_step": m["bytes_per_step"],
+        **({"moe_distinct_experts_per_layer": m["moe_distinct_experts_per_layer"]} if cfg.n_experts else {}),
+        "mbu": m["mbu"],
+        "roofline": m["roofline"],
+        "e2e": {"value": job_tokens_per_s(world, B, args.steps, m["e2e_ms"]), "unit": "tokens/s",
+                "h2d_bytes_per_step": 3 * 4 * B, "d2h_bytes_per_step": 4 * B * V},
+        "greedy_loop": {"value": job_tokens_per_s(world, B, args.steps, m["greedy_ms"]), "unit": "tokens/s",
+                        "note": "mk_decode_greedy: K steps in one call, arg-max fed back on the device"},
+        "gpu_launches": args.steps,
+        "clocks": m["clocks"],
+    }
+    if per_config:
+        out["per_config"] = per_config
     if not args.no_cpu_baseline and world == 1:  # the oracle baseline: rank 0 at one GPU only
         base = cpu_baseline(cfg)
         out["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
@@ -450,9 +504,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="dense-8b", choices=sorted(fx.CONFIGS))
+    ap.add_argument("--config", default=MAIN_CONFIG, choices=sorted(fx.CONFIGS))
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the other configurations the default line reports under per_config")
     ap.add_argument("--paged", action="store_true", help="run the KV cache as a paged pool (block table)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: the config with this many layers (same shapes); not a bench line")
