@@ -403,6 +403,7 @@ extern "C" size_t mk_state_bytes(const mk_handle* h, int which) {
     case MK_STATE_SEL_WEIGHT: return d.n_experts ? sizeof(float) * (size_t)d.n_layers * d.batch * d.top_k : 0;
     case MK_STATE_EXPERT_COUNT: return d.n_experts ? sizeof(int32_t) * (size_t)d.n_layers : 0;
     case MK_STATE_TRACE: return sizeof(uint64_t) * mk::kTraceStamps * h->n_instr;
+    case MK_STATE_COUNTERS: return sizeof(uint32_t) * (size_t)h->n_counters;
     default: return 0;
   }
 }
@@ -419,6 +420,7 @@ extern "C" int mk_read_state(mk_handle* h, int which, void* dst, size_t bytes, v
   if (which == MK_STATE_SELECTION) src = h->p.moe_sel;
   if (which == MK_STATE_SEL_WEIGHT) src = h->p.moe_selw;
   if (which == MK_STATE_EXPERT_COUNT) src = h->p.moe_count;
+  if (which == MK_STATE_COUNTERS) src = h->p.counters;
   if (cudaMemcpyAsync(dst, src, need, cudaMemcpyDefault, (cudaStream_t)stream) != cudaSuccess) return MK_ERR_CUDA;
   return MK_OK;
 }

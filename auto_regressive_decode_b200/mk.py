@@ -25,6 +25,7 @@ MK_STATE_SELECTION = 2
 MK_STATE_SEL_WEIGHT = 3
 MK_STATE_EXPERT_COUNT = 4
 MK_STATE_TRACE = 5
+MK_STATE_COUNTERS = 6
 
 OP_NAMES = {0: "nop", 1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead",
             8: "router", 9: "exp_gateup", 10: "exp_down"}
@@ -263,6 +264,14 @@ class Decoder:
         n = self.read_state(MK_STATE_EXPERT_COUNT, torch.empty((L,), dtype=torch.int32, device="cuda"))
         torch.cuda.synchronize()
         return r.cpu().numpy(), sel.cpu().numpy(), w.cpu().numpy(), n.cpu().numpy()
+
+    def counters(self):
+        """uint32 dependency counters after the last step (host numpy), in mk_plan_counter_targets order."""
+        import numpy as np
+        n = mk_state_bytes(self.h, MK_STATE_COUNTERS) // 4
+        c = self.read_state(MK_STATE_COUNTERS, self.torch.empty((n,), dtype=self.torch.int32, device="cuda"))
+        self.torch.cuda.synchronize()
+        return c.cpu().numpy().view(np.uint32)
 
     def close(self):
         if getattr(self, "h", None):

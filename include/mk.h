@@ -176,14 +176,20 @@ const char* mk_status_string(int status);
  *                        first copy issued, prologue done, first stage landed,
  *                        last stage consumed, producer's last copy issued.
  *                        Only for handles created with the environment variable
- *                        MK_TRACE=1 (0 bytes otherwise). */
+ *                        MK_TRACE=1 (0 bytes otherwise).
+ *   MK_STATE_COUNTERS    uint32[mk_plan_n_counters] the dependency counters
+ *                        after the last step: each has counted epoch x its
+ *                        target (mk_plan_counter_targets), epoch being the steps run
+ *                        since the handle was made or a failing step's status
+ *                        was read (that read clears them) */
 enum {
   MK_STATE_HIDDEN = 0,
   MK_STATE_ROUTER = 1,
   MK_STATE_SELECTION = 2,
   MK_STATE_SEL_WEIGHT = 3,
   MK_STATE_EXPERT_COUNT = 4,
-  MK_STATE_TRACE = 5
+  MK_STATE_TRACE = 5,
+  MK_STATE_COUNTERS = 6
 };
 int mk_read_state(mk_handle* h, int which, void* dst, size_t bytes, void* stream);
 
