@@ -34,7 +34,7 @@ struct Params {
   // cache and the V cache
   const uint8_t* tmaps;
   // batch-1 kernel: 2-D TMA maps of every weight matrix, kB1BoxHeights per
-  // matrix (boxes of kB1Chunk columns x 16, 8, 4, 2, 1 rows): [layer][wq wk wv
+  // matrix (boxes of kB1Chunk columns x 64, 32, 16, 8, 4, 2, 1 rows): [layer][wq wk wv
   // wo w_gate w_up w_down], then the LM head
   const uint8_t* tmaps_b1;
   // library scratch (device)

@@ -74,14 +74,15 @@ inline int n_counters(int n_layers) { return n_layers * C_PER_LAYER + 2; }
 // Row-stationary tiles: an instruction owns `lines` weight rows (rows x matrices;
 // gate/up pairs count twice) and streams K in chunks of kB1Chunk columns.  A
 // stage holds every line of the instruction for `nc` consecutive chunks, each
-// line a 512-byte row of shared memory, moved by 2-D TMA boxes of 8 rows or 1
-// row (no swizzle).  Consumer warp w owns the rows r == w (mod 8) of every
-// stage and keeps their partial dot products in registers across all chunks:
-// one warp reduction per instruction, none per stage.
+// line a 512-byte row of shared memory, moved by 2-D TMA boxes of 64 down to 1
+// rows (no swizzle; few, tall boxes: each box costs the copy engine a fixed
+// time).  Consumer warps keep the partial dot products of their lines in
+// registers across all chunks: one warp reduction per instruction, none per stage.
 constexpr int kB1Chunk = 256;          // columns per chunk (the TMA box width)
 constexpr int kB1LineBytes = kB1Chunk * 2;
 constexpr int kB1MaxLines = 64;        // lines per instruction (64 x 512 B = one stage)
-constexpr int kB1BoxHeights = 5;       // box maps of 16, 8, 4, 2 and 1 rows per matrix
+constexpr int kB1TallestBox = 64;      // box maps of 64, 32, 16, 8, 4, 2 and 1 rows per matrix
+constexpr int kB1BoxHeights = 7;
 constexpr int kB1MapsPerLayer = 7 * kB1BoxHeights;  // wq wk wv wo w_gate w_up w_down
 // The input vector of a batch-1 GEMV sits in shared memory (fp32, the norm's
 // gain applied) in pieces of at most kB1XPieceFloats columns, loaded once per

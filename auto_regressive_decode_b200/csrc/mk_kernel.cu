@@ -440,7 +440,7 @@ struct Gemv {
 };
 
 // Batch-1 box maps of matrix `mat` (0..6: wq wk wv wo w_gate w_up w_down) of
-// a layer: kB1BoxHeights maps, of 16, 8, 4, 2 and 1 rows.
+// a layer: kB1BoxHeights maps, of 64, 32, 16, 8, 4, 2 and 1 rows.
 __device__ __forceinline__ const uint8_t* b1_map(const Params& p, int layer, int mat) {
   return p.tmaps_b1 + ((size_t)layer * kB1MapsPerLayer + kB1BoxHeights * mat) * 128;
 }
@@ -707,8 +707,8 @@ struct Cursor {
   }
 
   // Batch-1 GEMV: the TMA boxes of one chunk of every line, into `box` (the
-  // same for every chunk but for the column): a segment's rows as boxes of 16,
-  // 8, 4, 2 and 1 rows, largest first (single rows only when K is narrower
+  // same for every chunk but for the column): a segment's rows as boxes of 64,
+  // 32, 16, 8, 4, 2 and 1 rows, largest first (single rows only when K is narrower
   // than a chunk, whose boxes are K wide).  Chunk j's line l lands at
   // shared-memory line (j - first chunk of the stage) * lines + l.  Returns
   // the number of boxes.
@@ -720,7 +720,7 @@ struct Cursor {
       const int n = g.seg_rows(s2), row = g.seg_row(s2), line = g.seg_line(s2);
       int r = 0;
       for (int m = wide ? 0 : kB1BoxHeights - 1; m < kB1BoxHeights; ++m) {
-        const int h = 16 >> m;
+        const int h = kB1TallestBox >> m;
         for (; r + h <= n; r += h) {
           box[nb].map = map + 128 * m;
           box[nb].row = row + r;
@@ -1879,15 +1879,15 @@ struct Consumer {
     constexpr int MT = P / 16 / kConsumerWarps;  // key tiles per warp per stage
     constexpr int KS = HD / 16;                  // k-steps of the score mma
     constexpr int DT = HD / 16;                  // dimension tiles of the P.V mma
-    // the batch-1 kernel unrolls its inner loops less: fewer fragments in
-    // flight keep its registers within the budget of the fp32 GEMV loops
+    // full unrolling on the tensor-core kernel (an instance in the batch-1
+    // kernel, which runs attn_ff, would unroll less to keep its registers)
     constexpr int KU = BATCHED ? KS : 2, DU = BATCHED ? DT : 4;
     constexpr uint32_t CBB = (uint32_t)P * 128u;  // bytes of one 64-column block of a stage
     const int gq = lane >> 2, cq = lane & 3;
-    // The batch-1 kernel (fp32 activations elsewhere) takes q and the
-    // probabilities as sums of two bf16 parts (hi + lo), whose two mma keep
-    // scores and outputs at about fp32 accuracy (keys and values are bf16
-    // already); the tensor-core kernel rounds them to one bf16, like its GEMV inputs.
+    // The tensor-core kernel rounds q and the probabilities to one bf16, like
+    // its GEMV inputs.  SPLIT (not taken: the batch-1 kernel runs attn_ff)
+    // would take them as sums of two bf16 parts (hi + lo), whose two mma keep
+    // scores and outputs at about fp32 accuracy (keys and values are bf16 already).
     constexpr bool SPLIT = !BATCHED;
     uint32_t qf[KS][2], ql[KS][2];
 #pragma unroll

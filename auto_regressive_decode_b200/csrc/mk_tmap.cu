@@ -13,6 +13,8 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <algorithm>
+
 #include "mk_device.h"
 
 namespace mk {
@@ -72,10 +74,11 @@ bool encode_2d(EncodeTiledFn enc, const void* w, int64_t rows, int K, int box_ro
   return true;
 }
 
-// The box maps of one matrix: 16, 8, 4, 2 and 1 rows.
+// The box maps of one matrix: 64, 32, 16, 8, 4, 2 and 1 rows (a height above the
+// matrix's row count is encoded at that count; the kernel never uses it).
 bool encode_set(EncodeTiledFn enc, const void* w, int64_t rows, int K, uint8_t* out) {
   for (int m = 0; m < kB1BoxHeights; ++m)
-    if (!encode_2d(enc, w, rows, K, 16 >> m, out + 128 * m)) return false;
+    if (!encode_2d(enc, w, rows, K, (int)std::min<int64_t>(kB1TallestBox >> m, rows), out + 128 * m)) return false;
   return true;
 }
 
