@@ -88,7 +88,8 @@ def kernel_source_hash() -> str:
 
 
 def ncu_traffic(workload: str):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken on the current kernel source."""
+    """DRAM bytes per launch of the full workload, scaled from a committed ncu capture of its small case
+    (`--layers`) by the algorithmic bytes, if that capture was taken on the current kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
