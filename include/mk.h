@@ -208,8 +208,7 @@ size_t mk_state_bytes(const mk_handle* h, int which);
  * until the process exits.  A model whose state (instruction lists, counters,
  * activations, RoPE table) needs more returns MK_ERR_UNSUPPORTED.
  *   - The first call on a device resolves the array's address there
- *     (cudaGetSymbolAddress with that device current); make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress with that device current).
  *   - Each call clears the counters and status words it uses, uploads the
  *     instruction lists from temporary host memory, launches on `stream` and
  *     then synchronises `stream` so that it can return the device-side status
