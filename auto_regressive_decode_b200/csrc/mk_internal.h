@@ -89,9 +89,13 @@ constexpr int kB1MapsPerLayer = 7 * kB1BoxHeights;  // wq wk wv wo w_gate w_up w
 // piece with one round trip to L2: the same op's next instruction on the SM
 // reuses it, and a K longer than a piece reloads mid-instruction.
 constexpr int kB1XPieceFloats = 6144;
-MK_HD int b1_max_rows(int op) { return op == OP_GATEUP ? kB1MaxLines / 2 : kB1MaxLines; }
+// rows (gate/up: neurons) per instruction; a gate/up instruction of more than
+// kB1MaxLines / 2 neurons streams its gate rows and its up rows as two groups
+MK_HD int b1_max_rows(int op) { return kB1MaxLines; }
 // chunks per stage: as many as fill a stage with the instruction's lines
 MK_HD int b1_chunks_per_stage(int lines) { return lines > 32 ? 1 : (lines > 16 ? 2 : 4); }
+// chunks per input piece: whole stages
+MK_HD int b1_piece_chunks(int ncs) { return kB1XPieceFloats / kB1Chunk / ncs * ncs; }
 static_assert(kB1MaxLines * kB1LineBytes == kStageBytes, "a stage of 64 lines fills a ring slot");
 
 // ---- batch > 1 GEMV (tensor cores) -------------------------------------------------

@@ -431,6 +431,9 @@ struct Gemv {
   // (the others follow it), first row within its matrix, rows and first line
   // within a stage
   int lines, nch, ncs, nst, nseg;
+  // gate/up of more than kB1MaxLines / 2 neurons: a stage holds one group (the
+  // gate rows or the up rows) of one chunk, gate then up for every chunk
+  bool split;
   const uint8_t *bm0, *bm1, *bm2;
   int brow0, brow1, brow2, bn0, bn1, bn2, bl0, bl1, bl2;
   __device__ __forceinline__ int seg_rows(int s) const { return s == 0 ? bn0 : (s == 1 ? bn1 : bn2); }
@@ -518,6 +521,13 @@ __device__ __forceinline__ Gemv gemv_geo(const Params& p, const mk_instr& in, in
   g.nch = (g.K + kB1Chunk - 1) / kB1Chunk;
   g.ncs = b1_chunks_per_stage(g.lines);
   g.nst = (g.nch + g.ncs - 1) / g.ncs;
+  g.split = !p.tc && g.gated && g.lines > kB1MaxLines;
+  if (g.split) {  // both groups start at line 0 of their stages
+    g.bl1 = 0;
+    g.lines = R;
+    g.ncs = 1;
+    g.nst = 2 * g.nch;
+  }
   if (p.tc) {
     const int tr = btile_rows(g.gated);
     g.bnch = (g.K + kBChunk - 1) / kBChunk;
@@ -545,6 +555,7 @@ __device__ __forceinline__ Gemv moe_gate_piece(const Params& p, const Ctl* ctl, 
   gm.r0 = e * p.Ie + t0 * 8;
   gm.r1 = e * p.Ie + t1 * 8;
   gm.gated = true;
+  gm.split = false;
   gm.bnch = (p.H + kBChunk - 1) / kBChunk;
   gm.bnt = t1 - t0;
   *slot = s;
@@ -711,11 +722,13 @@ struct Cursor {
   // 32, 16, 8, 4, 2 and 1 rows, largest first (single rows only when K is narrower
   // than a chunk, whose boxes are K wide).  Chunk j's line l lands at
   // shared-memory line (j - first chunk of the stage) * lines + l.  Returns
-  // the number of boxes.
-  __device__ __forceinline__ int b1_box_list(Ctl::B1Box* box) const {
+  // the number of boxes; *nb0 = those of the first segment.
+  __device__ __forceinline__ int b1_box_list(Ctl::B1Box* box, int* nb0) const {
     const bool wide = g.K >= kB1Chunk;
     int nb = 0;
+    *nb0 = 0;
     for (int s2 = 0; s2 < g.nseg; ++s2) {
+      if (s2 == 1) *nb0 = nb;
       const uint8_t* map = g.seg_map(s2);
       const int n = g.seg_rows(s2), row = g.seg_row(s2), line = g.seg_line(s2);
       int r = 0;
@@ -784,6 +797,7 @@ struct Cursor {
       return (uint32_t)kStageBytes;  // a TMA box: always a whole stage of positions
     if (pp->tc) return (g.gated || g.r1 - g.r0 - sg * 16 > 8) ? 2u * kBBoxBytes : (uint32_t)kBBoxBytes;
     // batch 1: every line of every chunk of the stage, one box width each
+    if (g.split) return (uint32_t)g.lines * (uint32_t)min(g.K, kB1Chunk) * 2u;  // one group of one chunk
     const int j0 = kc * g.ncs, nj = min(g.nch, j0 + g.ncs) - j0;
     return (uint32_t)(g.lines * nj) * (uint32_t)min(g.K, kB1Chunk) * 2u;
   }
@@ -884,22 +898,36 @@ __device__ __forceinline__ void run_producer(const Params& p, const mk_instr* li
       if (cur.op != OP_ATTN) {
         // a batch-1 GEMV instruction: its box list once, then every stage from it
         Ctl::B1Box* box = ctl->b1box;
-        const int nbox = cur.b1_box_list(box);
+        int nb0;
+        const int nbox = cur.b1_box_list(box, &nb0);
         const int nch = cur.g.nch, ncs = cur.g.ncs, nst = cur.g.nst;
         const uint32_t chunk_stride = (uint32_t)cur.g.lines * kB1LineBytes;
         const uint32_t chunk_bytes = (uint32_t)cur.g.lines * (uint32_t)min(cur.g.K, kB1Chunk) * 2u;
-        for (int kc = 0; kc < nst && ok; ++kc) {
-          uint8_t* dst;
-          unsigned long long* bar;
-          if (!(ok = pr.claim(&dst, &bar, [&]() {}))) break;
-          const int j0 = kc * ncs, nj = min(nch - j0, ncs);
-          mbar_arrive_expect_tx(bar, chunk_bytes * (uint32_t)nj);
-          for (int jj = 0; jj < nj; ++jj) {
-            uint8_t* dj = dst + jj * chunk_stride;
-            const int col = (j0 + jj) * kB1Chunk;
-            for (int b = 0; b < nbox; ++b) tma_box2(dj + box[b].off, box[b].map, col, box[b].row, bar, pr.pol);
+        if (cur.g.split) {
+          // two groups: stage 2c holds chunk c of the gate rows, stage 2c + 1 of the up rows
+          for (int kc = 0; kc < nst && ok; ++kc) {
+            uint8_t* dst;
+            unsigned long long* bar;
+            if (!(ok = pr.claim(&dst, &bar, [&]() {}))) break;
+            mbar_arrive_expect_tx(bar, chunk_bytes);
+            const int col = (kc >> 1) * kB1Chunk, b0 = (kc & 1) ? nb0 : 0, b1 = (kc & 1) ? nbox : nb0;
+            for (int b = b0; b < b1; ++b) tma_box2(dst + box[b].off, box[b].map, col, box[b].row, bar, pr.pol);
+            ++pr.k;
           }
-          ++pr.k;
+        } else {
+          for (int kc = 0; kc < nst && ok; ++kc) {
+            uint8_t* dst;
+            unsigned long long* bar;
+            if (!(ok = pr.claim(&dst, &bar, [&]() {}))) break;
+            const int j0 = kc * ncs, nj = min(nch - j0, ncs);
+            mbar_arrive_expect_tx(bar, chunk_bytes * (uint32_t)nj);
+            for (int jj = 0; jj < nj; ++jj) {
+              uint8_t* dj = dst + jj * chunk_stride;
+              const int col = (j0 + jj) * kB1Chunk;
+              for (int b = 0; b < nbox; ++b) tma_box2(dj + box[b].off, box[b].map, col, box[b].row, bar, pr.pol);
+            }
+            ++pr.k;
+          }
         }
         if (!ok) break;
         cur.seek(cur.i + 1);
@@ -1043,6 +1071,110 @@ struct Consumer {
     }
   }
 
+  // ---- GEMV, batch 1: gate/up of more than 32 neurons ------------------------
+  // The instruction's gate rows and its up rows stream as two groups, a stage
+  // holding one group's R <= 64 lines of one chunk: chunk c's gate stage, then
+  // its up stage.  Warp w owns the neurons w, w + 8, ... (< R); the partial
+  // sums of their gate and up lines stay in registers as fp32, each stage's
+  // pair of fma chains folded in (16 values per lane, as many registers as the
+  // 8 packed pairs of the one-group path), and one 16-value warp reduction
+  // ends the instruction.  Input pieces, norm and SwiGLU epilogue as in gemv_b1.
+  __device__ __forceinline__ bool gemv_b1_gu2(const mk_instr& in, int layer, const Gemv& g) {
+    const int H = p.H, K = g.K, R = g.r1 - g.r0, nch = g.nch;
+    const float* src = p.xres + (size_t)(2 * layer + 1) * H;
+    const uint16_t* gain = p.layers[layer].mlp_norm;
+    uint32_t own = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (warp + 8 * k < R) own |= 1u << k;
+    if (!wait_counter(in.wait_idx, in.wait_count)) return false;
+    if (tr) tr[1] = globaltimer();
+    float4* xb = reinterpret_cast<float4*>(red);
+    const uint32_t xs0 = smem_addr(red);
+    const int pch = b1_piece_chunks(1);
+    const bool narrow = K < kB1Chunk;
+    float ag[8], au[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ag[k] = au[k] = 0.f;
+    for (int c0 = 0; c0 < nch; c0 += pch) {
+      const int c1 = min(nch, c0 + pch);
+      const uint32_t tag = ((uint32_t)layer << 12 | (uint32_t)OP_GATEUP << 6 | (uint32_t)(c0 / pch)) + 1u;
+      if (ctl->xtag != tag) {
+        if (c0 > 0) consumer_bar();  // every warp is done with the previous piece
+        float ss = 0.f;
+        for (int f = t; f < (c1 - c0) * 64; f += kConsumerThreads) {
+          const int col = c0 * kB1Chunk + 4 * f;
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (col < K) {
+            v = __ldcg(reinterpret_cast<const float4*>(src + col));
+            const uint2 gv = __ldg(reinterpret_cast<const uint2*>(gain + col));
+            ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+            v.x *= bf16_lo(gv.x);
+            v.y *= bf16_hi(gv.x);
+            v.z *= bf16_lo(gv.y);
+            v.w *= bf16_hi(gv.y);
+          }
+          const int ff = f & 63;
+          xb[((f >> 6) * 2 + (ff & 1)) * 32 + (ff >> 1)] = v;
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) ctl->sred[warp] = ss;
+        consumer_bar();
+        if (t == 0) {
+          float s2 = 0.f;
+#pragma unroll
+          for (int w2 = 0; w2 < kConsumerWarps; ++w2) s2 += ctl->sred[w2];
+          ctl->xss = (c0 == 0 ? 0.f : ctl->xss) + s2;  // pieces of the same input, in order
+          ctl->xtag = tag;
+        }
+        consumer_bar();
+      }
+      if (tr && c0 == 0) tr[4] = globaltimer();
+#pragma unroll 1
+      for (int c = c0; c < c1; ++c) {
+        const uint32_t xa = xs0 + (uint32_t)((c - c0) * 2 * 32 + lane) * 16u;
+        const float4 x0 = lds_f4(xa), x1 = lds_f4(xa + 512u);
+        const unsigned long long xp[4] = {pack2(x0.x, x0.y), pack2(x0.z, x0.w), pack2(x1.x, x1.y),
+                                          pack2(x1.z, x1.w)};
+        const uint32_t lanes_ok = !narrow || c * kB1Chunk + lane * 8 < K;
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {  // the gate stage, then the up stage
+          const uint8_t* w = wait_full();
+          if (tr && c == 0 && grp == 0) tr[5] = globaltimer();
+          const uint32_t wj = smem_addr(w) + (uint32_t)(warp * kB1LineBytes + lane * 16);
+          uint4 wv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) wv[k] = lds_u4_if(wj + (uint32_t)(8 * k) * kB1LineBytes, ((own >> k) & 1u) & lanes_ok);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float d = sum2(dot8x2(wv[k], xp, 0ull));
+            if (grp == 0)
+              ag[k] += d;
+            else
+              au[k] += d;
+          }
+          release();
+        }
+      }
+    }
+    if (tr) tr[6] = globaltimer();
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      v[k] = ag[k];
+      v[8 + k] = au[k];
+    }
+    const float tot = warp_reduce_multi<16>(v, lane);     // item lane / 2 of this warp
+    const float up = __shfl_xor_sync(0xffffffffu, tot, 16);  // item q + 8: the up line of neuron q
+    const int q = lane >> 1;
+    if ((lane & 1) == 0 && q < 8 && ((own >> q) & 1u)) {
+      const float scale = 1.f / sqrtf(ctl->xss / (float)K + p.eps);
+      const float gs = tot * scale, us = up * scale;
+      p.act[g.r0 + warp + 8 * q] = gs / (1.f + expf(-gs)) * us;
+    }
+    return true;
+  }
+
   // ---- GEMV, batch 1: row-stationary tiles ------------------------------------
   // Stage s holds chunks [s * ncs, ...) of every line of the instruction, each
   // line kB1Chunk bf16 weights (512 bytes); a stage holds at most 64 line
@@ -1061,6 +1193,7 @@ struct Consumer {
   template <bool NORM, bool GATED>
   __device__ __forceinline__ bool gemv_b1(const mk_instr& in, int op, int layer) {
     const Gemv g = gemv_geo(p, in, op, layer);
+    if (GATED && g.split) return gemv_b1_gu2(in, layer, g);
     const int H = p.H, K = g.K, lines = g.lines, R = g.r1 - g.r0, nch = g.nch, NCS = g.ncs;
     const float* src;
     const uint16_t* gain = nullptr;

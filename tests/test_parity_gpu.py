@@ -21,6 +21,7 @@ def test_tiny_all_steps():
     ({"ctx": 255, "steps": 3}, "random"),                  # new token crosses a chunk boundary
     ({"n_q_heads": 8, "n_kv_heads": 1}, "ones"),           # 8 query heads per KV head
     ({"n_q_heads": 2, "n_kv_heads": 2}, "ones"),           # MHA
+    ({"ffn_dim": 5920, "steps": 3}, "random"),             # > 32 neurons per SM: gate and up as two stage groups
 ])
 def test_tiny_variants(kw, gains):
     res = run_teacher_forced(fx.CONFIGS["tiny"].replace(**kw), steps=kw.get("steps", 4), gains=gains)
