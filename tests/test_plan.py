@@ -320,3 +320,27 @@ def test_moe_shape_limits():
                 base.replace(expert_ffn_dim=100), base.replace(n_experts=512), base.replace(batch=8, top_k=9, n_experts=16)):
         with pytest.raises(mk.MkError):
             mk.Plan(mk.model_desc(bad), 148)
+
+
+@pytest.mark.parametrize("name,n_sm", [("dense-8b", 148), ("dense-8b", 132), ("dense-0.6b", 148), ("tiny", 7)])
+def test_batch1_gemv_instructions_cover_each_sm_share_in_bounded_pieces(name, n_sm):
+    """Batch 1: each SM's rows of an op are one contiguous share, cut into instructions of at most 64
+    rows (gate/up: 64 neurons, streamed as a gate group and an up group once above 32), in order."""
+    cfg, p = plan_of(name, n_sm)
+    for op in (OP_QKV, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LMHEAD):
+        N = {OP_QKV: cfg.q_dim + 2 * cfg.n_kv_heads * cfg.head_dim, OP_OPROJ: cfg.hidden,
+             OP_GATEUP: cfg.ffn_dim, OP_DOWN: cfg.hidden, OP_LMHEAD: cfg.vocab}[op]
+        layer = cfg.n_layers if op == OP_LMHEAD else 0
+        covered = []
+        for s in range(n_sm):
+            rows = [(int(r[4]), int(r[5])) for r in p.sm_list(s) if p.op(r) == op and p.layer(r) == layer]
+            for (a0, b0), (a1, b1) in zip(rows, rows[1:]):
+                assert b0 == a1, (op, s)                      # contiguous, in order
+            assert all(0 < b - a <= 64 for a, b in rows), (op, s, rows)
+            covered += rows
+        covered.sort()
+        assert covered[0][0] == 0 and covered[-1][1] == N and all(b == a for (_, b), (a, _) in zip(covered, covered[1:]))
+    if name == "dense-8b" and n_sm == 148:
+        # 14336 neurons: two gate/up instructions of 48-49 neurons per SM
+        per_sm = [sum(1 for r in p.sm_list(s) if p.op(r) == OP_GATEUP and p.layer(r) == 0) for s in range(n_sm)]
+        assert set(per_sm) == {2}
