@@ -228,7 +228,7 @@ def check_routing(res, gpu, ref, cfg):
 
 
 def summary(res) -> dict:
-    """The figures a parity run is judged on (also written to MK_PARITY_LOG when that is set)."""
+    """The summary figures of a parity run (also written to MK_PARITY_LOG when that is set)."""
     out = {"config": res.get("config"), "kernel": res.get("kernel"), "paged": res.get("paged", False),
            "steps_x_seqs": len(res["top1_exact"]), "top1_exact": float(np.mean(res["top1_exact"])),
            "top1_tie": float(np.mean(res["top1"])), "top1_miss_gaps": res["top1_gaps"],
