@@ -54,3 +54,20 @@ def test_8b_step_bytes():
     cfg = fx.CONFIGS["dense-8b"]
     b = bench.weight_bytes_read(cfg) + bench.kv_bytes(cfg, fx.context_lengths(cfg))
     assert b == 15_009_857_536 + 537_001_984
+
+
+def test_traffic_is_reported_only_for_the_captured_kernel_source(tmp_path, monkeypatch):
+    """`roofline.traffic` comes from profiles/traffic.json only while that capture's kernel source hash is
+    the current one; every committed entry is a whole-workload figure scaled from its small case."""
+    import json
+    d = json.load(open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for name, e in d.items():
+        assert name in fx.CONFIGS
+        ratio = e["traffic_over_algorithmic"]
+        assert 1.0 <= ratio < 1.05, name                          # no re-reads beyond whole attention stages
+        assert abs(e["dram_bytes_per_launch"] - ratio * e["algorithmic_full"]) <= 1e-5 * e["algorithmic_full"]  # ratio kept to 5 digits
+        assert e["algorithmic_small"] < e["algorithmic_full"]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "not-the-captured-source")
+    assert bench.ncu_traffic("dense-8b") is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: d["dense-8b"]["kernel_source"])
+    assert bench.ncu_traffic("dense-8b") == d["dense-8b"]["dram_bytes_per_launch"]
